@@ -1,0 +1,216 @@
+"""ctypes wrapper of the CPU oracle (``oracle/oracle.cpp``).
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline leg may import this module. The CUDA product path never does.
+
+All 16-bit tensors are numpy ``uint16`` bit patterns (bf16 or fp16, per ``dtype``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+LIB_PATH = os.path.join(_HERE, "liboracle.so")
+DTYPE_CODES = {"bf16": 0, "fp16": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (no FMA contraction, no fast-math)."""
+    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math",
+               "-fPIC", "-shared", _SRC, "-o", LIB_PATH + ".tmp"]
+        subprocess.check_call(cmd)
+        os.replace(LIB_PATH + ".tmp", LIB_PATH)
+    return LIB_PATH
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        # ORACLE_LIB lets the mutation tests load a deliberately broken copy.
+        path = os.environ.get("ORACLE_LIB") or build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        L.oracle_decode16.argtypes = [ctypes.c_uint16, i]
+        L.oracle_decode16.restype = ctypes.c_float
+        L.oracle_encode16.argtypes = [ctypes.c_float, i]
+        L.oracle_encode16.restype = ctypes.c_uint16
+        L.oracle_decode16_array.argtypes = [P, P, ctypes.c_long, i]
+        L.oracle_decode16_array.restype = None
+        L.oracle_encode16_array.argtypes = [P, P, ctypes.c_long, i]
+        L.oracle_encode16_array.restype = None
+        L.oracle_dispatch_layout.argtypes = [i, i, i, i, i, P, P, i, P, P, P]
+        L.oracle_dispatch_layout.restype = i
+        L.oracle_dispatch_permute.argtypes = [i, i, i, i, P, P, P]
+        L.oracle_dispatch_permute.restype = None
+        L.oracle_dispatch_permute_quant.argtypes = [i, i, i, i, i, P, P, P, P]
+        L.oracle_dispatch_permute_quant.restype = None
+        L.oracle_combine_fwd.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, i,
+                                         P, P, P, P, P, P]
+        L.oracle_combine_fwd.restype = None
+        L.oracle_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, i, P, P, P]
+        L.oracle_combine_bwd.restype = None
+        L.oracle_dispatch_bwd.argtypes = [i, i, i, i, i, P, P, P, i, P]
+        L.oracle_dispatch_bwd.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dt):
+    return None if a is None else np.ascontiguousarray(a, dtype=dt)
+
+
+def decode16(bits: int, dtype: str) -> float:
+    return lib().oracle_decode16(int(bits), DTYPE_CODES[dtype])
+
+
+def encode16(f: float, dtype: str) -> int:
+    return int(lib().oracle_encode16(float(f), DTYPE_CODES[dtype]))
+
+
+def decode16_array(bits, dtype: str) -> np.ndarray:
+    b = _c(bits, np.uint16)
+    f = np.empty(b.shape, np.float32)
+    lib().oracle_decode16_array(_p(b), _p(f), b.size, DTYPE_CODES[dtype])
+    return f
+
+
+def encode16_array(f, dtype: str) -> np.ndarray:
+    a = _c(f, np.float32)
+    b = np.empty(a.shape, np.uint16)
+    lib().oracle_encode16_array(_p(a), _p(b), a.size, DTYPE_CODES[dtype])
+    return b
+
+
+def assist_elems(bs: int, k: int, a_capacity: int) -> int:
+    return a_capacity + bs * k
+
+
+def dispatch_layout(topk_idx, num_experts, n_ids, a_capacity, mask=None):
+    """Returns (expert_token_nums (E,), ep_send_counts (E+1,), assist_info, status)."""
+    idx = _c(topk_idx, np.int32)
+    bs, k = idx.shape
+    m = _c(mask, np.uint8)
+    mask_ndim = 0 if m is None else m.ndim
+    counts = np.zeros(num_experts, np.int32)
+    send = np.zeros(num_experts + 1, np.int32)
+    assist = np.zeros(assist_elems(bs, k, a_capacity), np.int32)
+    st = lib().oracle_dispatch_layout(bs, k, num_experts, n_ids, a_capacity, _p(idx), _p(m),
+                                      mask_ndim, _p(counts), _p(send), _p(assist))
+    return counts, send, assist, int(st)
+
+
+def dispatch_permute(x, assist_info, k, a_capacity):
+    x = _c(x, np.uint16)
+    bs, h = x.shape
+    out = np.zeros((a_capacity, h), np.uint16)
+    lib().oracle_dispatch_permute(bs, k, h, a_capacity, _p(x), _p(_c(assist_info, np.int32)),
+                                  _p(out))
+    return out
+
+
+def dispatch_permute_quant(x, assist_info, k, a_capacity, dtype):
+    x = _c(x, np.uint16)
+    bs, h = x.shape
+    q = np.zeros((a_capacity, h), np.int8)
+    sc = np.zeros(a_capacity, np.float32)
+    lib().oracle_dispatch_permute_quant(bs, k, h, a_capacity, DTYPE_CODES[dtype], _p(x),
+                                        _p(_c(assist_info, np.int32)), _p(q), _p(sc))
+    return q, sc
+
+
+def combine_fwd(expand_x, topk_idx, topk_weights, assist_info, *, num_experts, a_capacity,
+                dtype, zero_expert_num=0, copy_expert_num=0, const_expert_num=0,
+                mask=None, shared=None, ori_x=None, alpha1=None, alpha2=None, const_v=None):
+    idx = _c(topk_idx, np.int32)
+    bs, k = idx.shape
+    ex = _c(expand_x, np.uint16)
+    h = ex.shape[1]
+    m = _c(mask, np.uint8)
+    out = np.zeros((bs, h), np.uint16)
+    args = [_c(shared, np.uint16), _c(ori_x, np.uint16), _c(alpha1, np.uint16),
+            _c(alpha2, np.uint16), _c(const_v, np.uint16)]
+    lib().oracle_combine_fwd(bs, k, h, num_experts, zero_expert_num, copy_expert_num,
+                             const_expert_num, a_capacity, DTYPE_CODES[dtype], _p(ex), _p(idx),
+                             _p(_c(topk_weights, np.float32)), _p(_c(assist_info, np.int32)),
+                             _p(m), 0 if m is None else m.ndim, *[_p(a) for a in args], _p(out))
+    return out
+
+
+def combine_bwd(grad_out, expand_x, topk_weights, assist_info, *, k, a_capacity, dtype,
+                mask=None):
+    """Returns (grad_expand (A, H), grad_w (BS, K) f32, abs_sum (BS, K) f64).
+
+    Rows of grad_expand without a slot are left zero.
+    """
+    g = _c(grad_out, np.uint16)
+    bs, h = g.shape
+    ex = _c(expand_x, np.uint16)
+    m = _c(mask, np.uint8)
+    ge = np.zeros((a_capacity, h), np.uint16)
+    gw = np.zeros((bs, k), np.float32)
+    mag = np.zeros((bs, k), np.float64)
+    lib().oracle_combine_bwd(bs, k, h, a_capacity, DTYPE_CODES[dtype], _p(g), _p(ex),
+                             _p(_c(topk_weights, np.float32)), _p(_c(assist_info, np.int32)),
+                             _p(m), 0 if m is None else m.ndim, _p(ge), _p(gw), _p(mag))
+    return ge, gw, mag
+
+
+def dispatch_bwd(grad_in, assist_info, *, bs, k, a_capacity, dtype, mask=None):
+    gi = _c(grad_in, np.uint16)
+    h = gi.shape[1]
+    m = _c(mask, np.uint8)
+    gx = np.zeros((bs, h), np.uint16)
+    lib().oracle_dispatch_bwd(bs, k, h, a_capacity, DTYPE_CODES[dtype], _p(gi),
+                              _p(_c(assist_info, np.int32)), _p(m), 0 if m is None else m.ndim,
+                              _p(gx))
+    return gx
+
+
+def run_chain(inputs: dict):
+    """The whole path on one workload: layout -> permute -> expert stand-in ->
+    combine fwd (-> combine bwd -> expert stand-in bwd -> dispatch bwd).
+
+    Returns a dict of every intermediate and output.
+    """
+    import workloads
+
+    wl = inputs["workload"]
+    r: dict = {}
+    r["counts"], r["send"], r["assist"], r["status"] = dispatch_layout(
+        inputs["topk_idx"], wl.num_experts, wl.n_ids, wl.a_capacity, inputs["mask"])
+    if wl.quant_mode == 2:
+        r["expand_q"], r["scales"] = dispatch_permute_quant(
+            inputs["x"], r["assist"], wl.k, wl.a_capacity, wl.dtype)
+        r["y"] = workloads.expert_forward(inputs, r["expand_q"], r["scales"])
+    else:
+        r["expand_x"] = dispatch_permute(inputs["x"], r["assist"], wl.k, wl.a_capacity)
+        r["y"] = workloads.expert_forward(inputs, r["expand_x"])
+    r["out"] = combine_fwd(
+        r["y"], inputs["topk_idx"], inputs["topk_weights"], r["assist"],
+        num_experts=wl.num_experts, a_capacity=wl.a_capacity, dtype=wl.dtype,
+        zero_expert_num=wl.zero_expert_num, copy_expert_num=wl.copy_expert_num,
+        const_expert_num=wl.const_expert_num, mask=inputs["mask"], shared=inputs["shared"],
+        ori_x=inputs["ori_x"], alpha1=inputs["alpha1"], alpha2=inputs["alpha2"],
+        const_v=inputs["v"])
+    if wl.backward:
+        r["grad_expand"], r["grad_w"], r["abs_sum"] = combine_bwd(
+            inputs["grad_out"], r["y"], inputs["topk_weights"], r["assist"], k=wl.k,
+            a_capacity=wl.a_capacity, dtype=wl.dtype, mask=inputs["mask"])
+        r["grad_in"] = workloads.expert_backward(inputs, r["grad_expand"])
+        r["grad_x"] = dispatch_bwd(r["grad_in"], r["assist"], bs=wl.bs, k=wl.k,
+                                   a_capacity=wl.a_capacity, dtype=wl.dtype, mask=inputs["mask"])
+    return r
