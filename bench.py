@@ -1,0 +1,499 @@
+"""Benchmark of the MoE dispatch + combine forward + backward path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  moe_dispatch_layout -> moe_dispatch_permute -> moe_combine_fwd -> moe_combine_bwd
+  -> moe_dispatch_bwd
+(forward-only workloads stop after moe_combine_fwd). The experts between dispatch and
+combine are outside the path: their outputs (and input gradients) are computed once,
+untimed, and stay resident in HBM like every other input.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
+
+Prints one JSON line (rank 0). Multi-GPU runs are independent replicas (one process
+per GPU, launched with torch.distributed.run); only the barrier and the max-over-ranks
+timing use the process group.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "dispatch+combine fwd+bwd tokens/s and achieved HBM GB/s (% of 8 TB/s), 1×B200"
+DEFAULT_WORKLOAD = "uniform_bs8192_h1536_k8_e64"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNELS = ("layout", "permute", "combine_fwd", "combine_bwd", "dispatch_bwd")
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic bytes per launch (each tensor counted once).
+
+def byte_model(wl: workloads.Workload, r: int, ori_tokens: int) -> dict:
+    bs, k, h, e = wl.bs, wl.k, wl.h, wl.elem_bytes
+    row, pairs = h * e, bs * k
+    mask = 0 if wl.mask_ndim == 0 else (bs if wl.mask_ndim == 1 else pairs)
+    slot_map = 4 * pairs
+    m = {}
+    m["layout"] = 4 * pairs + mask + 4 * (wl.a_capacity + pairs) + 4 * (2 * wl.num_experts + 1)
+    if wl.quant_mode == 2:
+        m["permute"] = bs * row + slot_map + r * h + 4 * r
+    else:
+        m["permute"] = bs * row + slot_map + r * row
+    special = wl.zero_expert_num + wl.copy_expert_num + wl.const_expert_num
+    m["combine_fwd"] = (r * row + 4 * pairs + slot_map + (4 * pairs if special else 0) + mask
+                        + (bs * row if wl.shared else 0) + ori_tokens * row
+                        + 3 * wl.const_expert_num * row + bs * row)
+    if wl.backward:
+        m["combine_bwd"] = bs * row + 2 * r * row + 4 * pairs + slot_map + 4 * pairs + mask
+        m["dispatch_bwd"] = r * row + bs * row + slot_map + mask
+    return m
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region.
+
+class ClockSampler:
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = (uuid or "").lower()
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        exe = shutil.which("nvidia-smi")
+        if exe is None:
+            return
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        self.f = open(self.path, "w")
+        self.proc = subprocess.Popen([exe, f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits", "-lms", "20"],
+                                     stdout=self.f, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self, t0: float, t1: float) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            p = [c.strip() for c in line.split(",")]
+            if len(p) < 10:
+                continue
+            if self.uuid and self.uuid not in p[1].lower():
+                continue
+            try:
+                ts = _dt.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(p[2]), float(p[3]), p[6:10]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.02 <= r[0] <= t1 + 0.02]
+        window = "timed region"
+        if not inside:  # timed region shorter than the sampling period
+            inside = [r for r in rows if r[0] <= t1 + 0.1][-3:]
+            window = "samples nearest the timed region"
+        if not inside:
+            return None
+        reasons = sorted({self.REASONS[i] for r in inside for i, v in enumerate(r[3])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------------------
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_moe_dispatch_04_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def oracle_chain_timed(inputs: dict, sample_tokens: int) -> tuple[float, int]:
+    """Times the oracle's five calls on the first `sample_tokens` tokens of the
+    workload (expert stand-ins excluded). Returns (seconds, tokens)."""
+    import oracle
+
+    wl = inputs["workload"]
+    n = min(sample_tokens, wl.bs)
+    sub = wl.scaled(bs=n, a_capacity_override=0)
+    inp = dict(inputs)
+    inp["workload"] = sub
+    for key in ("topk_idx", "topk_weights", "x", "mask", "shared", "grad_out"):
+        if inp.get(key) is not None:
+            inp[key] = np.ascontiguousarray(inp[key][:n])
+    inp["ori_x"] = inp["x"] if inputs.get("ori_x") is not None else None
+    if inp.get("expert_factor") is not None:
+        inp["expert_factor"] = np.ascontiguousarray(inp["expert_factor"][:sub.a_capacity])
+    secs = 0.0
+    t = time.perf_counter()
+    counts, send, assist, _ = oracle.dispatch_layout(inp["topk_idx"], sub.num_experts, sub.n_ids,
+                                                     sub.a_capacity, inp["mask"])
+    if sub.quant_mode == 2:
+        q, sc = oracle.dispatch_permute_quant(inp["x"], assist, sub.k, sub.a_capacity, sub.dtype)
+        secs += time.perf_counter() - t
+        y = workloads.expert_forward(inp, q, sc)
+    else:
+        ex = oracle.dispatch_permute(inp["x"], assist, sub.k, sub.a_capacity)
+        secs += time.perf_counter() - t
+        y = workloads.expert_forward(inp, ex)
+    t = time.perf_counter()
+    oracle.combine_fwd(y, inp["topk_idx"], inp["topk_weights"], assist,
+                       num_experts=sub.num_experts, a_capacity=sub.a_capacity, dtype=sub.dtype,
+                       zero_expert_num=sub.zero_expert_num, copy_expert_num=sub.copy_expert_num,
+                       const_expert_num=sub.const_expert_num, mask=inp["mask"],
+                       shared=inp["shared"], ori_x=inp["ori_x"], alpha1=inp["alpha1"],
+                       alpha2=inp["alpha2"], const_v=inp["v"])
+    if sub.backward:
+        ge, _, _ = oracle.combine_bwd(inp["grad_out"], y, inp["topk_weights"], assist, k=sub.k,
+                                      a_capacity=sub.a_capacity, dtype=sub.dtype, mask=inp["mask"])
+        oracle.dispatch_bwd(ge, assist, bs=sub.bs, k=sub.k, a_capacity=sub.a_capacity,
+                            dtype=sub.dtype, mask=inp["mask"])
+    secs += time.perf_counter() - t
+    return secs, n
+
+
+def cpu_baseline(inputs: dict, budget_s: float = 10.0) -> dict:
+    wl = inputs["workload"]
+    sample = min(wl.bs, 2048)
+    total_s, total_tok, passes = 0.0, 0, 0
+    while total_s < budget_s and passes < 50:
+        s, n = oracle_chain_timed(inputs, sample)
+        total_s += s
+        total_tok += n
+        passes += 1
+    return {"value": total_tok / total_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{passes} passes of the first {sample} tokens of {wl.name} through the "
+                      f"single-threaded C++ oracle (layout, permute, combine fwd"
+                      f"{', combine bwd, dispatch bwd' if wl.backward else ''}); "
+                      f"{total_s:.1f} s of CPU time"}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inputs = workloads.generate(wl)
+    sample = min(wl.bs, 512)
+    for _ in range(args.warmup):
+        oracle_chain_timed(inputs, sample)
+    total_s, total_tok = 0.0, 0
+    for _ in range(args.steps):
+        s, n = oracle_chain_timed(inputs, sample)
+        total_s += s
+        total_tok += n
+    value = total_tok / total_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "bs": wl.bs, "h": wl.h, "k": wl.k,
+                       "num_experts": wl.num_experts, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: the first {sample} tokens of {wl.name} "
+                                       "through the single-threaded C++ oracle"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="moe", choices=["moe", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    wl = workloads.BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    import torch
+    import torch.distributed as dist
+
+    import combine_moe_dispatch_04_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    inputs = workloads.generate(wl, seed=wl.seed + 1000 * rank)
+    dt = wl.dtype
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float16
+
+    def up(a):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(tdt)
+        return torch.from_numpy(a).to(dev)
+
+    def down16(t):
+        return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+    sh = moe.Shape(bs=wl.bs, k=wl.k, h=wl.h, num_experts=wl.num_experts,
+                   zero_expert_num=wl.zero_expert_num, copy_expert_num=wl.copy_expert_num,
+                   const_expert_num=wl.const_expert_num, a_capacity=wl.a_capacity,
+                   dtype=workloads.DTYPE_CODES[dt], mask_ndim=wl.mask_ndim)
+    d = {k: up(inputs[k]) for k in ("topk_idx", "topk_weights", "x", "mask", "shared", "ori_x",
+                                     "alpha1", "alpha2", "v", "grad_out")}
+    ws = moe.layout_workspace(sh, dev)
+    lay = moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws)
+    qm = wl.quant_mode
+    expand, scales = moe.dispatch_permute(sh, d["x"], lay, qm)
+    torch.cuda.synchronize()
+    r = int(lay.ep_send_counts[-1].item())
+    # untimed expert stand-ins, computed once on the host from the GPU's dispatch output
+    if qm == 2:
+        y_host = workloads.expert_forward(inputs, expand.cpu().numpy(), scales.cpu().numpy())
+    else:
+        y_host = workloads.expert_forward(inputs, down16(expand))
+    y = up(y_host)
+    out = moe.combine_fwd(sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
+                          shared_expert_x=d["shared"], ori_x=d["ori_x"],
+                          const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
+                          const_v=d["v"])
+    if wl.backward:
+        gexp, gw = moe.combine_bwd(sh, d["grad_out"], y, d["topk_weights"], lay,
+                                   x_active_mask=d["mask"])
+        torch.cuda.synchronize()
+        gin = up(workloads.expert_backward(inputs, down16(gexp)))
+        gx = moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"])
+    torch.cuda.synchronize()
+
+    ori_tokens = 0
+    if wl.copy_expert_num + wl.const_expert_num:
+        ids = inputs["topk_idx"]
+        lo = wl.num_experts + wl.zero_expert_num
+        ori_tokens = int(np.any(ids >= lo, axis=1).sum())
+    bytes_per = byte_model(wl, r, ori_tokens)
+    kernels = [k for k in KERNELS if k in bytes_per]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws, out=lay, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand, dynamic_scales=scales,
+                             stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        moe.combine_fwd(sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
+                        shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
+                        const_alpha_2=d["alpha2"], const_v=d["v"], out=out, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        if wl.backward:
+            moe.combine_bwd(sh, d["grad_out"], y, d["topk_weights"], lay,
+                            x_active_mask=d["mask"], grad_expand=gexp, grad_w=gw, stream=stream)
+            if ev is not None:
+                ev[4].record(stream)
+            moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"], grad_x=gx, stream=stream)
+            if ev is not None:
+                ev[5].record(stream)
+
+    layout_launches = 1 if wl.bs <= 1024 else 3
+    launches_per_step = layout_launches + 2 + (2 if wl.backward else 0)
+
+    # L2 flush between steps: write a buffer twice the size of L2
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
+    flush = torch.empty(2 * l2 // 4, dtype=torch.int32, device=dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    n_ev = len(kernels) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid if rank == 0 else None)
+    if rank == 0:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1) if rank == 0 else None
+
+    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
+    per_kernel_ms = {k: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]
+                     for j, k in enumerate(kernels)}
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    tokens = wl.bs * args.steps * world
+    value = tokens / (total_ms * 1e-3)
+    bytes_step = sum(bytes_per.values())
+
+    # e2e: pinned host inputs -> H2D -> the path through the C ABI -> D2H of the results
+    e2e = None
+    if not args.no_e2e:
+        in_keys = [k for k in ("topk_idx", "topk_weights", "x", "mask", "shared", "grad_out")
+                   if d[k] is not None]
+        h_in = {k: d[k].cpu().pin_memory() for k in in_keys}
+        outs = [out] + ([gx, gw] if wl.backward else [])
+        h_out = [o.cpu().pin_memory() for o in outs]
+        bi = sum(t.numel() * t.element_size() for t in h_in.values())
+        bo = sum(t.numel() * t.element_size() for t in h_out)
+        e2e_steps = max(3, args.steps // 4)
+
+        def e2e_step():
+            for k in in_keys:
+                d[k].copy_(h_in[k], non_blocking=True)
+            step()
+            for o, ho in zip(outs, h_out):
+                ho.copy_(o, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        ea.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        e_ms = ea.elapsed_time(eb)
+        if world > 1:
+            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": wl.bs * e2e_steps * world / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps}
+
+    if rank == 0:
+        peak, peak_kind = measured_hbm_peak()
+        kstats = {}
+        for k in kernels:
+            us = 1e3 * statistics.fmean(per_kernel_ms[k])
+            kstats[k] = {"us": round(us, 3), "bytes": bytes_per[k],
+                         "gbs": round(bytes_per[k] / (us * 1e-6) / 1e9, 1)}
+        dom = max(kernels, key=lambda k: kstats[k]["us"])
+        ach = kstats[dom]["gbs"]
+        gbs = bytes_step / (ms_per_step * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dt,
+            "data": "synthetic",
+            "config": {"workload": wl.name, "bs": wl.bs, "h": wl.h, "k": wl.k,
+                       "num_experts": wl.num_experts, "routed_pairs": r,
+                       "a_capacity": wl.a_capacity, "parallelism": "replicas",
+                       "l2": "flushed before every step (write of 2x L2), outside the step events"},
+            "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+            "hbm_frac_of_measured": round(gbs / peak, 4),
+            "algorithmic_bytes_per_step": bytes_step,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
+                         "traffic": profiled_traffic(dom, wl.name),
+                         "algorithmic_bytes": bytes_per[dom]},
+            "kernels": kstats,
+            "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e,
+            "clocks": clocks,
+            "step_ms_stats": {"mean": statistics.fmean(step_ms),
+                              "median": statistics.median(step_ms),
+                              "trimmed_mean_drop_top3": statistics.fmean(
+                                  sorted(step_ms)[:-3] if len(step_ms) > 6 else step_ms),
+                              "std": statistics.pstdev(step_ms)},
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(inputs)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

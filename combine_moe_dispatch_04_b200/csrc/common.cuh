@@ -1,0 +1,87 @@
+// Shared device helpers of the dispatch/combine kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_dc.h"
+
+namespace moe {
+
+constexpr int kMaxK = 16;
+constexpr int kVecElems = 8;  // 16-bit values per 16-byte vector
+
+// ---- 16-bit float traits: exact widening, round-to-nearest-even narrowing ----
+
+struct Bf16 {
+  static __device__ __forceinline__ float2 widen2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+  }
+  static __device__ __forceinline__ uint32_t narrow2(float lo, float hi) {
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+};
+
+struct Fp16 {
+  static __device__ __forceinline__ float2 widen2(uint32_t u) {
+    __half2 h = *reinterpret_cast<__half2*>(&u);
+    return __half22float2(h);
+  }
+  static __device__ __forceinline__ uint32_t narrow2(float lo, float hi) {
+    __half2 r = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ void widen8(const uint4& v, float (&f)[8]) {
+  float2 a = T::widen2(v.x), b = T::widen2(v.y), c = T::widen2(v.z), d = T::widen2(v.w);
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+  f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 narrow8(const float (&f)[8]) {
+  uint4 v;
+  v.x = T::narrow2(f[0], f[1]);
+  v.y = T::narrow2(f[2], f[3]);
+  v.z = T::narrow2(f[4], f[5]);
+  v.w = T::narrow2(f[6], f[7]);
+  return v;
+}
+
+// ---- global memory access ----
+
+// Read-only 16-byte load through the non-coherent path, not kept in L1.
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st_v4(void* p, const uint4& v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Whether pair (t, k) is active under x_active_mask (1-D per token, 2-D per pair).
+__device__ __forceinline__ bool pair_active(const uint8_t* mask, int mask_ndim, int t, int k,
+                                            int K) {
+  if (mask_ndim == 0) return true;
+  if (mask_ndim == 1) return __ldg(mask + t) != 0;
+  return __ldg(mask + static_cast<size_t>(t) * K + k) != 0;
+}
+
+}  // namespace moe

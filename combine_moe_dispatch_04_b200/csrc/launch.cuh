@@ -1,0 +1,70 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct LayoutArgs {
+  const int32_t* topk_idx;
+  const uint8_t* mask;
+  int mask_ndim;
+  int bs, K, E, N, A;
+  int32_t* expert_token_nums;
+  int32_t* ep_send_counts;
+  int32_t* assist;
+  uint32_t* dev_status;  // may be null
+  void* workspace;
+};
+
+// Tokens per CTA in the multi-CTA layout, and the largest BS of the one-CTA layout.
+constexpr int kLayoutTileTokens = 128;
+constexpr int kLayoutSmallMaxTokens = 1024;
+
+size_t layout_workspace_bytes(int bs, int E);
+cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st);
+
+struct PermuteArgs {
+  const void* x;
+  const int32_t* assist;
+  void* expand_x;
+  float* scales;
+  int bs, K, H, A, dtype, quant_mode;
+};
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
+
+struct CombineArgs {
+  const void* expand_x;  // (A, H): expert outputs, or slot gradients for dispatch bwd
+  const int32_t* topk_idx;
+  const float* weights;  // null: unit weights (dispatch backward)
+  const int32_t* assist;
+  const uint8_t* mask;
+  int mask_ndim;
+  const void* shared;
+  const void* ori_x;
+  const void* alpha1;
+  const void* alpha2;
+  const void* const_v;
+  void* out;
+  int bs, K, H, A, E, Z, C, Q, dtype;
+};
+cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st);
+
+struct CombineBwdArgs {
+  const void* grad_out;
+  const void* expand_x;
+  const float* weights;
+  const int32_t* assist;
+  const uint8_t* mask;
+  int mask_ndim;
+  void* grad_expand;
+  float* grad_w;
+  int bs, K, H, A, dtype;
+};
+cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st);
+
+int sm_count();
+
+}  // namespace moe

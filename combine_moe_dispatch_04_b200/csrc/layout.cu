@@ -1,0 +1,311 @@
+// Dispatch layout: per-expert histogram, exclusive prefix sum (ep_send_counts)
+// and the two slot maps of assist_info. [combine] Parameters
+// (assist_info_for_combine, ep_send_counts, x_active_mask).
+//
+// The order is a stable counting sort on the key (expert, token, k). Because a
+// valid row never repeats an id, a token holds at most one pair per expert,
+// and a pair's rank inside its expert's segment is the number of earlier
+// tokens routed to that expert. Each warp builds, per expert, a 32-bit mask of
+// its lanes (tokens) that route there (shared-memory atomicOr); popcounts of
+// those masks give counts and ranks with no ordering race, so the result is
+// deterministic.
+//
+//   BS <= 1024: one CTA of 32 warps does everything (one launch).
+//   otherwise : count (one CTA per 128-token tile) -> scan (one CTA) ->
+//               scatter (one CTA per tile); the per-(tile, expert) counts live
+//               in the caller's workspace.
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+// Classifies the K pairs of token t: e[k] = expert id of a routed active
+// pair, else -1. Returns the MOE_DEV_* bits of the row.
+__device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int (&e)[kMaxK]) {
+  const int32_t* row = a.topk_idx + static_cast<size_t>(t) * a.K;
+  int ids[kMaxK];
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) ids[k] = k < a.K ? __ldg(row + k) : -1;
+  uint32_t st = 0;
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) {
+    e[k] = -1;
+    if (k >= a.K) continue;
+    const int id = ids[k];
+    if (id < 0 || id >= a.N) {
+      st |= MOE_DEV_BAD_ID;
+      continue;
+    }
+    bool dup = false;
+#pragma unroll
+    for (int j = 0; j < k; ++j) dup |= ids[j] == id;
+    if (dup) {
+      st |= MOE_DEV_DUP_ID;
+      continue;
+    }
+    if (id < a.E && pair_active(a.mask, a.mask_ndim, t, k, a.K)) e[k] = id;
+  }
+  return st;
+}
+
+// words[warp * E + e] |= bit of this lane, for each routed pair of the lane.
+__device__ __forceinline__ void mark_words(uint32_t* words, int E, const int (&e)[kMaxK], int K) {
+  const int warp = threadIdx.x >> 5;
+  const uint32_t bit = 1u << (threadIdx.x & 31);
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k)
+    if (k < K && e[k] >= 0) atomicOr(&words[warp * E + e[k]], bit);
+}
+
+// Rank of this lane's token among the tile's tokens routed to expert ex.
+__device__ __forceinline__ int tile_rank(const uint32_t* words, int E, int ex) {
+  const int warp = threadIdx.x >> 5;
+  int r = __popc(words[warp * E + ex] & lanemask_lt());
+  for (int w = 0; w < warp; ++w) r += __popc(words[w * E + ex]);
+  return r;
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x <= 1024).
+// Returns the exclusive prefix; *total receives the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  int inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int n = __shfl_up_sync(0xFFFFFFFFu, inc, d);
+    if (lane >= d) inc += n;
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nwarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int n = __shfl_up_sync(0xFFFFFFFFu, s, d);
+      if (lane >= d) s += n;
+    }
+    if (lane < nwarps) warp_sums[lane] = s;  // inclusive warp prefix
+  }
+  __syncthreads();
+  const int before = warp == 0 ? 0 : warp_sums[warp - 1];
+  *total = warp_sums[nwarps - 1];
+  return before + inc - v;
+}
+
+// Writes both halves of assist_info for token t's pairs given their slots.
+__device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const int (&e)[kMaxK],
+                                            const int (&slot)[kMaxK]) {
+  const size_t A = static_cast<size_t>(a.A);
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) {
+    if (k >= a.K) continue;
+    const int tk = t * a.K + k;
+    if (e[k] >= 0) a.assist[slot[k]] = tk;
+    a.assist[A + tk] = e[k] >= 0 ? slot[k] : -1;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// One-CTA layout for BS <= 1024: 32 warps, one token per thread.
+// Dynamic shared memory: words[32][E].
+__global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
+  extern __shared__ uint32_t words[];
+  __shared__ int offs[1024];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t status;
+  const int E = a.E;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) words[i] = 0;
+  if (threadIdx.x == 0) status = 0;
+  __syncthreads();
+
+  const int t = threadIdx.x;
+  int e[kMaxK];
+  uint32_t st = 0;
+  if (t < a.bs) {
+    st = classify_row(a, t, e);
+    mark_words(words, E, e, a.K);
+  } else {
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) e[k] = -1;
+  }
+  if (st) atomicOr(&status, st);
+  __syncthreads();
+
+  int cnt = 0;
+  if (threadIdx.x < E)
+    for (int w = 0; w < 32; ++w) cnt += __popc(words[w * E + threadIdx.x]);
+  int total;
+  const int excl = block_exclusive_scan(cnt, warp_sums, &total);
+  if (threadIdx.x < E) {
+    offs[threadIdx.x] = excl;
+    a.expert_token_nums[threadIdx.x] = cnt;
+    a.ep_send_counts[threadIdx.x] = excl;
+  }
+  if (threadIdx.x == 0) a.ep_send_counts[E] = total;
+  __syncthreads();
+
+  if (t < a.bs) {
+    int slot[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k)
+      slot[k] = (k < a.K && e[k] >= 0) ? offs[e[k]] + tile_rank(words, E, e[k]) : -1;
+    write_slots(a, t, e, slot);
+  }
+  for (int s = total + threadIdx.x; s < a.A; s += blockDim.x) a.assist[s] = -1;
+  if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
+}
+
+// ---------------------------------------------------------------------------
+// Multi-CTA layout. Workspace: tile_counts[T][E] int32, then tile_status[T].
+
+struct TileWs {
+  int32_t* counts;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ TileWs tile_ws(const LayoutArgs& a, int T) {
+  TileWs w;
+  w.counts = static_cast<int32_t*>(a.workspace);
+  w.status = reinterpret_cast<uint32_t*>(w.counts + static_cast<size_t>(T) * a.E);
+  return w;
+}
+
+constexpr int kTileWarps = kLayoutTileTokens / 32;
+
+// Phase 1: per-tile expert counts and status bits.
+__global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutArgs a, int T) {
+  extern __shared__ uint32_t words[];  // [kTileWarps][E]
+  __shared__ uint32_t status;
+  const int E = a.E;
+  for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
+  if (threadIdx.x == 0) status = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
+  if (t < a.bs) {
+    int e[kMaxK];
+    const uint32_t st = classify_row(a, t, e);
+    mark_words(words, E, e, a.K);
+    if (st) atomicOr(&status, st);
+  }
+  __syncthreads();
+  TileWs ws = tile_ws(a, T);
+  for (int ex = threadIdx.x; ex < E; ex += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kTileWarps; ++w) c += __popc(words[w * E + ex]);
+    ws.counts[static_cast<size_t>(blockIdx.x) * E + ex] = c;
+  }
+  if (threadIdx.x == 0) ws.status[blockIdx.x] = status;
+}
+
+// Phase 2 (one CTA of 1024 threads): expert totals, their exclusive scan, and
+// the first slot of every (tile, expert) written back over the counts.
+__global__ void __launch_bounds__(1024) layout_scan_kernel(LayoutArgs a, int T) {
+  __shared__ int part[1024];  // [G][E], partial sums of tile groups
+  __shared__ int offs[1024];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t status;
+  const int E = a.E;
+  TileWs ws = tile_ws(a, T);
+  const int G = max(1, min(1024 / E, T));
+  const int chunk = (T + G - 1) / G;
+  const int ex = threadIdx.x % E, g = threadIdx.x / E;
+  const bool grp = g < G;
+  const int t0 = g * chunk, t1 = min(T, t0 + chunk);
+  if (threadIdx.x == 0) status = 0;
+  __syncthreads();
+  if (grp) {
+    int s = 0;
+    for (int tile = t0; tile < t1; ++tile) s += ws.counts[static_cast<size_t>(tile) * E + ex];
+    part[g * E + ex] = s;
+  }
+  uint32_t st = 0;
+  for (int tile = threadIdx.x; tile < T; tile += blockDim.x) st |= ws.status[tile];
+  if (st) atomicOr(&status, st);
+  __syncthreads();
+  int cnt = 0;
+  if (threadIdx.x < E) {
+    for (int gg = 0; gg < G; ++gg) {
+      const int v = part[gg * E + threadIdx.x];
+      part[gg * E + threadIdx.x] = cnt;
+      cnt += v;
+    }
+  }
+  int total;
+  const int excl = block_exclusive_scan(cnt, warp_sums, &total);
+  if (threadIdx.x < E) {
+    offs[threadIdx.x] = excl;
+    a.expert_token_nums[threadIdx.x] = cnt;
+    a.ep_send_counts[threadIdx.x] = excl;
+  }
+  if (threadIdx.x == 0) a.ep_send_counts[E] = total;
+  __syncthreads();
+  if (grp) {
+    int run = offs[ex] + part[g * E + ex];
+    for (int tile = t0; tile < t1; ++tile) {
+      int* p = &ws.counts[static_cast<size_t>(tile) * E + ex];
+      const int c = *p;
+      *p = run;
+      run += c;
+    }
+  }
+  if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
+}
+
+// Phase 3: slots of every pair of the tile, and -1 for the unused slots [R, A).
+__global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
+  extern __shared__ uint32_t words[];  // [kTileWarps][E]
+  const int E = a.E;
+  for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
+  int e[kMaxK];
+  if (t < a.bs) {
+    classify_row(a, t, e);
+    mark_words(words, E, e, a.K);
+  }
+  __syncthreads();
+  if (t < a.bs) {
+    TileWs ws = tile_ws(a, T);
+    const int32_t* base = ws.counts + static_cast<size_t>(blockIdx.x) * E;
+    int slot[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k)
+      slot[k] = (k < a.K && e[k] >= 0) ? base[e[k]] + tile_rank(words, E, e[k]) : -1;
+    write_slots(a, t, e, slot);
+  }
+  const int total = a.ep_send_counts[E];
+  for (int s = total + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
+       s += gridDim.x * blockDim.x)
+    a.assist[s] = -1;
+}
+
+}  // namespace
+
+size_t layout_workspace_bytes(int bs, int E) {
+  if (bs <= kLayoutSmallMaxTokens) return 0;
+  const size_t T = (static_cast<size_t>(bs) + kLayoutTileTokens - 1) / kLayoutTileTokens;
+  return T * static_cast<size_t>(E) * 4 + T * 4;
+}
+
+cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st) {
+  if (a.bs <= kLayoutSmallMaxTokens) {
+    const size_t smem = 32u * a.E * sizeof(uint32_t);
+    cudaError_t err = cudaFuncSetAttribute(layout_small_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    layout_small_kernel<<<1, 1024, smem, st>>>(a);
+    return cudaGetLastError();
+  }
+  const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
+  const size_t smem = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
+  layout_count_kernel<<<T, kLayoutTileTokens, smem, st>>>(a, T);
+  layout_scan_kernel<<<1, 1024, 0, st>>>(a, T);
+  layout_scatter_kernel<<<T, kLayoutTileTokens, smem, st>>>(a, T);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

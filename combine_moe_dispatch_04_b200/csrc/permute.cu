@@ -1,0 +1,144 @@
+// Dispatch permute: expand_x[slot(t, k)] = x[t] for every pair with a slot,
+// optionally quantised to int8 per token ([combine] Parameters:
+// comm_quant_mode 2; Example: quant_mode = 2).
+//
+// Plain copy: one thread per 16-byte vector of x (coalesced along the row),
+// read once and stored to each of the token's K slots. The slot list of a
+// token is shared by the threads of its row and comes from L1.
+//
+// int8: one CTA per token (grid-stride); each thread keeps 16-element chunks
+// of the row in registers, the CTA reduces max|x|, and every chunk becomes one
+// 16-byte int8 store per slot.
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyItems = 2;  // vectors per thread
+
+__global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
+    int bs, int K, int V, int A) {
+  const int n = bs * V;
+  const int32_t* slots_all = assist + static_cast<size_t>(A);
+#pragma unroll
+  for (int i = 0; i < kCopyItems; ++i) {
+    const int item = (blockIdx.x * kCopyItems + i) * kCopyThreads + threadIdx.x;
+    if (item >= n) return;
+    const int t = item / V;
+    const int v = item - t * V;
+    const uint4 val = ld_nc_v4(x + item);
+    const int32_t* slots = slots_all + static_cast<size_t>(t) * K;
+    for (int k = 0; k < K; ++k) {
+      const int s = __ldg(slots + k);
+      if (s >= 0) st_v4(out + static_cast<size_t>(s) * V + v, val);
+    }
+  }
+}
+
+constexpr int kQuantChunksPerThread = 4;  // 16-element chunks per thread
+
+template <typename T16>
+__global__ void __launch_bounds__(256) permute_quant_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
+    float* __restrict__ scales, int bs, int K, int H, int A) {
+  __shared__ float warp_max[8];
+  const int C = H / 16;  // chunks per row
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  for (int t = blockIdx.x; t < bs; t += gridDim.x) {
+    const uint4* xr = x + static_cast<size_t>(t) * (H / 8);
+    float f[kQuantChunksPerThread][16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kQuantChunksPerThread; ++j) {
+      const int c = threadIdx.x + j * blockDim.x;
+      if (c < C) {
+        float lo[8], hi[8];
+        widen8<T16>(ld_nc_v4(xr + 2 * c), lo);
+        widen8<T16>(ld_nc_v4(xr + 2 * c + 1), hi);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          f[j][i] = lo[i];
+          f[j][8 + i] = hi[i];
+          amax = fmaxf(amax, fmaxf(fabsf(lo[i]), fabsf(hi[i])));
+        }
+      }
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+    if (lane == 0) warp_max[warp] = amax;
+    __syncthreads();
+    amax = warp_max[0];
+    for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, warp_max[w]);
+    __syncthreads();  // warp_max is reused by the next token
+    const float scale = __fdiv_rn(amax, 127.0f);
+    const int32_t* slots = assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K;
+#pragma unroll
+    for (int j = 0; j < kQuantChunksPerThread; ++j) {
+      const int c = threadIdx.x + j * blockDim.x;
+      if (c >= C) continue;
+      uint32_t packed[4];
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          int q = 0;
+          if (amax != 0.0f) {
+            float r = rintf(__fdiv_rn(f[j][w4 * 4 + b], scale));
+            r = fminf(127.0f, fmaxf(-127.0f, r));
+            q = __float2int_rn(r);
+          }
+          word |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * b);
+        }
+        packed[w4] = word;
+      }
+      const uint4 val = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      for (int k = 0; k < K; ++k) {
+        const int s = __ldg(slots + k);
+        if (s >= 0) st_v4(out + static_cast<size_t>(s) * C + c, val);
+      }
+    }
+    if (threadIdx.x < K) {
+      const int s = __ldg(slots + threadIdx.x);
+      if (s >= 0) scales[s] = scale;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
+  if (a.bs == 0) return cudaSuccess;
+  if (a.quant_mode == 0) {
+    const int V = a.H / kVecElems;
+    const long long n = static_cast<long long>(a.bs) * V;
+    const int per_block = kCopyThreads * kCopyItems;
+    const int blocks = static_cast<int>((n + per_block - 1) / per_block);
+    permute_copy_kernel<<<blocks, kCopyThreads, 0, st>>>(
+        static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x), a.bs, a.K, V,
+        a.A);
+    return cudaGetLastError();
+  }
+  // One chunk per thread up to 256 threads, then up to 4 chunks per thread
+  // (H <= 16384, checked by the caller).
+  const int C = a.H / 16;
+  int threads = (C + 31) / 32 * 32;
+  threads = threads > 256 ? 256 : threads;
+  const int cap = sm_count() * 16;
+  const int blocks = a.bs < cap ? a.bs : cap;
+  if (a.dtype == MOE_BF16)
+    permute_quant_kernel<Bf16><<<blocks, threads, 0, st>>>(
+        static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x), a.scales,
+        a.bs, a.K, a.H, a.A);
+  else
+    permute_quant_kernel<Fp16><<<blocks, threads, 0, st>>>(
+        static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x), a.scales,
+        a.bs, a.K, a.H, a.A);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,188 @@
+/*
+ * moe_dc.h — C ABI of the B200 (sm_100a) MoE token dispatch / combine library.
+ *
+ * One device, no collective: the expert-parallel alltoallv of the Ascend CANN
+ * "low_latency_combine" page (Function: Description and Formula) collapses to a
+ * local permute, and combine returns every row "along the same path".
+ *
+ * Conventions shared by every call below
+ * --------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller, dense and
+ *   row-major, 16-byte aligned where a row of 16-bit values is read or
+ *   written. The library allocates nothing and keeps no state between calls.
+ * - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *   stream. Work is enqueued asynchronously on it; nothing synchronises.
+ * - Host-side checks run first and return a status before anything is
+ *   launched: nothing is written when a call returns an error other than
+ *   MOE_ERR_CUDA.
+ * - Data errors found on the device (an id outside [0, N), an id repeated
+ *   within a row) never fault: the pair is ignored and a bit is set in the
+ *   layout's `dev_status` word.
+ * - Every call is deterministic: no floating-point atomics, a fixed k order
+ *   and fixed reduction trees ([combine] Deterministic Computation).
+ *
+ * Symbols: BS tokens, K experts per token, H hidden size, E routed experts,
+ * Z zero, C copy, Q const experts, N = E + Z + C + Q ids, A expanded-row
+ * capacity, R routed active pairs (R <= A).
+ */
+#ifndef MOE_DC_H
+#define MOE_DC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,          /* bad size, null pointer, bad mode */
+  MOE_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement */
+  MOE_ERR_ALIGN = 3,        /* H * 2 not a multiple of 16, or a misaligned pointer */
+  MOE_ERR_CAPACITY = 4,     /* a_capacity < BS * min(E, K), or workspace too small */
+  MOE_ERR_CUDA = 5          /* a CUDA launch failed; see moe_last_cuda_error() */
+} moe_status;
+
+typedef enum { MOE_BF16 = 0, MOE_FP16 = 1 } moe_dtype;
+
+/* Bits of the device status word written by moe_dispatch_layout. */
+#define MOE_DEV_BAD_ID 1u  /* some id outside [0, N) */
+#define MOE_DEV_DUP_ID 2u  /* some id repeated within a row; later copies ignored */
+
+/*
+ * Problem shape. [combine] Parameters table and Constraints:
+ *   bs               tokens (BS >= 0; the page's BS <= 512 is not enforced)
+ *   k                experts per token, 0 < K <= 16 and K <= N
+ *   h                hidden size, H > 0 and H * 2 a multiple of 16
+ *   num_experts      routed experts E, 1 <= E <= 1024
+ *   zero/copy/const_expert_num   Z, C, Q >= 0; ids [E, E+Z) are zero experts,
+ *                    [E+Z, E+Z+C) copy experts, [E+Z+C, N) const experts
+ *   a_capacity       A, rows of expand_x; A >= BS * min(E, K)
+ *   dtype            moe_dtype of x, expand_x and every 16-bit tensor
+ *   mask_ndim        0: no x_active_mask; 1: mask (BS,); 2: mask (BS, K)
+ */
+typedef struct {
+  int32_t bs, k, h, num_experts, zero_expert_num, copy_expert_num, const_expert_num,
+      a_capacity;
+  int32_t dtype;
+  int32_t mask_ndim;
+} moe_shape;
+
+/* Text of a status code (static storage). */
+const char* moe_status_string(int status);
+
+/* The CUDA error (cudaError_t value) behind the last MOE_ERR_CUDA on this thread. */
+int moe_last_cuda_error(void);
+
+/* Elements of the int32 assist_info buffer: A + BS * K. */
+size_t moe_assist_info_elems(const moe_shape* shape);
+
+/* Bytes of device workspace moe_dispatch_layout needs (may be 0). */
+size_t moe_layout_workspace_bytes(const moe_shape* shape);
+
+/*
+ * moe_dispatch_layout — [combine] Parameters (assist_info_for_combine,
+ * ep_send_counts, x_active_mask) and Constraints.
+ *
+ * A pair (t, k) is routed when topk_idx[t, k] is in [0, E), is not a repeat of
+ * an earlier id in row t, and is active in the mask. Routed pairs are laid out
+ * expert by expert, and inside an expert by token (a stable order); pair
+ * (t, k) gets slot s.
+ *   topk_idx           int32 (BS, K), in
+ *   x_active_mask      uint8 (BS,) or (BS, K) per shape->mask_ndim, or NULL
+ *   expert_token_nums  int32 (E,), out: routed pairs per expert
+ *   ep_send_counts     int32 (E + 1,), out: exclusive prefix sum of
+ *                      expert_token_nums with the total R appended; expert e
+ *                      owns slots [ep_send_counts[e], ep_send_counts[e + 1])
+ *   assist_info        int32 (A + BS * K,), out, opaque to callers: entry s < A
+ *                      holds t * K + k of the pair in slot s (-1 for s >= R);
+ *                      entry A + t * K + k holds the slot of pair (t, k), or -1
+ *   dev_status         uint32 (1,), out, or NULL: overwritten with the
+ *                      MOE_DEV_* bits found in topk_idx
+ *   workspace          device scratch of moe_layout_workspace_bytes() bytes
+ *                      (NULL allowed when that is 0); its contents on entry do
+ *                      not matter
+ */
+moe_status moe_dispatch_layout(const moe_shape* shape, const int32_t* topk_idx,
+                               const uint8_t* x_active_mask, int32_t* expert_token_nums,
+                               int32_t* ep_send_counts, int32_t* assist_info,
+                               uint32_t* dev_status, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * moe_dispatch_permute — the local stand-in for dispatch's alltoallv
+ * ([combine] Function: Description) with the optional per-row int8
+ * quantisation of comm_quant_mode / quant_mode 2 ([combine] Parameters,
+ * Example).
+ *   x                (BS, H) dtype, in
+ *   assist_info      from moe_dispatch_layout, in
+ *   ep_send_counts   accepted for interface parity with the page; not read
+ *   comm_quant_mode  0: expand_x[s] = x[t] bit for bit, expand_x is (A, H) dtype
+ *                    2: scale[t] = max_h |x[t, h]| / 127 (fp32, IEEE division),
+ *                       expand_x[s] = int8(clamp(rne(x[t] / scale), -127, 127)),
+ *                       dynamic_scales[s] = scale; expand_x is (A, H) int8 and
+ *                       H must be a multiple of 16; all-zero rows give scale 0
+ *   Rows s >= R of expand_x (and dynamic_scales) are not written.
+ */
+moe_status moe_dispatch_permute(const moe_shape* shape, const void* x,
+                                const int32_t* assist_info, const int32_t* ep_send_counts,
+                                int comm_quant_mode, void* expand_x, float* dynamic_scales,
+                                void* stream);
+
+/*
+ * moe_combine_fwd — [combine] Function (Formula; special expert use cases),
+ * Parameters, Return Value:
+ *   out[t] = round16( sum_{k active, ascending} w[t,k] * M(t,k)  +  shared[t] )
+ * with M = expand_x[slot(t,k)] for routed pairs, 0 for zero experts, ori_x[t]
+ * for copy experts, alpha_1[j] * ori_x[t] + alpha_2[j] * v[j] for const expert
+ * j = id - (E + Z + C). Everything is fp32 with each product and each sum
+ * rounded on its own (no fused multiply-add), then one round-to-nearest-even
+ * cast.
+ *   expand_x         (A, H) dtype: the experts' outputs, in slot order
+ *   topk_idx         int32 (BS, K); topk_weights fp32 (BS, K)
+ *   assist_info      from moe_dispatch_layout; ep_send_counts: not read
+ *   x_active_mask    as for the layout, or NULL
+ *   shared_expert_x  (BS, H) dtype or NULL (added once, unweighted)
+ *   ori_x            (BS, H) dtype; required when C > 0 or Q > 0
+ *   const_alpha_1, const_alpha_2, const_v   (Q, H) dtype; required when Q > 0
+ *   out              (BS, H) dtype
+ */
+moe_status moe_combine_fwd(const moe_shape* shape, const void* expand_x,
+                           const int32_t* topk_idx, const float* topk_weights,
+                           const int32_t* assist_info, const int32_t* ep_send_counts,
+                           const uint8_t* x_active_mask, const void* shared_expert_x,
+                           const void* ori_x, const void* const_alpha_1,
+                           const void* const_alpha_2, const void* const_v, void* out,
+                           void* stream);
+
+/*
+ * moe_combine_bwd — gradient of the combine Formula for routed pairs (the
+ * fused EP MoE layer of the Triton-distributed ep_moe_fused PR has a backward):
+ *   grad_expand[slot(t,k)] = round16(w[t,k] * grad_out[t])     (fp32 product)
+ *   grad_w[t,k]            = sum_h grad_out[t,h] * expand_x[slot(t,k),h] (fp32)
+ * Pairs without a slot or masked get grad_w = 0 and write no row. The gradient
+ * of shared_expert_x is grad_out itself (no call needed).
+ *   grad_out (BS, H), expand_x (A, H), topk_weights fp32 (BS, K),
+ *   grad_expand (A, H) out, grad_w fp32 (BS, K) out. topk_idx is not read.
+ */
+moe_status moe_combine_bwd(const moe_shape* shape, const void* grad_out, const void* expand_x,
+                           const int32_t* topk_idx, const float* topk_weights,
+                           const int32_t* assist_info, const uint8_t* x_active_mask,
+                           void* grad_expand, float* grad_w, void* stream);
+
+/*
+ * moe_dispatch_bwd — gradient of the permute: every token gathers the
+ * gradients of its slots, unweighted, summed in fp32 in ascending k:
+ *   grad_x[t] = round16( sum_{k with a slot, active} grad_expand_in[slot(t,k)] )
+ *   grad_expand_in (A, H), grad_x (BS, H) out.
+ */
+moe_status moe_dispatch_bwd(const moe_shape* shape, const void* grad_expand_in,
+                            const int32_t* assist_info, const uint8_t* x_active_mask,
+                            void* grad_x, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DC_H */
