@@ -67,6 +67,26 @@ def byte_model(wl: workloads.Workload, r: int, ori_tokens: int) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# Replicas: only the timing is reduced across ranks (max), never data.
+
+def reduce_max(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(tokens_per_rank_step: int, steps: int, world: int,
+                         max_total_ms: float) -> float:
+    """Tokens of all replicas divided by the slowest replica's time."""
+    return tokens_per_rank_step * steps * world / (max_total_ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # Clock sampling during the timed region.
 
 class ClockSampler:
@@ -401,14 +421,9 @@ def main():
     step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
     per_kernel_ms = {k: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]
                      for j, k in enumerate(kernels)}
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = reduce_max(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
-    tokens = wl.bs * args.steps * world
-    value = tokens / (total_ms * 1e-3)
+    value = whole_job_throughput(wl.bs, args.steps, world, total_ms)
     bytes_step = sum(bytes_per.values())
 
     # e2e: pinned host inputs -> H2D -> the path through the C ABI -> D2H of the results
@@ -442,12 +457,8 @@ def main():
             e2e_step()
         eb.record(stream)
         torch.cuda.synchronize()
-        e_ms = ea.elapsed_time(eb)
-        if world > 1:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": wl.bs * e2e_steps * world / (e_ms * 1e-3), "unit": "tokens/s",
+        e_ms = reduce_max(ea.elapsed_time(eb), dev)
+        e2e = {"value": whole_job_throughput(wl.bs, e2e_steps, world, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps}
 
     if rank == 0:

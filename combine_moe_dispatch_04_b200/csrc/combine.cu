@@ -20,110 +20,176 @@ namespace moe {
 namespace {
 
 constexpr int kFwdThreads = 256;
+constexpr int kFwdWarps = kFwdThreads / 32;
 
 enum PairKind : int { kSkip = 0, kRouted = 1, kZero = 2, kCopy = 3, kConst = 4 };
 
-template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
-__global__ void __launch_bounds__(kFwdThreads) combine_fwd_kernel(CombineArgs a) {
-  const int V = a.H / kVecElems;
-  const int item = blockIdx.x * kFwdThreads + threadIdx.x;
-  if (item >= a.bs * V) return;
-  const int t = item / V;
-  const int v = item - t * V;
+// Metadata of pair (t, lane) held by lane k < K of the warp.
+struct PairMeta {
+  int kind;
+  int slot;  // routed: expand_x row; const: row of alpha_1/alpha_2/v
+  float w;
+};
+
+template <bool SPECIAL, bool UNIT>
+__device__ __forceinline__ PairMeta load_meta(const CombineArgs& a, int t, int lane) {
+  PairMeta m{kSkip, -1, 1.0f};
   const int K = a.K;
+  int id = -1;
+  if (lane < K) {
+    const size_t tk = static_cast<size_t>(t) * K + lane;
+    const bool act = pair_active(a.mask, a.mask_ndim, t, lane, K);
+    const int s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
+    if (!UNIT) m.w = __ldg(a.weights + tk);
+    if (!SPECIAL) {
+      if (act && s >= 0) {
+        m.kind = kRouted;
+        m.slot = s;
+      }
+    } else {
+      id = __ldg(a.topk_idx + tk);
+      const int n_ids = a.E + a.Z + a.C + a.Q;
+      if (act && id >= 0 && id < n_ids) {
+        if (id < a.E) {
+          if (s >= 0) {
+            m.kind = kRouted;
+            m.slot = s;
+          }
+        } else if (id < a.E + a.Z) {
+          m.kind = kZero;
+        } else if (id < a.E + a.Z + a.C) {
+          m.kind = kCopy;
+        } else {
+          m.kind = kConst;
+          m.slot = id - (a.E + a.Z + a.C);
+        }
+      }
+    }
+  }
+  if (SPECIAL) {  // a repeat of an earlier id in the row takes no part
+    bool dup = false;
+    for (int j = 0; j < K; ++j) {
+      const int idj = __shfl_sync(0xFFFFFFFFu, id, j);
+      dup |= j < lane && idj == id;
+    }
+    if (dup) m.kind = kSkip;
+  }
+  return m;
+}
+
+// The 8 values m of pair j for one vector: the routed row, 0, ori_x, or
+// alpha_1 * ori_x + alpha_2 * v (each product and the sum rounded on its own).
+template <typename T16, bool SPECIAL>
+__device__ __forceinline__ void pair_values(const CombineArgs& a, int kind, int row, int V, int v,
+                                            const uint4& val, const float (&ori)[8],
+                                            float (&m)[8]) {
+  if (!SPECIAL || kind == kRouted) {
+    widen8<T16>(val, m);
+  } else if (kind == kZero) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+  } else if (kind == kCopy) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = ori[i];
+  } else {
+    const size_t r = static_cast<size_t>(row) * V + v;
+    float a1[8], a2[8], cv[8];
+    widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + r), a1);
+    widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + r), a2);
+    widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + r), cv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(__fmul_rn(a1[i], ori[i]), __fmul_rn(a2[i], cv[i]));
+  }
+}
+
+// One warp per (token, chunk of 32 * U vectors) item, items strided over a
+// persistent grid. Lane k < K holds pair k's metadata (broadcast by shuffle);
+// every lane owns U vectors of the chunk and issues the loads of all K rows
+// before accumulating, so K * U 16-byte loads are in flight per lane. The next
+// item's metadata is fetched while the current rows are in flight.
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
+__global__ void __launch_bounds__(kFwdThreads) combine_fwd_kernel(CombineArgs a, int chunks,
+                                                                  int n_items) {
+  constexpr int U = KMAX <= 4 ? 2 : 1;
+  pdl_trigger();
+  pdl_wait();
+  const int V = a.H / kVecElems;
+  const int K = a.K;
+  const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * kFwdWarps;
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
-  const int32_t* slots = a.assist + static_cast<size_t>(a.A) + static_cast<size_t>(t) * K;
-  const int32_t* ids = SPECIAL ? a.topk_idx + static_cast<size_t>(t) * K : nullptr;
-  const int n_ids = a.E + a.Z + a.C + a.Q;
-
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-
-  for (int k0 = 0; k0 < K; k0 += KMAX) {
-    uint4 val[KMAX];
-    int kind[KMAX];
-    bool need_ori = false;
+  int item = blockIdx.x * kFwdWarps + (threadIdx.x >> 5);
+  PairMeta meta;
+  if (item < n_items) meta = load_meta<SPECIAL, UNIT>(a, item / chunks, lane);
+  for (; item < n_items; item += stride) {
+    const int t = item / chunks;
+    const int v0 = (item - t * chunks) * 32 * U + lane;
+    uint4 val[KMAX][U];
+    int kind[KMAX], row[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      const int k = k0 + j;
-      kind[j] = kSkip;
-      if (k >= K) continue;
-      if (!pair_active(a.mask, a.mask_ndim, t, k, K)) continue;
-      if (!SPECIAL) {
-        const int s = __ldg(slots + k);
-        if (s >= 0) {
-          val[j] = ld_nc_v4(Y + static_cast<size_t>(s) * V + v);
-          kind[j] = kRouted;
+      kind[j] = __shfl_sync(0xFFFFFFFFu, meta.kind, j);
+      row[j] = __shfl_sync(0xFFFFFFFFu, meta.slot, j);
+      if (j >= K) kind[j] = kSkip;
+      if (kind[j] == kRouted) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * 32;
+          if (v < V) val[j][u] = ld_nc_v4(Y + static_cast<size_t>(row[j]) * V + v);
         }
-        continue;
-      }
-      const int id = __ldg(ids + k);
-      if (id < 0 || id >= n_ids) continue;
-      bool dup = false;
-      for (int jj = 0; jj < k; ++jj) dup |= __ldg(ids + jj) == id;
-      if (dup) continue;
-      if (id < a.E) {
-        const int s = __ldg(slots + k);
-        if (s >= 0) {
-          val[j] = ld_nc_v4(Y + static_cast<size_t>(s) * V + v);
-          kind[j] = kRouted;
-        }
-      } else if (id < a.E + a.Z) {
-        kind[j] = kZero;
-      } else if (id < a.E + a.Z + a.C) {
-        kind[j] = kCopy;
-        need_ori = true;
-      } else {
-        const size_t q = static_cast<size_t>(id - (a.E + a.Z + a.C));
-        // alpha_1[q], alpha_2[q], v[q] are combined below; stash row q here.
-        val[j] = make_uint4(static_cast<uint32_t>(q), 0u, 0u, 0u);
-        kind[j] = kConst;
-        need_ori = true;
       }
     }
-    float ori[8];
-    if (SPECIAL && need_ori) {
-      widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
+    float ori[U][8];
+    if (SPECIAL) {
+      bool need = false;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) need |= kind[j] == kCopy || kind[j] == kConst;
+      if (need) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * 32;
+          if (v < V)
+            widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + static_cast<size_t>(t) * V + v),
+                        ori[u]);
+        }
+      }
     }
+    const float w_lane = meta.w;
+    if (item + stride < n_items) meta = load_meta<SPECIAL, UNIT>(a, (item + stride) / chunks, lane);
+    float acc[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
+      const float w = UNIT ? 1.0f : __shfl_sync(0xFFFFFFFFu, w_lane, j);
       if (kind[j] == kSkip) continue;
-      float m[8];
-      if (!SPECIAL || kind[j] == kRouted) {
-        widen8<T16>(val[j], m);
-      } else if (kind[j] == kZero) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m[i] = 0.0f;
-      } else if (kind[j] == kCopy) {
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + u * 32;
+        if (v >= V) continue;
+        float m[8];
+        pair_values<T16, SPECIAL>(a, kind[j], row[j], V, v, val[j][u], ori[u], m);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m[i] = ori[i];
-      } else {
-        const size_t row = static_cast<size_t>(val[j].x) * V + v;
-        float a1[8], a2[8], cv[8];
-        widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + row), a1);
-        widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + row), a2);
-        widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + row), cv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(__fmul_rn(a1[i], ori[i]), __fmul_rn(a2[i], cv[i]));
-      }
-      if (UNIT) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], m[i]);
-      } else {
-        const float w = __ldg(a.weights + static_cast<size_t>(t) * K + k0 + j);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, m[i]));
+        for (int i = 0; i < 8; ++i)
+          acc[u][i] = UNIT ? __fadd_rn(acc[u][i], m[i]) : __fadd_rn(acc[u][i], __fmul_rn(w, m[i]));
       }
     }
-  }
-  if (!UNIT && a.shared != nullptr) {
-    float sh[8];
-    widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], sh[i]);
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * 32;
+      if (v >= V) continue;
+      const size_t o = static_cast<size_t>(t) * V + v;
+      if (!UNIT && a.shared != nullptr) {
+        float sh[8];
+        widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + o), sh);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], sh[i]);
+      }
+      st_v4(static_cast<uint4*>(a.out) + o, narrow8<T16>(acc[u]));
+    }
   }
-  st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
 }
 
 constexpr int kBwdThreads = 256;
@@ -131,10 +197,7 @@ constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kBwdUnroll = 4;
 
 template <typename T16>
-__global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(CombineBwdArgs a) {
-  const int pair = blockIdx.x * kBwdWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (pair >= a.bs * a.K) return;
+__device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pair, int lane) {
   const int t = pair / a.K;
   const int k = pair - t * a.K;
   const int s = __ldg(a.assist + static_cast<size_t>(a.A) + pair);
@@ -181,19 +244,51 @@ __global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(CombineBwdArgs
   if (lane == 0) a.grad_w[pair] = dot;
 }
 
+template <typename T16>
+__global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(CombineBwdArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int n_pairs = a.bs * a.K;
+  const int stride = gridDim.x * kBwdWarps;
+  for (int pair = blockIdx.x * kBwdWarps + (threadIdx.x >> 5); pair < n_pairs; pair += stride)
+    combine_bwd_pair<T16>(a, pair, lane);
+}
+
+// Resident blocks per SM of a kernel (occupancy API), cached per kernel.
+template <auto Kernel>
+int blocks_per_sm(int threads, size_t smem) {
+  static int cached = 0;
+  if (cached == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    cached = n;
+  }
+  return cached;
+}
+
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
+cudaError_t launch_fwd_kmax(const CombineArgs& a, cudaStream_t st) {
+  constexpr int U = KMAX <= 4 ? 2 : 1;
+  constexpr auto kernel = combine_fwd_kernel<T16, KMAX, SPECIAL, UNIT>;
+  const int V = a.H / kVecElems;
+  const int chunks = (V + 32 * U - 1) / (32 * U);
+  const long long items = static_cast<long long>(a.bs) * chunks;
+  const long long want = (items + kFwdWarps - 1) / kFwdWarps;
+  const long long cap = static_cast<long long>(sm_count()) * blocks_per_sm<kernel>(kFwdThreads, 0);
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(kernel, dim3(blocks), dim3(kFwdThreads), 0, st, a, chunks,
+                    static_cast<int>(items));
+}
+
 template <typename T16, bool SPECIAL, bool UNIT>
 cudaError_t launch_fwd_k(const CombineArgs& a, cudaStream_t st) {
-  const long long n = static_cast<long long>(a.bs) * (a.H / kVecElems);
-  const int blocks = static_cast<int>((n + kFwdThreads - 1) / kFwdThreads);
-  if (a.K <= 2)
-    combine_fwd_kernel<T16, 2, SPECIAL, UNIT><<<blocks, kFwdThreads, 0, st>>>(a);
-  else if (a.K <= 4)
-    combine_fwd_kernel<T16, 4, SPECIAL, UNIT><<<blocks, kFwdThreads, 0, st>>>(a);
-  else if (a.K <= 8)
-    combine_fwd_kernel<T16, 8, SPECIAL, UNIT><<<blocks, kFwdThreads, 0, st>>>(a);
-  else
-    combine_fwd_kernel<T16, 16, SPECIAL, UNIT><<<blocks, kFwdThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  if (a.K <= 2) return launch_fwd_kmax<T16, 2, SPECIAL, UNIT>(a, st);
+  if (a.K <= 4) return launch_fwd_kmax<T16, 4, SPECIAL, UNIT>(a, st);
+  if (a.K <= 8) return launch_fwd_kmax<T16, 8, SPECIAL, UNIT>(a, st);
+  return launch_fwd_kmax<T16, 16, SPECIAL, UNIT>(a, st);
 }
 
 template <typename T16>
@@ -212,13 +307,14 @@ cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st) {
 
 cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
+  auto kernel = a.dtype == MOE_BF16 ? combine_bwd_kernel<Bf16> : combine_bwd_kernel<Fp16>;
   const long long pairs = static_cast<long long>(a.bs) * a.K;
-  const int blocks = static_cast<int>((pairs + kBwdWarps - 1) / kBwdWarps);
-  if (a.dtype == MOE_BF16)
-    combine_bwd_kernel<Bf16><<<blocks, kBwdThreads, 0, st>>>(a);
-  else
-    combine_bwd_kernel<Fp16><<<blocks, kBwdThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  const long long want = (pairs + kBwdWarps - 1) / kBwdWarps;
+  const long long cap = static_cast<long long>(sm_count()) *
+                        (a.dtype == MOE_BF16 ? blocks_per_sm<combine_bwd_kernel<Bf16>>(kBwdThreads, 0)
+                                             : blocks_per_sm<combine_bwd_kernel<Fp16>>(kBwdThreads, 0));
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(kernel, dim3(blocks), dim3(kBwdThreads), 0, st, a);
 }
 
 }  // namespace moe

@@ -76,6 +76,32 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// ---- programmatic dependent launch (PDL) ----
+// Every kernel lets its successor in the stream begin launching as soon as all
+// of its CTAs are running, and waits for its predecessor's results (and their
+// memory) before touching any data. Both are no-ops without the launch
+// attribute.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Whether pair (t, k) is active under x_active_mask (1-D per token, 2-D per pair).
 __device__ __forceinline__ bool pair_active(const uint8_t* mask, int mask_ndim, int t, int k,
                                             int K) {

@@ -20,7 +20,7 @@ struct LayoutArgs {
 };
 
 // Tokens per CTA in the multi-CTA layout, and the largest BS of the one-CTA layout.
-constexpr int kLayoutTileTokens = 128;
+constexpr int kLayoutTileTokens = 256;
 constexpr int kLayoutSmallMaxTokens = 1024;
 
 size_t layout_workspace_bytes(int bs, int E);

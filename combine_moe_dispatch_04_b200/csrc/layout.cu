@@ -11,9 +11,11 @@
 // deterministic.
 //
 //   BS <= 1024: one CTA of 32 warps does everything (one launch).
-//   otherwise : count (one CTA per 128-token tile) -> scan (one CTA) ->
-//               scatter (one CTA per tile); the per-(tile, expert) counts live
-//               in the caller's workspace.
+//   otherwise : count (one CTA per 256-token tile) -> scatter (same tiles):
+//               every scatter CTA sums the per-(tile, expert) counts of the
+//               caller's workspace itself (its tile's prefix and the expert
+//               totals), scans the totals, and writes its tile's slots; CTA 0
+//               also writes the counts and the status word.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -115,6 +117,8 @@ __global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
   __shared__ int offs[1024];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
+  pdl_trigger();
+  pdl_wait();
   const int E = a.E;
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) words[i] = 0;
   if (threadIdx.x == 0) status = 0;
@@ -178,6 +182,8 @@ constexpr int kTileWarps = kLayoutTileTokens / 32;
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutArgs a, int T) {
   extern __shared__ uint32_t words[];  // [kTileWarps][E]
   __shared__ uint32_t status;
+  pdl_trigger();
+  pdl_wait();
   const int E = a.E;
   for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
   if (threadIdx.x == 0) status = 0;
@@ -200,67 +206,62 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutA
   if (threadIdx.x == 0) ws.status[blockIdx.x] = status;
 }
 
-// Phase 2 (one CTA of 1024 threads): expert totals, their exclusive scan, and
-// the first slot of every (tile, expert) written back over the counts.
-__global__ void __launch_bounds__(1024) layout_scan_kernel(LayoutArgs a, int T) {
-  __shared__ int part[1024];  // [G][E], partial sums of tile groups
-  __shared__ int offs[1024];
+// Phase 2: the tile's first slot per expert, from the count matrix
+// (prefix over earlier tiles + exclusive scan of the expert totals), then the
+// slots of every pair of the tile and -1 for the unused slots [R, A).
+// Dynamic shared memory: words[kTileWarps][E], base[E], total[E].
+__global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
+  extern __shared__ uint32_t smem[];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
   const int E = a.E;
-  TileWs ws = tile_ws(a, T);
-  const int G = max(1, min(1024 / E, T));
-  const int chunk = (T + G - 1) / G;
-  const int ex = threadIdx.x % E, g = threadIdx.x / E;
-  const bool grp = g < G;
-  const int t0 = g * chunk, t1 = min(T, t0 + chunk);
-  if (threadIdx.x == 0) status = 0;
-  __syncthreads();
-  if (grp) {
-    int s = 0;
-    for (int tile = t0; tile < t1; ++tile) s += ws.counts[static_cast<size_t>(tile) * E + ex];
-    part[g * E + ex] = s;
-  }
-  uint32_t st = 0;
-  for (int tile = threadIdx.x; tile < T; tile += blockDim.x) st |= ws.status[tile];
-  if (st) atomicOr(&status, st);
-  __syncthreads();
-  int cnt = 0;
-  if (threadIdx.x < E) {
-    for (int gg = 0; gg < G; ++gg) {
-      const int v = part[gg * E + threadIdx.x];
-      part[gg * E + threadIdx.x] = cnt;
-      cnt += v;
-    }
-  }
-  int total;
-  const int excl = block_exclusive_scan(cnt, warp_sums, &total);
-  if (threadIdx.x < E) {
-    offs[threadIdx.x] = excl;
-    a.expert_token_nums[threadIdx.x] = cnt;
-    a.ep_send_counts[threadIdx.x] = excl;
-  }
-  if (threadIdx.x == 0) a.ep_send_counts[E] = total;
-  __syncthreads();
-  if (grp) {
-    int run = offs[ex] + part[g * E + ex];
-    for (int tile = t0; tile < t1; ++tile) {
-      int* p = &ws.counts[static_cast<size_t>(tile) * E + ex];
-      const int c = *p;
-      *p = run;
-      run += c;
-    }
-  }
-  if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
-}
-
-// Phase 3: slots of every pair of the tile, and -1 for the unused slots [R, A).
-__global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
-  extern __shared__ uint32_t words[];  // [kTileWarps][E]
-  const int E = a.E;
+  uint32_t* words = smem;
+  int* base = reinterpret_cast<int*>(smem + kTileWarps * E);
+  int* total = base + E;
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
+  if (threadIdx.x == 0) status = 0;
+  const TileWs ws = tile_ws(a, T);
+  const int tile = blockIdx.x;
+  for (int ex = threadIdx.x; ex < E; ex += blockDim.x) {
+    int before = 0, all = 0;
+#pragma unroll 8
+    for (int i = 0; i < T; ++i) {
+      const int c = ws.counts[static_cast<size_t>(i) * E + ex];
+      before += i < tile ? c : 0;
+      all += c;
+    }
+    base[ex] = before;
+    total[ex] = all;
+  }
+  if (blockIdx.x == 0) {
+    uint32_t st = 0;
+    for (int i = threadIdx.x; i < T; i += blockDim.x) st |= ws.status[i];
+    if (st) atomicOr(&status, st);
+  }
   __syncthreads();
-  const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
+  // exclusive scan of total[0, E): each thread owns a contiguous run of experts
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
+  int run = 0;
+  for (int ex = e0; ex < e1; ++ex) run += total[ex];
+  int grand;
+  int off = block_exclusive_scan(run, warp_sums, &grand);
+  for (int ex = e0; ex < e1; ++ex) {
+    const int c = total[ex];
+    if (blockIdx.x == 0) {
+      a.expert_token_nums[ex] = c;
+      a.ep_send_counts[ex] = off;
+    }
+    base[ex] += off;
+    off += c;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.ep_send_counts[E] = grand;
+    if (a.dev_status) *a.dev_status = status;
+  }
+  const int t = tile * kLayoutTileTokens + threadIdx.x;
   int e[kMaxK];
   if (t < a.bs) {
     classify_row(a, t, e);
@@ -268,16 +269,13 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
   }
   __syncthreads();
   if (t < a.bs) {
-    TileWs ws = tile_ws(a, T);
-    const int32_t* base = ws.counts + static_cast<size_t>(blockIdx.x) * E;
     int slot[kMaxK];
 #pragma unroll
     for (int k = 0; k < kMaxK; ++k)
       slot[k] = (k < a.K && e[k] >= 0) ? base[e[k]] + tile_rank(words, E, e[k]) : -1;
     write_slots(a, t, e, slot);
   }
-  const int total = a.ep_send_counts[E];
-  for (int s = total + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
+  for (int s = grand + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
        s += gridDim.x * blockDim.x)
     a.assist[s] = -1;
 }
@@ -293,19 +291,22 @@ size_t layout_workspace_bytes(int bs, int E) {
 cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st) {
   if (a.bs <= kLayoutSmallMaxTokens) {
     const size_t smem = 32u * a.E * sizeof(uint32_t);
-    cudaError_t err = cudaFuncSetAttribute(layout_small_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    layout_small_kernel<<<1, 1024, smem, st>>>(a);
-    return cudaGetLastError();
+    if (smem > 48 * 1024) {
+      cudaError_t err = cudaFuncSetAttribute(layout_small_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+      if (err != cudaSuccess) return err;
+    }
+    return launch_pdl(layout_small_kernel, dim3(1), dim3(1024), smem, st, a);
   }
   const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
-  const size_t smem = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
-  layout_count_kernel<<<T, kLayoutTileTokens, smem, st>>>(a, T);
-  layout_scan_kernel<<<1, 1024, 0, st>>>(a, T);
-  layout_scatter_kernel<<<T, kLayoutTileTokens, smem, st>>>(a, T);
-  return cudaGetLastError();
+  const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
+  const size_t smem_scatter = smem_count + 2u * a.E * sizeof(int);
+  cudaError_t err = launch_pdl(layout_count_kernel, dim3(T), dim3(kLayoutTileTokens), smem_count,
+                               st, a, T);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(layout_scatter_kernel, dim3(T), dim3(kLayoutTileTokens), smem_scatter, st,
+                    a, T);
 }
 
 }  // namespace moe

@@ -16,24 +16,38 @@ namespace moe {
 namespace {
 
 constexpr int kCopyThreads = 256;
-constexpr int kCopyItems = 2;  // vectors per thread
+constexpr int kCopyWarps = kCopyThreads / 32;
+constexpr int kCopyU = 2;  // vectors per lane per item
 
+// One warp per (token, chunk of 32 * kCopyU vectors) item over a persistent
+// grid: the chunk of x[t] is read once into registers and stored to each of
+// the token's slots. Lane k < K holds slot k and broadcasts it by shuffle.
 __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
-    int bs, int K, int V, int A) {
-  const int n = bs * V;
-  const int32_t* slots_all = assist + static_cast<size_t>(A);
+    int K, int V, int A, int chunks, int n_items) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * kCopyWarps;
+  for (int item = blockIdx.x * kCopyWarps + (threadIdx.x >> 5); item < n_items; item += stride) {
+    const int t = item / chunks;
+    const int v0 = (item - t * chunks) * 32 * kCopyU + lane;
+    const int my_slot =
+        lane < K ? __ldg(assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K + lane) : -1;
+    uint4 val[kCopyU];
 #pragma unroll
-  for (int i = 0; i < kCopyItems; ++i) {
-    const int item = (blockIdx.x * kCopyItems + i) * kCopyThreads + threadIdx.x;
-    if (item >= n) return;
-    const int t = item / V;
-    const int v = item - t * V;
-    const uint4 val = ld_nc_v4(x + item);
-    const int32_t* slots = slots_all + static_cast<size_t>(t) * K;
+    for (int u = 0; u < kCopyU; ++u) {
+      const int v = v0 + u * 32;
+      if (v < V) val[u] = ld_nc_v4(x + static_cast<size_t>(t) * V + v);
+    }
     for (int k = 0; k < K; ++k) {
-      const int s = __ldg(slots + k);
-      if (s >= 0) st_v4(out + static_cast<size_t>(s) * V + v, val);
+      const int s = __shfl_sync(0xFFFFFFFFu, my_slot, k);
+      if (s < 0) continue;
+#pragma unroll
+      for (int u = 0; u < kCopyU; ++u) {
+        const int v = v0 + u * 32;
+        if (v < V) st_v4(out + static_cast<size_t>(s) * V + v, val[u]);
+      }
     }
   }
 }
@@ -45,6 +59,8 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
     float* __restrict__ scales, int bs, int K, int H, int A) {
   __shared__ float warp_max[8];
+  pdl_trigger();
+  pdl_wait();
   const int C = H / 16;  // chunks per row
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -115,13 +131,22 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
   if (a.quant_mode == 0) {
     const int V = a.H / kVecElems;
-    const long long n = static_cast<long long>(a.bs) * V;
-    const int per_block = kCopyThreads * kCopyItems;
-    const int blocks = static_cast<int>((n + per_block - 1) / per_block);
-    permute_copy_kernel<<<blocks, kCopyThreads, 0, st>>>(
-        static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x), a.bs, a.K, V,
-        a.A);
-    return cudaGetLastError();
+    const int chunks = (V + 32 * kCopyU - 1) / (32 * kCopyU);
+    const long long items = static_cast<long long>(a.bs) * chunks;
+    const long long want = (items + kCopyWarps - 1) / kCopyWarps;
+    static int per_sm = 0;
+    if (per_sm == 0) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, permute_copy_kernel, kCopyThreads, 0) !=
+              cudaSuccess || n < 1)
+        n = 1;
+      per_sm = n;
+    }
+    const long long cap = static_cast<long long>(sm_count()) * per_sm;
+    const int blocks = static_cast<int>(want < cap ? want : cap);
+    return launch_pdl(permute_copy_kernel, dim3(blocks), dim3(kCopyThreads), 0, st,
+                      static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
+                      a.K, V, a.A, chunks, static_cast<int>(items));
   }
   // One chunk per thread up to 256 threads, then up to 4 chunks per thread
   // (H <= 16384, checked by the caller).
@@ -130,15 +155,9 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   threads = threads > 256 ? 256 : threads;
   const int cap = sm_count() * 16;
   const int blocks = a.bs < cap ? a.bs : cap;
-  if (a.dtype == MOE_BF16)
-    permute_quant_kernel<Bf16><<<blocks, threads, 0, st>>>(
-        static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x), a.scales,
-        a.bs, a.K, a.H, a.A);
-  else
-    permute_quant_kernel<Fp16><<<blocks, threads, 0, st>>>(
-        static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x), a.scales,
-        a.bs, a.K, a.H, a.A);
-  return cudaGetLastError();
+  auto kernel = a.dtype == MOE_BF16 ? permute_quant_kernel<Bf16> : permute_quant_kernel<Fp16>;
+  return launch_pdl(kernel, dim3(blocks), dim3(threads), 0, st, static_cast<const uint4*>(a.x),
+                    a.assist, static_cast<uint4*>(a.expand_x), a.scales, a.bs, a.K, a.H, a.A);
 }
 
 }  // namespace moe
