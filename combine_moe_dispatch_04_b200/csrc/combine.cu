@@ -2,17 +2,18 @@
 // combine backward. [combine] Function (Formula; special expert use cases),
 // Parameters, Return Value.
 //
-// Forward: one thread per 16-byte vector (8 values) of an output row. The
-// thread issues the loads of all of its token's K slot rows first, then
-// accumulates in fp32 in ascending k with every product and every sum rounded
-// on its own (__fmul_rn / __fadd_rn: never contracted into an FMA), adds
-// shared_expert_x once, and narrows with round-to-nearest-even.
+// Forward: one thread per 16-byte vector (8 values) of an output row (or a
+// few vectors when K is small), in one-shot blocks. The thread issues the
+// loads of all of its token's K slot rows first, then accumulates in fp32 in
+// ascending k with every product and every sum rounded on its own
+// (__fmul_rn / __fadd_rn: never contracted into an FMA), adds shared_expert_x
+// once, and narrows with round-to-nearest-even.
 //
-// Backward: one warp per (token, k) pair; the warp streams the pair's
-// expand_x row against grad_out[t] (the K warps of a token share grad_out[t]
-// through L1), writes grad_expand = round16(w * grad_out) and reduces grad_w
-// with eight per-element accumulators per lane and a fixed butterfly, so the
-// result does not depend on scheduling.
+// Backward: one warp per (token, k) pair on a persistent grid; the warp
+// streams the pair's expand_x row against grad_out[t] (the K warps of a token
+// share grad_out[t] through L1), writes grad_expand = round16(w * grad_out)
+// and reduces grad_w with eight per-element accumulators per lane and a fixed
+// butterfly, so the result does not depend on scheduling.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -20,64 +21,10 @@ namespace moe {
 namespace {
 
 constexpr int kFwdThreads = 256;
-constexpr int kFwdWarps = kFwdThreads / 32;
 
 enum PairKind : int { kSkip = 0, kRouted = 1, kZero = 2, kCopy = 3, kConst = 4 };
 
-// Metadata of pair (t, lane) held by lane k < K of the warp.
-struct PairMeta {
-  int kind;
-  int slot;  // routed: expand_x row; const: row of alpha_1/alpha_2/v
-  float w;
-};
-
-template <bool SPECIAL, bool UNIT>
-__device__ __forceinline__ PairMeta load_meta(const CombineArgs& a, int t, int lane) {
-  PairMeta m{kSkip, -1, 1.0f};
-  const int K = a.K;
-  int id = -1;
-  if (lane < K) {
-    const size_t tk = static_cast<size_t>(t) * K + lane;
-    const bool act = pair_active(a.mask, a.mask_ndim, t, lane, K);
-    const int s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
-    if (!UNIT) m.w = __ldg(a.weights + tk);
-    if (!SPECIAL) {
-      if (act && s >= 0) {
-        m.kind = kRouted;
-        m.slot = s;
-      }
-    } else {
-      id = __ldg(a.topk_idx + tk);
-      const int n_ids = a.E + a.Z + a.C + a.Q;
-      if (act && id >= 0 && id < n_ids) {
-        if (id < a.E) {
-          if (s >= 0) {
-            m.kind = kRouted;
-            m.slot = s;
-          }
-        } else if (id < a.E + a.Z) {
-          m.kind = kZero;
-        } else if (id < a.E + a.Z + a.C) {
-          m.kind = kCopy;
-        } else {
-          m.kind = kConst;
-          m.slot = id - (a.E + a.Z + a.C);
-        }
-      }
-    }
-  }
-  if (SPECIAL) {  // a repeat of an earlier id in the row takes no part
-    bool dup = false;
-    for (int j = 0; j < K; ++j) {
-      const int idj = __shfl_sync(0xFFFFFFFFu, id, j);
-      dup |= j < lane && idj == id;
-    }
-    if (dup) m.kind = kSkip;
-  }
-  return m;
-}
-
-// The 8 values m of pair j for one vector: the routed row, 0, ori_x, or
+// The 8 values m of one pair for one vector: the routed row, 0, ori_x, or
 // alpha_1 * ori_x + alpha_2 * v (each product and the sum rounded on its own).
 template <typename T16, bool SPECIAL>
 __device__ __forceinline__ void pair_values(const CombineArgs& a, int kind, int row, int V, int v,
@@ -102,93 +49,106 @@ __device__ __forceinline__ void pair_values(const CombineArgs& a, int kind, int 
   }
 }
 
-// One warp per (token, chunk of 32 * U vectors) item, items strided over a
-// persistent grid. Lane k < K holds pair k's metadata (broadcast by shuffle);
-// every lane owns U vectors of the chunk and issues the loads of all K rows
-// before accumulating, so K * U 16-byte loads are in flight per lane. The next
-// item's metadata is fetched while the current rows are in flight.
+// Vectors per thread: enough that every thread keeps eight 16-byte row loads
+// in flight when K is small.
+template <int KMAX>
+__host__ __device__ constexpr int fwd_vectors_per_thread() {
+  return KMAX >= 8 ? 1 : 8 / KMAX;
+}
+
+// One thread per U output vectors (8 values each) spaced a block apart, so a
+// warp's loads stay coalesced along the rows. For each vector the thread
+// classifies its token's K pairs, issues the loads of all routed rows, then
+// accumulates in ascending k.
 template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
-__global__ void __launch_bounds__(kFwdThreads) combine_fwd_kernel(CombineArgs a, int chunks,
-                                                                  int n_items) {
-  constexpr int U = KMAX <= 4 ? 2 : 1;
+__global__ void __launch_bounds__(kFwdThreads) combine_fwd_kernel(CombineArgs a) {
+  constexpr int U = fwd_vectors_per_thread<KMAX>();
   pdl_trigger();
   pdl_wait();
   const int V = a.H / kVecElems;
   const int K = a.K;
-  const int lane = threadIdx.x & 31;
-  const int stride = gridDim.x * kFwdWarps;
+  const int n = a.bs * V;
+  const int n_ids = a.E + a.Z + a.C + a.Q;
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
-  int item = blockIdx.x * kFwdWarps + (threadIdx.x >> 5);
-  PairMeta meta;
-  if (item < n_items) meta = load_meta<SPECIAL, UNIT>(a, item / chunks, lane);
-  for (; item < n_items; item += stride) {
-    const int t = item / chunks;
-    const int v0 = (item - t * chunks) * 32 * U + lane;
-    uint4 val[KMAX][U];
-    int kind[KMAX], row[KMAX];
+  const int base = blockIdx.x * (kFwdThreads * U) + threadIdx.x;
+  uint4 val[U][KMAX];
+  int kind[U][KMAX], row[U][KMAX];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int item = base + u * kFwdThreads;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) kind[u][j] = kSkip;
+    if (item >= n) continue;
+    const int t = item / V;
+    const int v = item - t * V;
+    const int32_t* slots = a.assist + static_cast<size_t>(a.A) + static_cast<size_t>(t) * K;
+    int ids[KMAX];
+    if (SPECIAL) {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        ids[j] = j < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + j) : -1;
+    }
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      kind[j] = __shfl_sync(0xFFFFFFFFu, meta.kind, j);
-      row[j] = __shfl_sync(0xFFFFFFFFu, meta.slot, j);
-      if (j >= K) kind[j] = kSkip;
-      if (kind[j] == kRouted) {
+      if (j >= K || !pair_active(a.mask, a.mask_ndim, t, j, K)) continue;
+      int kd = kRouted, r = 0;
+      if (SPECIAL) {
+        const int id = ids[j];
+        bool dup = false;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + u * 32;
-          if (v < V) val[j][u] = ld_nc_v4(Y + static_cast<size_t>(row[j]) * V + v);
+        for (int jj = 0; jj < j; ++jj) dup |= ids[jj] == id;
+        if (dup || id < 0 || id >= n_ids) continue;
+        if (id >= a.E) {
+          kd = id < a.E + a.Z ? kZero : id < a.E + a.Z + a.C ? kCopy : kConst;
+          r = id - (a.E + a.Z + a.C);
         }
       }
+      if (kd == kRouted) {
+        const int s = __ldg(slots + j);
+        if (s < 0) continue;
+        val[u][j] = ld_nc_v4(Y + static_cast<size_t>(s) * V + v);
+      }
+      kind[u][j] = kd;
+      row[u][j] = r;
     }
-    float ori[U][8];
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int item = base + u * kFwdThreads;
+    if (item >= n) continue;
+    const int t = item / V;
+    const int v = item - t * V;
+    float ori[8];
     if (SPECIAL) {
       bool need = false;
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) need |= kind[j] == kCopy || kind[j] == kConst;
-      if (need) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + u * 32;
-          if (v < V)
-            widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + static_cast<size_t>(t) * V + v),
-                        ori[u]);
-        }
-      }
+      for (int j = 0; j < KMAX; ++j) need |= kind[u][j] == kCopy || kind[u][j] == kConst;
+      if (need) widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
     }
-    const float w_lane = meta.w;
-    if (item + stride < n_items) meta = load_meta<SPECIAL, UNIT>(a, (item + stride) / chunks, lane);
-    float acc[U][8];
+    float acc[8];
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      const float w = UNIT ? 1.0f : __shfl_sync(0xFFFFFFFFu, w_lane, j);
-      if (kind[j] == kSkip) continue;
+      if (kind[u][j] == kSkip) continue;
+      float m[8];
+      pair_values<T16, SPECIAL>(a, kind[u][j], row[u][j], V, v, val[u][j], ori, m);
+      if (UNIT) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int v = v0 + u * 32;
-        if (v >= V) continue;
-        float m[8];
-        pair_values<T16, SPECIAL>(a, kind[j], row[j], V, v, val[j][u], ori[u], m);
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], m[i]);
+      } else {
+        const float w = __ldg(a.weights + static_cast<size_t>(t) * K + j);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          acc[u][i] = UNIT ? __fadd_rn(acc[u][i], m[i]) : __fadd_rn(acc[u][i], __fmul_rn(w, m[i]));
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, m[i]));
       }
     }
+    if (!UNIT && a.shared != nullptr) {
+      float sh[8];
+      widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int v = v0 + u * 32;
-      if (v >= V) continue;
-      const size_t o = static_cast<size_t>(t) * V + v;
-      if (!UNIT && a.shared != nullptr) {
-        float sh[8];
-        widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + o), sh);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], sh[i]);
-      }
-      st_v4(static_cast<uint4*>(a.out) + o, narrow8<T16>(acc[u]));
+      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], sh[i]);
     }
+    st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
   }
 }
 
@@ -271,16 +231,11 @@ int blocks_per_sm(int threads, size_t smem) {
 
 template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
 cudaError_t launch_fwd_kmax(const CombineArgs& a, cudaStream_t st) {
-  constexpr int U = KMAX <= 4 ? 2 : 1;
-  constexpr auto kernel = combine_fwd_kernel<T16, KMAX, SPECIAL, UNIT>;
-  const int V = a.H / kVecElems;
-  const int chunks = (V + 32 * U - 1) / (32 * U);
-  const long long items = static_cast<long long>(a.bs) * chunks;
-  const long long want = (items + kFwdWarps - 1) / kFwdWarps;
-  const long long cap = static_cast<long long>(sm_count()) * blocks_per_sm<kernel>(kFwdThreads, 0);
-  const int blocks = static_cast<int>(want < cap ? want : cap);
-  return launch_pdl(kernel, dim3(blocks), dim3(kFwdThreads), 0, st, a, chunks,
-                    static_cast<int>(items));
+  constexpr int U = fwd_vectors_per_thread<KMAX>();
+  const long long n = static_cast<long long>(a.bs) * (a.H / kVecElems);
+  const int blocks = static_cast<int>((n + kFwdThreads * U - 1) / (kFwdThreads * U));
+  return launch_pdl(combine_fwd_kernel<T16, KMAX, SPECIAL, UNIT>, dim3(blocks), dim3(kFwdThreads),
+                    0, st, a);
 }
 
 template <typename T16, bool SPECIAL, bool UNIT>

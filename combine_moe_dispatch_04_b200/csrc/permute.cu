@@ -3,8 +3,7 @@
 // comm_quant_mode 2; Example: quant_mode = 2).
 //
 // Plain copy: one thread per 16-byte vector of x (coalesced along the row),
-// read once and stored to each of the token's K slots. The slot list of a
-// token is shared by the threads of its row and comes from L1.
+// read once and stored to each of the token's K slots; one-shot blocks.
 //
 // int8: one CTA per token (grid-stride); each thread keeps 16-element chunks
 // of the row in registers, the CTA reduces max|x|, and every chunk becomes one
@@ -16,38 +15,28 @@ namespace moe {
 namespace {
 
 constexpr int kCopyThreads = 256;
-constexpr int kCopyWarps = kCopyThreads / 32;
-constexpr int kCopyU = 2;  // vectors per lane per item
+constexpr int kCopyItems = 2;  // vectors per thread, a block apart
 
-// One warp per (token, chunk of 32 * kCopyU vectors) item over a persistent
-// grid: the chunk of x[t] is read once into registers and stored to each of
-// the token's slots. Lane k < K holds slot k and broadcasts it by shuffle.
+// One thread per 16-byte vector of x (coalesced along the row) in one-shot
+// blocks: the vector is read once and stored to each of the token's K slots.
 __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
-    int K, int V, int A, int chunks, int n_items) {
+    int bs, int K, int V, int A) {
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int stride = gridDim.x * kCopyWarps;
-  for (int item = blockIdx.x * kCopyWarps + (threadIdx.x >> 5); item < n_items; item += stride) {
-    const int t = item / chunks;
-    const int v0 = (item - t * chunks) * 32 * kCopyU + lane;
-    const int my_slot =
-        lane < K ? __ldg(assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K + lane) : -1;
-    uint4 val[kCopyU];
+  const int n = bs * V;
+  const int32_t* slots_all = assist + static_cast<size_t>(A);
 #pragma unroll
-    for (int u = 0; u < kCopyU; ++u) {
-      const int v = v0 + u * 32;
-      if (v < V) val[u] = ld_nc_v4(x + static_cast<size_t>(t) * V + v);
-    }
+  for (int i = 0; i < kCopyItems; ++i) {
+    const int item = (blockIdx.x * kCopyItems + i) * kCopyThreads + threadIdx.x;
+    if (item >= n) return;
+    const int t = item / V;
+    const int v = item - t * V;
+    const uint4 val = ld_nc_v4(x + item);
+    const int32_t* slots = slots_all + static_cast<size_t>(t) * K;
     for (int k = 0; k < K; ++k) {
-      const int s = __shfl_sync(0xFFFFFFFFu, my_slot, k);
-      if (s < 0) continue;
-#pragma unroll
-      for (int u = 0; u < kCopyU; ++u) {
-        const int v = v0 + u * 32;
-        if (v < V) st_v4(out + static_cast<size_t>(s) * V + v, val[u]);
-      }
+      const int s = __ldg(slots + k);
+      if (s >= 0) st_v4(out + static_cast<size_t>(s) * V + v, val);
     }
   }
 }
@@ -131,22 +120,12 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
   if (a.quant_mode == 0) {
     const int V = a.H / kVecElems;
-    const int chunks = (V + 32 * kCopyU - 1) / (32 * kCopyU);
-    const long long items = static_cast<long long>(a.bs) * chunks;
-    const long long want = (items + kCopyWarps - 1) / kCopyWarps;
-    static int per_sm = 0;
-    if (per_sm == 0) {
-      int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, permute_copy_kernel, kCopyThreads, 0) !=
-              cudaSuccess || n < 1)
-        n = 1;
-      per_sm = n;
-    }
-    const long long cap = static_cast<long long>(sm_count()) * per_sm;
-    const int blocks = static_cast<int>(want < cap ? want : cap);
+    const long long n = static_cast<long long>(a.bs) * V;
+    const int per_block = kCopyThreads * kCopyItems;
+    const int blocks = static_cast<int>((n + per_block - 1) / per_block);
     return launch_pdl(permute_copy_kernel, dim3(blocks), dim3(kCopyThreads), 0, st,
                       static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
-                      a.K, V, a.A, chunks, static_cast<int>(items));
+                      a.bs, a.K, V, a.A);
   }
   // One chunk per thread up to 256 threads, then up to 4 chunks per thread
   // (H <= 16384, checked by the caller).
