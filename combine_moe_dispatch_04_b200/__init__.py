@@ -24,7 +24,8 @@ MOE_DEV_BAD_ID, MOE_DEV_DUP_ID = 1, 2
 # Every entry point include/moe_dc.h declares.
 EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_layout_workspace_bytes", "moe_dispatch_layout", "moe_dispatch_permute",
-           "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd")
+           "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd",
+           "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes")
 
 
 class MoeShape(ctypes.Structure):
@@ -59,8 +60,11 @@ def _load():
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_combine_bwd.argtypes = [S, P, P, P, P, P, P, P, P, P]
     L.moe_dispatch_bwd.argtypes = [S, P, P, P, P, P]
+    L.moe_dispatch_layout_noalloc.argtypes = [S, P, P, P, P, P, P, P]
+    L.moe_layout_noalloc_max_workspace_bytes.argtypes = []
+    L.moe_layout_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
-              "moe_combine_bwd", "moe_dispatch_bwd"):
+              "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc"):
         getattr(L, n).restype = I
     return L
 
@@ -77,6 +81,8 @@ moe_dispatch_permute = _lib.moe_dispatch_permute
 moe_combine_fwd = _lib.moe_combine_fwd
 moe_combine_bwd = _lib.moe_combine_bwd
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
+moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
+moe_layout_noalloc_max_workspace_bytes = _lib.moe_layout_noalloc_max_workspace_bytes
 
 
 def library():
@@ -173,6 +179,17 @@ def dispatch_layout(shape: Shape, topk_idx, x_active_mask=None, *, workspace=Non
         ctypes.byref(shape.c()), _ptr(topk_idx), _ptr(x_active_mask), _ptr(out.expert_token_nums),
         _ptr(out.ep_send_counts), _ptr(out.assist_info), _ptr(out.dev_status), _ptr(workspace),
         ws_bytes, _stream(stream)))
+    return out
+
+
+def dispatch_layout_noalloc(shape: Shape, topk_idx, x_active_mask=None, *, out: Layout,
+                            stream=None) -> Layout:
+    """The layout without a workspace, for callers that cannot allocate device memory:
+    the library's own fixed scratch array stands in for it. ``out`` (caller-provided
+    outputs) is required, since this path allocates nothing."""
+    _check("moe_dispatch_layout_noalloc", moe_dispatch_layout_noalloc(
+        ctypes.byref(shape.c()), _ptr(topk_idx), _ptr(x_active_mask), _ptr(out.expert_token_nums),
+        _ptr(out.ep_send_counts), _ptr(out.assist_info), _ptr(out.dev_status), _stream(stream)))
     return out
 
 

@@ -248,6 +248,8 @@ moe_status moe_dispatch_bwd(const moe_shape* s, const void* grad_expand_in,
 
 namespace moe {
 
+moe_status report_cuda_error(cudaError_t err) { return cuda_status(err); }
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)

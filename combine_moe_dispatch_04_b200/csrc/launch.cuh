@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "moe_dc.h"
+
 namespace moe {
 
 struct LayoutArgs {
@@ -66,5 +68,8 @@ struct CombineBwdArgs {
 cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st);
 
 int sm_count();
+
+// Records err as the thread's last CUDA error; returns MOE_ERR_CUDA (MOE_OK for success).
+moe_status report_cuda_error(cudaError_t err);
 
 }  // namespace moe

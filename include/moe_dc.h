@@ -181,6 +181,41 @@ moe_status moe_dispatch_bwd(const moe_shape* shape, const void* grad_expand_in,
                             const int32_t* assist_info, const uint8_t* x_active_mask,
                             void* grad_x, void* stream);
 
+/*
+ * moe_dispatch_layout_noalloc — moe_dispatch_layout for callers that cannot
+ * allocate device memory. No counterpart in the paper: an addition of this
+ * library. It is for code that runs where every byte of device memory is
+ * owned by someone else — a plugin or kernel library handed buffers by a host
+ * framework that exposes no allocator, or a latency-critical serving loop that
+ * must not call cudaMalloc (which can synchronise the device) — and so cannot
+ * provide the workspace moe_dispatch_layout wants.
+ *
+ * Same arguments and results as moe_dispatch_layout, minus the workspace: the
+ * scratch is one fixed array of moe_layout_noalloc_max_workspace_bytes()
+ * bytes (1 MiB) compiled into the library, which every GPU that loads the
+ * library keeps until the process exits. A shape whose
+ * moe_layout_workspace_bytes() exceeds that size returns MOE_ERR_CAPACITY
+ * before anything runs (1 MiB covers, e.g., BS = 65 280 tokens with E = 1024,
+ * or about a million tokens with E = 64).
+ *
+ * The call allocates nothing (no cudaMalloc, no cudaFree, no allocator of any
+ * library). The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture. Every call shares the one array and
+ * leaves its contents behind; nothing in it needs clearing, because every
+ * entry the layout reads is written earlier in the same call. Calls whose
+ * work can overlap on the GPU (other streams, other threads) race on the
+ * array: serialise them, or give each its own workspace with
+ * moe_dispatch_layout.
+ */
+moe_status moe_dispatch_layout_noalloc(const moe_shape* shape, const int32_t* topk_idx,
+                                       const uint8_t* x_active_mask, int32_t* expert_token_nums,
+                                       int32_t* ep_send_counts, int32_t* assist_info,
+                                       uint32_t* dev_status, void* stream);
+
+/* Bytes of the fixed scratch array moe_dispatch_layout_noalloc uses. */
+size_t moe_layout_noalloc_max_workspace_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif
