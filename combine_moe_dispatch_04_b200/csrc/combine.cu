@@ -56,68 +56,132 @@ __host__ __device__ constexpr int fwd_vectors_per_thread() {
   return KMAX >= 8 ? 1 : 8 / KMAX;
 }
 
-// One thread per U output vectors (8 values each) spaced a block apart, so a
-// warp's loads stay coalesced along the rows. For each vector the thread
-// classifies its token's K pairs, issues the loads of all routed rows, then
-// accumulates in ascending k.
-template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
-__global__ void __launch_bounds__(kFwdThreads) combine_fwd_kernel(CombineArgs a) {
+// Pair metadata of one (token, k): kind, expand_x row or const row, weight.
+struct PairMeta {
+  int kind;
+  int row;
+  float w;
+};
+
+// Classifies pair (t, k) (k < K, t < BS). With CHECK_REPEATS the ids of the
+// same token's earlier k are read again (L1) for the repeat check; without it
+// the caller does that check itself.
+template <bool SPECIAL, bool UNIT, bool CHECK_REPEATS = true>
+__device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, int k) {
+  PairMeta m{kSkip, 0, 1.0f};
+  const size_t tk = static_cast<size_t>(t) * a.K + k;
+  if (!UNIT) m.w = __ldg(a.weights + tk);
+  if (!pair_active(a.mask, a.mask_ndim, t, k, a.K)) return m;
+  if (SPECIAL) {
+    const int32_t* ids = a.topk_idx + static_cast<size_t>(t) * a.K;
+    const int id = __ldg(ids + k);
+    if (id < 0 || id >= a.E + a.Z + a.C + a.Q) return m;
+    if (CHECK_REPEATS)
+      for (int j = 0; j < k; ++j)
+        if (__ldg(ids + j) == id) return m;
+    if (id >= a.E) {
+      m.kind = id < a.E + a.Z ? kZero : id < a.E + a.Z + a.C ? kCopy : kConst;
+      m.row = id - (a.E + a.Z + a.C);
+      return m;
+    }
+  }
+  const int s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
+  if (s >= 0) {
+    m.kind = kRouted;
+    m.row = s;
+  }
+  return m;
+}
+
+// Each warp owns a contiguous span of 32 * U output vectors (8 values each);
+// lane l handles vectors l, l + 32, ... of the span, so every load of the warp
+// is 32 consecutive 16-byte vectors. When a span fits in two tokens' rows
+// (V >= 32 * U), lanes 0..K-1 classify the first token's pairs and lanes
+// 16..16+K-1 the second's, once for the whole span, and every lane takes its
+// token's metadata by shuffle. (Narrower rows: every thread classifies its own
+// token's pairs.) All routed rows' loads are issued before accumulating in
+// ascending k.
+// Resident blocks per SM the forward kernel is compiled for (a register cap
+// that avoids spills for each variant).
+template <int KMAX, bool SPECIAL>
+__host__ __device__ constexpr int fwd_min_blocks() {
+  return SPECIAL ? (KMAX <= 8 ? 3 : 2) : KMAX == 16 ? 2 : KMAX == 4 ? 3 : 4;
+}
+
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool SHARED>
+__global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>()))
+    combine_fwd_kernel(CombineArgs a) {
   constexpr int U = fwd_vectors_per_thread<KMAX>();
   pdl_trigger();
   pdl_wait();
   const int V = a.H / kVecElems;
   const int K = a.K;
   const int n = a.bs * V;
-  const int n_ids = a.E + a.Z + a.C + a.Q;
+  const int lane = threadIdx.x & 31;
+  const int span = blockIdx.x * (kFwdThreads * U) + (threadIdx.x >> 5) * (32 * U);
+  if (span >= n) return;  // warp-uniform
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
-  const int base = blockIdx.x * (kFwdThreads * U) + threadIdx.x;
   uint4 val[U][KMAX];
   int kind[U][KMAX], row[U][KMAX];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int item = base + u * kFwdThreads;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) kind[u][j] = kSkip;
-    if (item >= n) continue;
-    const int t = item / V;
-    const int v = item - t * V;
-    const int32_t* slots = a.assist + static_cast<size_t>(a.A) + static_cast<size_t>(t) * K;
-    int ids[KMAX];
+  float wt[U][KMAX];
+  if (SHARED) {  // the launcher picks SHARED only when V >= 32 * U
+    const int t0 = span / V;
+    const int tm = t0 + (lane >> 4), km = lane & 15;
+    const bool mine = km < K && tm < a.bs;
+    PairMeta m{kSkip, 0, 1.0f};
+    if (mine) m = classify_pair<SPECIAL, UNIT, false>(a, tm, km);
     if (SPECIAL) {
+      // a repeat of an id held by an earlier lane of the same token takes no part
+      const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
+      bool dup = false;
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        ids[j] = j < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + j) : -1;
+      for (int jj = 0; jj < 15; ++jj) {
+        const int other = __shfl_sync(0xFFFFFFFFu, id, (lane & 16) | jj);
+        dup |= jj < km && other == id;
+      }
+      if (dup) m.kind = kSkip;
     }
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j >= K || !pair_active(a.mask, a.mask_ndim, t, j, K)) continue;
-      int kd = kRouted, r = 0;
-      if (SPECIAL) {
-        const int id = ids[j];
-        bool dup = false;
+    for (int u = 0; u < U; ++u) {
+      const int item = span + u * 32 + lane;
+      const int src_base = item / V == t0 ? 0 : 16;
 #pragma unroll
-        for (int jj = 0; jj < j; ++jj) dup |= ids[jj] == id;
-        if (dup || id < 0 || id >= n_ids) continue;
-        if (id >= a.E) {
-          kd = id < a.E + a.Z ? kZero : id < a.E + a.Z + a.C ? kCopy : kConst;
-          r = id - (a.E + a.Z + a.C);
-        }
+      for (int j = 0; j < KMAX; ++j) {
+        kind[u][j] = __shfl_sync(0xFFFFFFFFu, m.kind, src_base + j);
+        row[u][j] = __shfl_sync(0xFFFFFFFFu, m.row, src_base + j);
+        wt[u][j] = UNIT ? 1.0f : __shfl_sync(0xFFFFFFFFu, m.w, src_base + j);
+        if (j >= K || item >= n) kind[u][j] = kSkip;
       }
-      if (kd == kRouted) {
-        const int s = __ldg(slots + j);
-        if (s < 0) continue;
-        val[u][j] = ld_nc_v4(Y + static_cast<size_t>(s) * V + v);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = span + u * 32 + lane;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        kind[u][j] = kSkip;
+        wt[u][j] = 1.0f;
+        if (j >= K || item >= n) continue;
+        const PairMeta m = classify_pair<SPECIAL, UNIT>(a, item / V, j);
+        kind[u][j] = m.kind;
+        row[u][j] = m.row;
+        wt[u][j] = m.w;
       }
-      kind[u][j] = kd;
-      row[u][j] = r;
     }
   }
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    const int item = base + u * kFwdThreads;
+    const int item = span + u * 32 + lane;
+    const int v = item % V;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (kind[u][j] == kRouted) val[u][j] = ld_nc_v4(Y + static_cast<size_t>(row[u][j]) * V + v);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int item = span + u * 32 + lane;
     if (item >= n) continue;
-    const int t = item / V;
-    const int v = item - t * V;
+    const int v = item % V;
     float ori[8];
     if (SPECIAL) {
       bool need = false;
@@ -137,7 +201,7 @@ __global__ void __launch_bounds__(kFwdThreads) combine_fwd_kernel(CombineArgs a)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], m[i]);
       } else {
-        const float w = __ldg(a.weights + static_cast<size_t>(t) * K + j);
+        const float w = wt[u][j];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, m[i]));
       }
@@ -232,10 +296,14 @@ int blocks_per_sm(int threads, size_t smem) {
 template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
 cudaError_t launch_fwd_kmax(const CombineArgs& a, cudaStream_t st) {
   constexpr int U = fwd_vectors_per_thread<KMAX>();
-  const long long n = static_cast<long long>(a.bs) * (a.H / kVecElems);
+  const int V = a.H / kVecElems;
+  const long long n = static_cast<long long>(a.bs) * V;
   const int blocks = static_cast<int>((n + kFwdThreads * U - 1) / (kFwdThreads * U));
-  return launch_pdl(combine_fwd_kernel<T16, KMAX, SPECIAL, UNIT>, dim3(blocks), dim3(kFwdThreads),
-                    0, st, a);
+  if (V >= 32 * U)
+    return launch_pdl(combine_fwd_kernel<T16, KMAX, SPECIAL, UNIT, true>, dim3(blocks),
+                      dim3(kFwdThreads), 0, st, a);
+  return launch_pdl(combine_fwd_kernel<T16, KMAX, SPECIAL, UNIT, false>, dim3(blocks),
+                    dim3(kFwdThreads), 0, st, a);
 }
 
 template <typename T16, bool SPECIAL, bool UNIT>

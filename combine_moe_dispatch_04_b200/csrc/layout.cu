@@ -27,8 +27,21 @@ namespace {
 __device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int (&e)[kMaxK]) {
   const int32_t* row = a.topk_idx + static_cast<size_t>(t) * a.K;
   int ids[kMaxK];
+  if ((a.K & 3) == 0 && (reinterpret_cast<uintptr_t>(a.topk_idx) & 15) == 0) {
+    // rows of a multiple of 4 ids: 16-byte loads
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k) ids[k] = k < a.K ? __ldg(row + k) : -1;
+    for (int q = 0; q < kMaxK / 4; ++q) {
+      int4 v = make_int4(-1, -1, -1, -1);
+      if (4 * q < a.K) v = __ldg(reinterpret_cast<const int4*>(row) + q);
+      ids[4 * q] = v.x;
+      ids[4 * q + 1] = v.y;
+      ids[4 * q + 2] = v.z;
+      ids[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) ids[k] = k < a.K ? __ldg(row + k) : -1;
+  }
   uint32_t st = 0;
 #pragma unroll
   for (int k = 0; k < kMaxK; ++k) {
@@ -209,7 +222,8 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutA
 // Phase 2: the tile's first slot per expert, from the count matrix
 // (prefix over earlier tiles + exclusive scan of the expert totals), then the
 // slots of every pair of the tile and -1 for the unused slots [R, A).
-// Dynamic shared memory: words[kTileWarps][E], base[E], total[E].
+// Dynamic shared memory: words[kTileWarps][E], base[E], total[E], and two
+// [G][E] partial-sum arrays (G * E <= blockDim).
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
   extern __shared__ uint32_t smem[];
   __shared__ int warp_sums[32];
@@ -224,16 +238,46 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
   if (threadIdx.x == 0) status = 0;
   const TileWs ws = tile_ws(a, T);
   const int tile = blockIdx.x;
-  for (int ex = threadIdx.x; ex < E; ex += blockDim.x) {
-    int before = 0, all = 0;
-#pragma unroll 8
-    for (int i = 0; i < T; ++i) {
-      const int c = ws.counts[static_cast<size_t>(i) * E + ex];
-      before += i < tile ? c : 0;
-      all += c;
+  // Sum the count matrix over tiles: G groups of E threads split the tiles
+  // (G = 1 when E >= blockDim), then one thread per expert adds the groups.
+  const int G = E < static_cast<int>(blockDim.x) ? blockDim.x / E : 1;
+  int* part_before = total + E;       // [G][E]
+  int* part_all = part_before + G * E;  // [G][E]
+  if (G > 1) {
+    const int g = threadIdx.x / E, ex = threadIdx.x - g * E;
+    if (g < G) {
+      int before = 0, all = 0;
+#pragma unroll 4
+      for (int i = g; i < T; i += G) {
+        const int c = ws.counts[static_cast<size_t>(i) * E + ex];
+        before += i < tile ? c : 0;
+        all += c;
+      }
+      part_before[g * E + ex] = before;
+      part_all[g * E + ex] = all;
     }
-    base[ex] = before;
-    total[ex] = all;
+    __syncthreads();
+    for (int ex2 = threadIdx.x; ex2 < E; ex2 += blockDim.x) {
+      int before = 0, all = 0;
+      for (int gg = 0; gg < G; ++gg) {
+        before += part_before[gg * E + ex2];
+        all += part_all[gg * E + ex2];
+      }
+      base[ex2] = before;
+      total[ex2] = all;
+    }
+  } else {
+    for (int ex = threadIdx.x; ex < E; ex += blockDim.x) {
+      int before = 0, all = 0;
+#pragma unroll 8
+      for (int i = 0; i < T; ++i) {
+        const int c = ws.counts[static_cast<size_t>(i) * E + ex];
+        before += i < tile ? c : 0;
+        all += c;
+      }
+      base[ex] = before;
+      total[ex] = all;
+    }
   }
   if (blockIdx.x == 0) {
     uint32_t st = 0;
@@ -301,7 +345,7 @@ cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st) {
   }
   const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
   const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
-  const size_t smem_scatter = smem_count + 2u * a.E * sizeof(int);
+  const size_t smem_scatter = smem_count + 2u * a.E * sizeof(int) + 2u * kLayoutTileTokens * sizeof(int);
   cudaError_t err = launch_pdl(layout_count_kernel, dim3(T), dim3(kLayoutTileTokens), smem_count,
                                st, a, T);
   if (err != cudaSuccess) return err;
