@@ -25,7 +25,8 @@ MOE_DEV_BAD_ID, MOE_DEV_DUP_ID = 1, 2
 EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_layout_workspace_bytes", "moe_dispatch_layout", "moe_dispatch_permute",
            "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd",
-           "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes")
+           "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes",
+           "moe_combine_fwd_comm_quant")
 
 
 class MoeShape(ctypes.Structure):
@@ -46,7 +47,7 @@ class MoeError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m combine_moe_dispatch_04_b200.build`"
+            f"{LIB_PATH} is missing: build it with `python combine_moe_dispatch_04_b200/build.py`"
             " (there is no fallback implementation)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(MoeShape)
@@ -58,13 +59,15 @@ def _load():
     L.moe_dispatch_layout.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_dispatch_permute.argtypes = [S, P, P, P, I, P, P, P]
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
+    L.moe_combine_fwd_comm_quant.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P]
     L.moe_combine_bwd.argtypes = [S, P, P, P, P, P, P, P, P, P]
     L.moe_dispatch_bwd.argtypes = [S, P, P, P, P, P]
     L.moe_dispatch_layout_noalloc.argtypes = [S, P, P, P, P, P, P, P]
     L.moe_layout_noalloc_max_workspace_bytes.argtypes = []
     L.moe_layout_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
-              "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc"):
+              "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
+              "moe_combine_fwd_comm_quant"):
         getattr(L, n).restype = I
     return L
 
@@ -82,6 +85,7 @@ moe_combine_fwd = _lib.moe_combine_fwd
 moe_combine_bwd = _lib.moe_combine_bwd
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
 moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
+moe_combine_fwd_comm_quant = _lib.moe_combine_fwd_comm_quant
 moe_layout_noalloc_max_workspace_bytes = _lib.moe_layout_noalloc_max_workspace_bytes
 
 
@@ -211,16 +215,20 @@ def dispatch_permute(shape: Shape, x, layout: Layout, comm_quant_mode: int = 0, 
 
 def combine_fwd(shape: Shape, expand_x, topk_idx, topk_weights, layout: Layout, *,
                 x_active_mask=None, shared_expert_x=None, ori_x=None, const_alpha_1=None,
-                const_alpha_2=None, const_v=None, out=None, stream=None):
+                const_alpha_2=None, const_v=None, comm_quant_mode=0, out=None, stream=None):
     import torch
 
     if out is None:
         out = torch.empty(shape.bs, shape.h, dtype=_torch_dtype(shape), device=expand_x.device)
-    _check("moe_combine_fwd", moe_combine_fwd(
-        ctypes.byref(shape.c()), _ptr(expand_x), _ptr(topk_idx), _ptr(topk_weights),
-        _ptr(layout.assist_info), _ptr(layout.ep_send_counts), _ptr(x_active_mask),
-        _ptr(shared_expert_x), _ptr(ori_x), _ptr(const_alpha_1), _ptr(const_alpha_2),
-        _ptr(const_v), _ptr(out), _stream(stream)))
+    args = (ctypes.byref(shape.c()), _ptr(expand_x), _ptr(topk_idx), _ptr(topk_weights),
+            _ptr(layout.assist_info), _ptr(layout.ep_send_counts), _ptr(x_active_mask),
+            _ptr(shared_expert_x), _ptr(ori_x), _ptr(const_alpha_1), _ptr(const_alpha_2),
+            _ptr(const_v))
+    if comm_quant_mode == 0:
+        _check("moe_combine_fwd", moe_combine_fwd(*args, _ptr(out), _stream(stream)))
+    else:
+        _check("moe_combine_fwd_comm_quant", moe_combine_fwd_comm_quant(
+            *args, comm_quant_mode, _ptr(out), _stream(stream)))
     return out
 
 

@@ -1,6 +1,8 @@
 """Builds libmoe_dc.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m combine_moe_dispatch_04_b200.build [--verbose]
+    python combine_moe_dispatch_04_b200/build.py [--verbose]
+
+Run it as a script (or load it by path): importing the package needs the library.
 """
 from __future__ import annotations
 

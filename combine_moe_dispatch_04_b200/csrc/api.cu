@@ -145,7 +145,20 @@ moe_status moe_combine_fwd(const moe_shape* s, const void* expand_x, const int32
                            const void* shared_expert_x, const void* ori_x,
                            const void* const_alpha_1, const void* const_alpha_2,
                            const void* const_v, void* out, void* stream) {
+  return moe_combine_fwd_comm_quant(s, expand_x, topk_idx, topk_weights, assist_info,
+                                    ep_send_counts, x_active_mask, shared_expert_x, ori_x,
+                                    const_alpha_1, const_alpha_2, const_v, 0, out, stream);
+}
+
+moe_status moe_combine_fwd_comm_quant(const moe_shape* s, const void* expand_x,
+                                      const int32_t* topk_idx, const float* topk_weights,
+                                      const int32_t* assist_info, const int32_t* ep_send_counts,
+                                      const uint8_t* x_active_mask, const void* shared_expert_x,
+                                      const void* ori_x, const void* const_alpha_1,
+                                      const void* const_alpha_2, const void* const_v,
+                                      int comm_quant_mode, void* out, void* stream) {
   (void)ep_send_counts;
+  if (comm_quant_mode != 0 && comm_quant_mode != 2) return MOE_ERR_ARG;
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
   if ((st = check_mask(s, x_active_mask)) != MOE_OK) return st;
@@ -186,7 +199,9 @@ moe_status moe_combine_fwd(const moe_shape* s, const void* expand_x, const int32
   a.C = s->copy_expert_num;
   a.Q = s->const_expert_num;
   a.dtype = s->dtype;
-  return cuda_status(moe::launch_combine_fwd(a, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return cuda_status(comm_quant_mode == 2 ? moe::launch_combine_fwd_q8(a, cs)
+                                          : moe::launch_combine_fwd(a, cs));
 }
 
 moe_status moe_combine_bwd(const moe_shape* s, const void* grad_out, const void* expand_x,

@@ -216,6 +216,93 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
   }
 }
 
+// ---------------------------------------------------------------------------
+// Combine forward with comm_quant_mode 2 ([combine] Parameters): every routed
+// row returns through the per-row int8 round trip (scale = max|y| / 127 in
+// fp32, q = clamp(rne(y / scale), -127, 127), value = q * scale) before the
+// same weighted fp32 sum. One CTA per token, thread i owning vectors
+// i, i + blockDim, ... of each row. Pass 1 reads the token's routed rows
+// (through L1) and reduces each row's max|y| (shuffle + shared memory; a max
+// does not depend on order); pass 2 reads them again, dequantises and
+// accumulates in ascending k.
+template <typename T16, int KMAX, bool SPECIAL>
+__global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
+  __shared__ PairMeta meta[KMAX];
+  __shared__ float red[32][KMAX];
+  __shared__ float rmax[KMAX];
+  pdl_trigger();
+  pdl_wait();
+  const int V = a.H / kVecElems;
+  const int K = a.K;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const uint4* Y = static_cast<const uint4*>(a.expand_x);
+  for (int t = blockIdx.x; t < a.bs; t += gridDim.x) {
+    if (threadIdx.x < K) meta[threadIdx.x] = classify_pair<SPECIAL, false>(a, t, threadIdx.x);
+    __syncthreads();
+    for (int j = 0; j < K; ++j) {  // meta is block-uniform: no divergence around the shuffles
+      if (meta[j].kind != kRouted) continue;
+      float mx = 0.0f;
+      for (int v = threadIdx.x; v < V; v += blockDim.x) {
+        float f[8];
+        widen8<T16>(__ldg(Y + static_cast<size_t>(meta[j].row) * V + v), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(f[i]));
+      }
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+      if (lane == 0) red[warp][j] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x < K && meta[threadIdx.x].kind == kRouted) {
+      float mx = 0.0f;
+      for (int w = 0; w < nwarps; ++w) mx = fmaxf(mx, red[w][threadIdx.x]);
+      rmax[threadIdx.x] = mx;
+    }
+    __syncthreads();
+    bool need_ori = false;
+    if (SPECIAL)
+      for (int j = 0; j < K; ++j) need_ori |= meta[j].kind == kCopy || meta[j].kind == kConst;
+    for (int v = threadIdx.x; v < V; v += blockDim.x) {
+      const size_t item = static_cast<size_t>(t) * V + v;
+      float ori[8];
+      if (SPECIAL && need_ori) widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      for (int j = 0; j < K; ++j) {
+        const PairMeta pm = meta[j];
+        if (pm.kind == kSkip) continue;
+        float m[8];
+        if (pm.kind == kRouted) {
+          const float mx = rmax[j];
+          float y[8];
+          widen8<T16>(__ldg(Y + static_cast<size_t>(pm.row) * V + v), y);
+          const float scale = __fdiv_rn(mx, 127.0f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float q = mx == 0.0f ? 0.0f : rintf(__fdiv_rn(y[i], scale));
+            q = fminf(127.0f, fmaxf(-127.0f, q));
+            m[i] = __fmul_rn(q, scale);
+          }
+        } else {
+          pair_values<T16, SPECIAL>(a, pm.kind, pm.row, V, v, make_uint4(0, 0, 0, 0), ori, m);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(pm.w, m[i]));
+      }
+      if (a.shared != nullptr) {
+        float sh[8];
+        widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], sh[i]);
+      }
+      st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
+    }
+    __syncthreads();  // meta, red and rmax are reused by the next token
+  }
+}
+
 constexpr int kBwdThreads = 256;
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kBwdUnroll = 4;
@@ -321,11 +408,37 @@ cudaError_t launch_fwd_t(const CombineArgs& a, cudaStream_t st) {
   return launch_fwd_k<T16, false, false>(a, st);
 }
 
+template <typename T16, bool SPECIAL>
+cudaError_t launch_fwd_q8_t(const CombineArgs& a, cudaStream_t st) {
+  const int V = a.H / kVecElems;
+  const int threads = V < 256 ? (V + 31) / 32 * 32 : 256;
+  const int cap = sm_count() * (2048 / threads);
+  const int blocks = a.bs < cap ? a.bs : cap;
+  if (a.K <= 2)
+    return launch_pdl(combine_fwd_q8_kernel<T16, 2, SPECIAL>, dim3(blocks), dim3(threads), 0, st, a);
+  if (a.K <= 4)
+    return launch_pdl(combine_fwd_q8_kernel<T16, 4, SPECIAL>, dim3(blocks), dim3(threads), 0, st, a);
+  if (a.K <= 8)
+    return launch_pdl(combine_fwd_q8_kernel<T16, 8, SPECIAL>, dim3(blocks), dim3(threads), 0, st, a);
+  return launch_pdl(combine_fwd_q8_kernel<T16, 16, SPECIAL>, dim3(blocks), dim3(threads), 0, st, a);
+}
+
+template <typename T16>
+cudaError_t launch_fwd_q8(const CombineArgs& a, cudaStream_t st) {
+  if (a.Z + a.C + a.Q > 0) return launch_fwd_q8_t<T16, true>(a, st);
+  return launch_fwd_q8_t<T16, false>(a, st);
+}
+
 }  // namespace
 
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
   return a.dtype == MOE_BF16 ? launch_fwd_t<Bf16>(a, st) : launch_fwd_t<Fp16>(a, st);
+}
+
+cudaError_t launch_combine_fwd_q8(const CombineArgs& a, cudaStream_t st) {
+  if (a.bs == 0) return cudaSuccess;
+  return a.dtype == MOE_BF16 ? launch_fwd_q8<Bf16>(a, st) : launch_fwd_q8<Fp16>(a, st);
 }
 
 cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st) {

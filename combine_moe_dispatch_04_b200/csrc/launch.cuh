@@ -53,6 +53,8 @@ struct CombineArgs {
   int bs, K, H, A, E, Z, C, Q, dtype;
 };
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st);
+// comm_quant_mode 2: every routed row through the per-row int8 round trip (H <= 16384).
+cudaError_t launch_combine_fwd_q8(const CombineArgs& a, cudaStream_t st);
 
 struct CombineBwdArgs {
   const void* grad_out;

@@ -157,6 +157,24 @@ moe_status moe_combine_fwd(const moe_shape* shape, const void* expand_x,
                            void* stream);
 
 /*
+ * moe_combine_fwd_comm_quant — moe_combine_fwd with the combine side's
+ * comm_quant_mode ([combine] Parameters: 0 no quantisation, 2 int8
+ * quantisation of the communicated rows). At one device the expert-output
+ * rows do not travel, so mode 2 is the round trip each routed row would make:
+ * scale = max_h |y[s, h]| / 127 (fp32, IEEE division), q = clamp(rne(y / scale),
+ * -127, 127), and the weighted sum uses the fp32 value q * scale (an all-zero
+ * row contributes 0). Copy/const experts and shared_expert_x are local and are
+ * not quantised. Mode 0 is exactly moe_combine_fwd. Other arguments as there.
+ */
+moe_status moe_combine_fwd_comm_quant(const moe_shape* shape, const void* expand_x,
+                                      const int32_t* topk_idx, const float* topk_weights,
+                                      const int32_t* assist_info, const int32_t* ep_send_counts,
+                                      const uint8_t* x_active_mask, const void* shared_expert_x,
+                                      const void* ori_x, const void* const_alpha_1,
+                                      const void* const_alpha_2, const void* const_v,
+                                      int comm_quant_mode, void* out, void* stream);
+
+/*
  * moe_combine_bwd — gradient of the combine Formula for routed pairs (the
  * fused EP MoE layer of the Triton-distributed ep_moe_fused PR has a backward):
  *   grad_expand[slot(t,k)] = round16(w[t,k] * grad_out[t])     (fp32 product)

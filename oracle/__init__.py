@@ -55,7 +55,7 @@ def lib():
         L.oracle_dispatch_permute_quant.argtypes = [i, i, i, i, i, P, P, P, P]
         L.oracle_dispatch_permute_quant.restype = None
         L.oracle_combine_fwd.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, i,
-                                         P, P, P, P, P, P]
+                                         P, P, P, P, P, i, P]
         L.oracle_combine_fwd.restype = None
         L.oracle_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, i, P, P, P]
         L.oracle_combine_bwd.restype = None
@@ -134,7 +134,8 @@ def dispatch_permute_quant(x, assist_info, k, a_capacity, dtype):
 
 def combine_fwd(expand_x, topk_idx, topk_weights, assist_info, *, num_experts, a_capacity,
                 dtype, zero_expert_num=0, copy_expert_num=0, const_expert_num=0,
-                mask=None, shared=None, ori_x=None, alpha1=None, alpha2=None, const_v=None):
+                mask=None, shared=None, ori_x=None, alpha1=None, alpha2=None, const_v=None,
+                comm_quant_mode=0):
     idx = _c(topk_idx, np.int32)
     bs, k = idx.shape
     ex = _c(expand_x, np.uint16)
@@ -146,7 +147,8 @@ def combine_fwd(expand_x, topk_idx, topk_weights, assist_info, *, num_experts, a
     lib().oracle_combine_fwd(bs, k, h, num_experts, zero_expert_num, copy_expert_num,
                              const_expert_num, a_capacity, DTYPE_CODES[dtype], _p(ex), _p(idx),
                              _p(_c(topk_weights, np.float32)), _p(_c(assist_info, np.int32)),
-                             _p(m), 0 if m is None else m.ndim, *[_p(a) for a in args], _p(out))
+                             _p(m), 0 if m is None else m.ndim, *[_p(a) for a in args],
+                             comm_quant_mode, _p(out))
     return out
 
 

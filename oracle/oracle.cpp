@@ -39,6 +39,10 @@
 //   R10 an id outside [0, N) or a repeat of an id earlier in its row makes the
 //      pair invalid: it is flagged in the status word and takes no part.
 //   R11 grad_w of a pair without a slot (masked, invalid or special) is 0.
+//   R15 combine with comm_quant_mode 2: each expanded row that returns to its
+//      token is quantised as in R9 (per row, scale = max|y| / 127) and used as
+//      the fp32 value q * scale; special experts and shared_expert_x are local
+//      and are not quantised.
 
 #include <cfenv>
 #include <cmath>
@@ -229,18 +233,31 @@ void oracle_dispatch_permute_quant(int bs, int K, int h, int a_capacity, int dty
   }
 }
 
+// Per-row int8 round trip of R9/R15: the fp32 value q * scale of element j.
+static float int8_roundtrip(const uint16_t* row, int h, int j, int dtype) {
+  float amax = 0.0f;
+  for (int i = 0; i < h; ++i) amax = std::max(amax, std::fabs(load16(row, i, dtype)));
+  if (amax == 0.0f) return 0.0f;
+  const float scale = amax / 127.0f;
+  float q = std::nearbyint(load16(row, j, dtype) / scale);
+  q = std::min(127.0f, std::max(-127.0f, q));
+  return q * scale;
+}
+
 // Combine forward. [combine] Function (Formula: weighted sum of the returned
 // rows plus shared_expert_x; special expert use cases: zero, copy, const),
 // Parameters (topk_weights, x_active_mask, shared_expert_x, ori_x,
-// const_expert_alpha_1/2, const_expert_v), Return Value. Readings R1, R2, R4,
-// R8, R10. fp32, product and sum rounded separately, k ascending.
+// const_expert_alpha_1/2, const_expert_v, comm_quant_mode), Return Value.
+// Readings R1, R2, R4, R8, R10, R15. fp32, product and sum rounded
+// separately, k ascending.
 void oracle_combine_fwd(int bs, int K, int h, int num_experts, int zero_num, int copy_num,
                         int const_num, int a_capacity, int dtype, const uint16_t* expand_x,
                         const int32_t* topk_idx, const float* topk_weights,
                         const int32_t* assist_info, const uint8_t* mask, int mask_ndim,
                         const uint16_t* shared_x, const uint16_t* ori_x,
                         const uint16_t* alpha1, const uint16_t* alpha2,
-                        const uint16_t* const_v, uint16_t* out) {
+                        const uint16_t* const_v, int comm_quant_mode, uint16_t* out) {
+  std::fesetround(FE_TONEAREST);
   const size_t A = static_cast<size_t>(a_capacity);
   const int n_ids = num_experts + zero_num + copy_num + const_num;
   const int zero_end = num_experts + zero_num;
@@ -257,7 +274,9 @@ void oracle_combine_fwd(int bs, int K, int h, int num_experts, int zero_num, int
         if (id < num_experts) {
           int32_t s = assist_info[A + static_cast<size_t>(t) * K + k];
           if (s < 0) continue;
-          m = load16(expand_x, static_cast<size_t>(s) * h + j, dtype);
+          m = comm_quant_mode == 2
+                  ? int8_roundtrip(expand_x + static_cast<size_t>(s) * h, h, j, dtype)
+                  : load16(expand_x, static_cast<size_t>(s) * h + j, dtype);
         } else if (id < zero_end) {
           m = 0.0f;
         } else if (id < copy_end) {

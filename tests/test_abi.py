@@ -97,6 +97,9 @@ def test_other_entry_points_check_first():
     args[7] = p  # ori_x
     args[8] = None  # alpha_1 missing
     assert moe.moe_combine_fwd(ctypes.byref(sp.c()), *args) == moe.MOE_ERR_ARG
+    # combine comm_quant_mode outside {0, 2}
+    args2 = [p, p, p, p, None, None, None, None, None, None, None]
+    assert moe.moe_combine_fwd_comm_quant(s, *args2, 1, p, None) == moe.MOE_ERR_ARG
     assert moe.moe_combine_bwd(s, None, p, None, p, p, None, p, p, None) == moe.MOE_ERR_ARG
     assert moe.moe_dispatch_bwd(s, p, None, None, p, None) == moe.MOE_ERR_ARG
 

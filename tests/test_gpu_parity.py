@@ -104,3 +104,52 @@ def test_all_tokens_one_expert():
     inp = workloads.generate(wl)
     inp["topk_idx"] = np.full((wl.bs, 1), 2, np.int32)
     _chain().run_compare(inp)
+
+
+COMM_QUANT = [
+    W["special"].scaled(bs=1500, h=1040, name="special_q8"),
+    W["uniform"].scaled(bs=2100, h=520, name="uniform_q8"),
+    W["mixtral"].scaled(bs=1200, h=264, name="mixtral_fp16_mask_q8"),
+    W["dsv3"].scaled(bs=300, h=7168, name="dsv3_shared_q8"),
+    _custom("k16_q8", bs=700, k=16, num_experts=40, h=136, zero_expert_num=2,
+            const_expert_num=2, backward=False),
+    W["special"],  # full size
+]
+
+
+@pytest.mark.parametrize("wl", COMM_QUANT, ids=lambda w: w.name)
+def test_combine_comm_quant_mode2(wl):
+    """Combine with comm_quant_mode 2 (per-row int8 round trip of the returning
+    rows) against the oracle on the same expert outputs."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    inp = workloads.generate(wl)
+    dt = wl.dtype
+    _, send, assist, st = oracle.dispatch_layout(inp["topk_idx"], wl.num_experts, wl.n_ids,
+                                                 wl.a_capacity, inp["mask"])
+    rng = np.random.default_rng(5)
+    y = workloads.encode16(rng.standard_normal((wl.a_capacity, wl.h)) *
+                           rng.uniform(0.01, 10, (wl.a_capacity, 1)), dt)
+    y[:3] = 0  # all-zero rows: scale 0
+    want = oracle.combine_fwd(y, inp["topk_idx"], inp["topk_weights"], assist,
+                              num_experts=wl.num_experts, a_capacity=wl.a_capacity, dtype=dt,
+                              zero_expert_num=wl.zero_expert_num,
+                              copy_expert_num=wl.copy_expert_num,
+                              const_expert_num=wl.const_expert_num, mask=inp["mask"],
+                              shared=inp["shared"], ori_x=inp["ori_x"], alpha1=inp["alpha1"],
+                              alpha2=inp["alpha2"], const_v=inp["v"], comm_quant_mode=2)
+    sh = gpu_chain.shape_of(wl)
+    dev = gpu_chain.dev
+    lay = moe.dispatch_layout(sh, dev(inp["topk_idx"]), dev(inp["mask"]))
+    out = moe.combine_fwd(sh, dev(y, dt), dev(inp["topk_idx"]), dev(inp["topk_weights"]), lay,
+                          x_active_mask=dev(inp["mask"]), shared_expert_x=dev(inp["shared"], dt),
+                          ori_x=dev(inp["ori_x"], dt), const_alpha_1=dev(inp["alpha1"], dt),
+                          const_alpha_2=dev(inp["alpha2"], dt), const_v=dev(inp["v"], dt),
+                          comm_quant_mode=2)
+    torch.cuda.synchronize()
+    got = gpu_chain.host(out)
+    d = gpu_chain.ulp_dist(got, want)
+    assert d.max() <= gpu_chain.ULP_TOL
+    assert (d == 0).mean() == 1.0  # same fp32 operations in the same order

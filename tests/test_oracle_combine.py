@@ -245,3 +245,46 @@ def test_chain_runs_on_every_workload_shape():
         assert r["out"].shape == (48, 32)
         if small.backward:
             assert r["grad_x"].shape == (48, 32)
+
+
+def test_int8_roundtrip_hand_case():
+    g = read("combine_int8_roundtrip.txt")
+    y = workloads.encode16(np.array(g["y"], np.float32), g["dtype"])
+    bs = len(y)
+    idx = np.zeros((bs, 1), np.int32)
+    assist, _ = _layout(idx, 1, 1, bs)
+    out = oracle.combine_fwd(y, idx, np.ones((bs, 1), np.float32), assist, num_experts=1,
+                             a_capacity=bs, dtype=g["dtype"], comm_quant_mode=2)
+    assert np.array_equal(out, workloads.encode16(np.array(g["out"], np.float32), g["dtype"]))
+
+
+def test_int8_roundtrip_exact_rows_and_bound():
+    rng = np.random.default_rng(41)
+    bs, h = 64, 48
+    # rows of integers with max |y| = 127: scale 1, the round trip is exact
+    yi = rng.integers(-127, 128, (bs, h)).astype(np.float32)
+    yi[:, 0] = 127.0
+    y_exact = workloads.encode16(yi, "bf16")
+    idx = np.zeros((bs, 1), np.int32)
+    assist, _ = _layout(idx, 1, 1, bs)
+    w1 = np.ones((bs, 1), np.float32)
+    kw = dict(num_experts=1, a_capacity=bs, dtype="bf16")
+    assert np.array_equal(oracle.combine_fwd(y_exact, idx, w1, assist, comm_quant_mode=2, **kw),
+                          y_exact)
+    # general rows: within half a quantisation step (plus the bf16 rounding)
+    y = workloads.encode16(rng.standard_normal((bs, h)) * 3, "bf16")
+    yf = workloads.decode16(y, "bf16").astype(np.float64)
+    got = workloads.decode16(oracle.combine_fwd(y, idx, w1, assist, comm_quant_mode=2, **kw),
+                             "bf16").astype(np.float64)
+    step = np.abs(yf).max(axis=1, keepdims=True) / 127
+    assert np.all(np.abs(got - yf) <= step / 2 + np.abs(got) * 2.0**-8 + 1e-30)
+    assert not np.array_equal(got, yf)  # the round trip does change some values
+
+
+def test_int8_roundtrip_leaves_local_terms_alone():
+    # copy/const experts and shared_expert_x are not communicated: unchanged by mode 2
+    d = _random_case("bf16", k=2, e=2, z=1, c=1, q=1, seed=8)
+    bs = d["bs"]
+    d["idx"] = np.tile(np.array([[3, 4]], np.int32), (bs, 1))  # copy + const only
+    d["assist"], _ = _layout(d["idx"], 2, 5, bs * 2)
+    assert np.array_equal(_combine(d, "bf16", comm_quant_mode=2), _combine(d, "bf16"))

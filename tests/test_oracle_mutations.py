@@ -47,6 +47,9 @@ MUTATIONS = [
     ("mask_ignored_in_layout",
      "      if (!pair_active(mask, mask_ndim, t, k, K)) continue;\n      if (row[k] >= num_experts)",
      "      if (row[k] >= num_experts)"),
+    ("int8_roundtrip_skipped",
+     "  if (amax == 0.0f) return 0.0f;\n  const float scale = amax / 127.0f;",
+     "  if (amax >= 0.0f) return load16(row, j, dtype);\n  const float scale = amax / 127.0f;"),
     ("duplicate_ids_accepted",
      "    if (row[j] == id) return ST_DUP_ID;", "    if (false) return ST_DUP_ID;"),
 ]
