@@ -166,10 +166,16 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {"layout": "layout.cu", "dispatch": "layout.cu", "permute": "permute.cu",
+                  "combine_fwd": "combine.cu",
+                  "combine_bwd": "combine.cu", "dispatch_bwd": "combine.cu"}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the source file that defines `kernel` and of the shared device helpers."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_moe_dispatch_04_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in (KERNEL_SOURCES[kernel], "common.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -177,7 +183,7 @@ def kernel_source_hash() -> str:
 
 def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources; else None."""
+    current sources of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
@@ -185,7 +191,7 @@ def profiled_traffic(kernel: str, workload: str):
     except (OSError, ValueError):
         return None
     ent = rec.get(workload, {}).get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -288,6 +294,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="moe", choices=["moe", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--fused-dispatch", action="store_true",
+                    help="layout + permute through the single moe_dispatch call")
+    ap.add_argument("--combine-comm-quant", type=int, default=0, choices=[0, 2],
+                    help="combine forward with comm_quant_mode 2 (int8 round trip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -365,15 +375,26 @@ def main():
     bytes_per = byte_model(wl, r, ori_tokens)
     kernels = [k for k in KERNELS if k in bytes_per]
 
-    calls = [
-        ("layout", lambda: moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws,
-                                               out=lay, stream=stream)),
-        ("permute", lambda: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
-                                                 dynamic_scales=scales, stream=stream)),
+    cq = args.combine_comm_quant
+    if args.fused_dispatch:
+        calls = [("dispatch", lambda: moe.dispatch(
+            sh, d["topk_idx"], d["x"], x_active_mask=d["mask"], comm_quant_mode=qm,
+            workspace=ws, layout=lay, expand_x=expand, dynamic_scales=scales, stream=stream))]
+        bytes_per["dispatch"] = bytes_per.pop("layout") + bytes_per.pop("permute")
+        kernels = ["dispatch"] + [k for k in kernels if k not in ("layout", "permute")]
+    else:
+        calls = [
+            ("layout", lambda: moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws,
+                                                   out=lay, stream=stream)),
+            ("permute", lambda: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
+                                                     dynamic_scales=scales, stream=stream)),
+        ]
+    calls += [
         ("combine_fwd", lambda: moe.combine_fwd(
             sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
             shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
-            const_alpha_2=d["alpha2"], const_v=d["v"], out=out, stream=stream)),
+            const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, out=out,
+            stream=stream)),
     ]
     if wl.backward:
         calls += [
@@ -384,7 +405,8 @@ def main():
                                                       grad_x=gx, stream=stream)),
         ]
     # the kernel that moves the most bytes; the timed steps bracket it with events
-    dominant = max((k for k in kernels if k != "layout"), key=lambda k: bytes_per[k])
+    dominant = max((k for k in kernels if k not in ("layout", "dispatch")),
+                   key=lambda k: bytes_per[k])
 
     def step(marks=None):
         """One pass of the path. `marks` maps "start"/"end" to an event and kernel
@@ -409,7 +431,11 @@ def main():
         return m
 
     tiled = wl.bs > moe_layout_small_max_tokens()
-    launches_per_step = (2 if tiled else 1) + 2 + (2 if wl.backward else 0)
+    if args.fused_dispatch and not tiled and qm == 0:
+        dispatch_launches = 1
+    else:
+        dispatch_launches = (2 if tiled else 1) + 1
+    launches_per_step = dispatch_launches + 1 + (2 if wl.backward else 0)
 
     # L2 flush between steps: write a buffer twice the size of L2
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
@@ -516,6 +542,8 @@ def main():
             "config": {"workload": wl.name, "bs": wl.bs, "h": wl.h, "k": wl.k,
                        "num_experts": wl.num_experts, "routed_pairs": r,
                        "a_capacity": wl.a_capacity, "parallelism": "replicas",
+                       "fused_dispatch": bool(args.fused_dispatch),
+                       "combine_comm_quant_mode": cq,
                        "l2": "flushed before every step (write of 2x L2), outside the step events"},
             "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
             "hbm_frac_of_measured": round(gbs / peak, 4),

@@ -26,7 +26,7 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_layout_workspace_bytes", "moe_dispatch_layout", "moe_dispatch_permute",
            "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd",
            "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes",
-           "moe_combine_fwd_comm_quant")
+           "moe_combine_fwd_comm_quant", "moe_dispatch")
 
 
 class MoeShape(ctypes.Structure):
@@ -60,6 +60,7 @@ def _load():
     L.moe_dispatch_permute.argtypes = [S, P, P, P, I, P, P, P]
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_combine_fwd_comm_quant.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P]
+    L.moe_dispatch.argtypes = [S, P, P, P, I, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_combine_bwd.argtypes = [S, P, P, P, P, P, P, P, P, P]
     L.moe_dispatch_bwd.argtypes = [S, P, P, P, P, P]
     L.moe_dispatch_layout_noalloc.argtypes = [S, P, P, P, P, P, P, P]
@@ -67,7 +68,7 @@ def _load():
     L.moe_layout_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
               "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
-              "moe_combine_fwd_comm_quant"):
+              "moe_combine_fwd_comm_quant", "moe_dispatch"):
         getattr(L, n).restype = I
     return L
 
@@ -86,6 +87,7 @@ moe_combine_bwd = _lib.moe_combine_bwd
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
 moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
 moe_combine_fwd_comm_quant = _lib.moe_combine_fwd_comm_quant
+moe_dispatch = _lib.moe_dispatch
 moe_layout_noalloc_max_workspace_bytes = _lib.moe_layout_noalloc_max_workspace_bytes
 
 
@@ -195,6 +197,35 @@ def dispatch_layout_noalloc(shape: Shape, topk_idx, x_active_mask=None, *, out: 
         ctypes.byref(shape.c()), _ptr(topk_idx), _ptr(x_active_mask), _ptr(out.expert_token_nums),
         _ptr(out.ep_send_counts), _ptr(out.assist_info), _ptr(out.dev_status), _stream(stream)))
     return out
+
+
+def dispatch(shape: Shape, topk_idx, x, x_active_mask=None, comm_quant_mode: int = 0, *,
+             workspace=None, layout: Layout | None = None, expand_x=None, dynamic_scales=None,
+             stream=None):
+    """Layout and permute in one call (one launch for BS <= 1024 without quantisation).
+    Returns (layout, expand_x, dynamic_scales)."""
+    import torch
+
+    dev = topk_idx.device
+    if layout is None:
+        layout = Layout(torch.empty(shape.num_experts, dtype=torch.int32, device=dev),
+                        torch.empty(shape.num_experts + 1, dtype=torch.int32, device=dev),
+                        torch.empty(shape.A + shape.bs * shape.k, dtype=torch.int32, device=dev),
+                        torch.empty(1, dtype=torch.int32, device=dev))
+    if expand_x is None:
+        dt = torch.int8 if comm_quant_mode == 2 else _torch_dtype(shape)
+        expand_x = torch.empty(shape.A, shape.h, dtype=dt, device=dev)
+    if comm_quant_mode == 2 and dynamic_scales is None:
+        dynamic_scales = torch.empty(shape.A, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = layout_workspace(shape, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("moe_dispatch", moe_dispatch(
+        ctypes.byref(shape.c()), _ptr(topk_idx), _ptr(x_active_mask), _ptr(x), comm_quant_mode,
+        _ptr(layout.expert_token_nums), _ptr(layout.ep_send_counts), _ptr(layout.assist_info),
+        _ptr(layout.dev_status), _ptr(expand_x), _ptr(dynamic_scales), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+    return layout, expand_x, dynamic_scales
 
 
 def dispatch_permute(shape: Shape, x, layout: Layout, comm_quant_mode: int = 0, *,

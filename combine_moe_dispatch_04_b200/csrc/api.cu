@@ -139,6 +139,45 @@ moe_status moe_dispatch_permute(const moe_shape* s, const void* x, const int32_t
   return cuda_status(moe::launch_permute(a, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_dispatch(const moe_shape* s, const int32_t* topk_idx, const uint8_t* x_active_mask,
+                        const void* x, int comm_quant_mode, int32_t* expert_token_nums,
+                        int32_t* ep_send_counts, int32_t* assist_info, uint32_t* dev_status,
+                        void* expand_x, float* dynamic_scales, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  const bool fused = comm_quant_mode == 0 && s->bs <= moe::kLayoutSmallMaxTokens;
+  if (!fused) {
+    st = moe_dispatch_layout(s, topk_idx, x_active_mask, expert_token_nums, ep_send_counts,
+                             assist_info, dev_status, workspace, workspace_bytes, stream);
+    if (st != MOE_OK) return st;
+    return moe_dispatch_permute(s, x, assist_info, ep_send_counts, comm_quant_mode, expand_x,
+                                dynamic_scales, stream);
+  }
+  if ((st = check_mask(s, x_active_mask)) != MOE_OK) return st;
+  if ((s->bs > 0 && (topk_idx == nullptr || x == nullptr || expand_x == nullptr)) ||
+      expert_token_nums == nullptr || ep_send_counts == nullptr ||
+      (moe_assist_info_elems(s) > 0 && assist_info == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(expand_x)) return MOE_ERR_ALIGN;
+  moe::LayoutArgs a;
+  a.topk_idx = topk_idx;
+  a.mask = x_active_mask;
+  a.mask_ndim = s->mask_ndim;
+  a.bs = s->bs;
+  a.K = s->k;
+  a.E = s->num_experts;
+  a.N = s->num_experts + s->zero_expert_num + s->copy_expert_num + s->const_expert_num;
+  a.A = s->a_capacity;
+  a.expert_token_nums = expert_token_nums;
+  a.ep_send_counts = ep_send_counts;
+  a.assist = assist_info;
+  a.dev_status = dev_status;
+  a.workspace = nullptr;
+  return cuda_status(
+      moe::launch_dispatch_small(a, x, expand_x, s->h, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_combine_fwd(const moe_shape* s, const void* expand_x, const int32_t* topk_idx,
                            const float* topk_weights, const int32_t* assist_info,
                            const int32_t* ep_send_counts, const uint8_t* x_active_mask,

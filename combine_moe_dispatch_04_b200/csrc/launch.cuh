@@ -37,6 +37,10 @@ struct PermuteArgs {
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
 
+// Layout and the plain (no quantisation) permute in one launch, BS <= kLayoutSmallMaxTokens.
+cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                  cudaStream_t st);
+
 struct CombineArgs {
   const void* expand_x;  // (A, H): expert outputs, or slot gradients for dispatch bwd
   const int32_t* topk_idx;

@@ -175,6 +175,83 @@ __global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Fused dispatch for BS <= 1024 (layout + permute in one launch). Every CTA
+// rebuilds the whole layout in shared memory exactly as layout_small_kernel
+// does (the ids are at most 64 KB and sit in L2), CTA 0 alone writes the
+// layout's outputs, and CTA c copies the rows of tokens [c * per, (c+1) * per)
+// to their slots: one thread per 16-byte vector, read once, stored K times.
+// Dynamic shared memory: words[32][E].
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, const uint4* x,
+                                                              uint4* expand_x, int V, int per) {
+  extern __shared__ uint32_t words[];
+  __shared__ int offs[1024];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t status;
+  __shared__ int slot_sh[kLayoutSmallMaxTokens / 8][kMaxK];  // slots of this CTA's tokens
+  pdl_trigger();
+  pdl_wait();
+  const int E = a.E;
+  const bool writer = blockIdx.x == 0;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) words[i] = 0;
+  if (threadIdx.x == 0) status = 0;
+  __syncthreads();
+  const int t = threadIdx.x;
+  int e[kMaxK];
+  uint32_t st = 0;
+  if (t < a.bs) {
+    st = classify_row(a, t, e);
+    mark_words(words, E, e, a.K);
+  } else {
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) e[k] = -1;
+  }
+  if (st) atomicOr(&status, st);
+  __syncthreads();
+  int cnt = 0;
+  if (threadIdx.x < E)
+    for (int w = 0; w < 32; ++w) cnt += __popc(words[w * E + threadIdx.x]);
+  int total;
+  const int excl = block_exclusive_scan(cnt, warp_sums, &total);
+  if (threadIdx.x < E) {
+    offs[threadIdx.x] = excl;
+    if (writer) {
+      a.expert_token_nums[threadIdx.x] = cnt;
+      a.ep_send_counts[threadIdx.x] = excl;
+    }
+  }
+  if (writer && threadIdx.x == 0) a.ep_send_counts[E] = total;
+  __syncthreads();
+  const int t0 = blockIdx.x * per;
+  if (t < a.bs) {
+    int slot[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k)
+      slot[k] = (k < a.K && e[k] >= 0) ? offs[e[k]] + tile_rank(words, E, e[k]) : -1;
+    if (writer) write_slots(a, t, e, slot);
+    if (t >= t0 && t < t0 + per) {
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k)
+        if (k < a.K) slot_sh[t - t0][k] = slot[k];
+    }
+  }
+  if (writer) {
+    for (int s = total + threadIdx.x; s < a.A; s += blockDim.x) a.assist[s] = -1;
+    if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
+  }
+  __syncthreads();
+  const int t1 = min(a.bs, t0 + per);
+  for (int i = threadIdx.x; i < (t1 - t0) * V; i += blockDim.x) {
+    const int tl = i / V;
+    const int v = i - tl * V;
+    const uint4 val = ld_nc_v4(x + static_cast<size_t>(t0 + tl) * V + v);
+    for (int k = 0; k < a.K; ++k) {
+      const int s = slot_sh[tl][k];
+      if (s >= 0) st_v4(expand_x + static_cast<size_t>(s) * V + v, val);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Multi-CTA layout. Workspace: tile_counts[T][E] int32, then tile_status[T].
 
 struct TileWs {
@@ -325,6 +402,27 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
 }
 
 }  // namespace
+
+cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                  cudaStream_t st) {
+  const int V = H / kVecElems;
+  // at most kLayoutSmallMaxTokens / 8 tokens per CTA (the slot buffer's size)
+  int blocks = sm_count();
+  if (blocks > a.bs) blocks = a.bs > 0 ? a.bs : 1;
+  int per = (a.bs + blocks - 1) / blocks;
+  if (per > kLayoutSmallMaxTokens / 8) per = kLayoutSmallMaxTokens / 8;
+  if (per < 1) per = 1;
+  blocks = a.bs > 0 ? (a.bs + per - 1) / per : 1;
+  const size_t smem = 32u * a.E * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(dispatch_small_kernel, dim3(blocks), dim3(1024), smem, st, a,
+                    static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
+}
 
 size_t layout_workspace_bytes(int bs, int E) {
   if (bs <= kLayoutSmallMaxTokens) return 0;

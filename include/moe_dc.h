@@ -131,6 +131,22 @@ moe_status moe_dispatch_permute(const moe_shape* shape, const void* x,
                                 void* stream);
 
 /*
+ * moe_dispatch — moe_dispatch_layout followed by moe_dispatch_permute, in one
+ * call (the dispatch of the [combine] Example: low_latency_dispatch returns
+ * the expanded rows, the counts and assist_info together). For BS <= 1024
+ * without quantisation both run in one launch (every CTA rebuilds the small
+ * layout in shared memory and copies its share of rows); otherwise the two
+ * launches of the separate calls. Arguments and results as in those calls;
+ * the workspace may be NULL on the one-launch path.
+ */
+moe_status moe_dispatch(const moe_shape* shape, const int32_t* topk_idx,
+                        const uint8_t* x_active_mask, const void* x, int comm_quant_mode,
+                        int32_t* expert_token_nums, int32_t* ep_send_counts,
+                        int32_t* assist_info, uint32_t* dev_status, void* expand_x,
+                        float* dynamic_scales, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
  * moe_combine_fwd — [combine] Function (Formula; special expert use cases),
  * Parameters, Return Value:
  *   out[t] = round16( sum_{k active, ascending} w[t,k] * M(t,k)  +  shared[t] )

@@ -233,13 +233,18 @@ void oracle_dispatch_permute_quant(int bs, int K, int h, int a_capacity, int dty
   }
 }
 
-// Per-row int8 round trip of R9/R15: the fp32 value q * scale of element j.
-static float int8_roundtrip(const uint16_t* row, int h, int j, int dtype) {
+// Per-row int8 round trip of R9/R15: max |y| of a row, and the fp32 value
+// q * scale of one element given it.
+static float row_amax(const uint16_t* row, int h, int dtype) {
   float amax = 0.0f;
   for (int i = 0; i < h; ++i) amax = std::max(amax, std::fabs(load16(row, i, dtype)));
+  return amax;
+}
+
+static float int8_roundtrip(float y, float amax) {
   if (amax == 0.0f) return 0.0f;
   const float scale = amax / 127.0f;
-  float q = std::nearbyint(load16(row, j, dtype) / scale);
+  float q = std::nearbyint(y / scale);
   q = std::min(127.0f, std::max(-127.0f, q));
   return q * scale;
 }
@@ -262,8 +267,14 @@ void oracle_combine_fwd(int bs, int K, int h, int num_experts, int zero_num, int
   const int n_ids = num_experts + zero_num + copy_num + const_num;
   const int zero_end = num_experts + zero_num;
   const int copy_end = zero_end + copy_num;
+  std::vector<float> amax(K);
   for (int t = 0; t < bs; ++t) {
     const int32_t* row = topk_idx + static_cast<size_t>(t) * K;
+    if (comm_quant_mode == 2)
+      for (int k = 0; k < K; ++k) {
+        int32_t s = assist_info[A + static_cast<size_t>(t) * K + k];
+        amax[k] = s < 0 ? 0.0f : row_amax(expand_x + static_cast<size_t>(s) * h, h, dtype);
+      }
     for (int j = 0; j < h; ++j) {
       float acc = 0.0f;
       for (int k = 0; k < K; ++k) {
@@ -274,9 +285,8 @@ void oracle_combine_fwd(int bs, int K, int h, int num_experts, int zero_num, int
         if (id < num_experts) {
           int32_t s = assist_info[A + static_cast<size_t>(t) * K + k];
           if (s < 0) continue;
-          m = comm_quant_mode == 2
-                  ? int8_roundtrip(expand_x + static_cast<size_t>(s) * h, h, j, dtype)
-                  : load16(expand_x, static_cast<size_t>(s) * h + j, dtype);
+          m = load16(expand_x, static_cast<size_t>(s) * h + j, dtype);
+          if (comm_quant_mode == 2) m = int8_roundtrip(m, amax[k]);
         } else if (id < zero_end) {
           m = 0.0f;
         } else if (id < copy_end) {

@@ -153,3 +153,53 @@ def test_combine_comm_quant_mode2(wl):
     d = gpu_chain.ulp_dist(got, want)
     assert d.max() <= gpu_chain.ULP_TOL
     assert (d == 0).mean() == 1.0  # same fp32 operations in the same order
+
+
+FUSED = [
+    W["tiny"],
+    _custom("fused_ragged", bs=1000, h=1032),
+    _custom("fused_max", bs=1024, h=264, k=8, num_experts=64),
+    _custom("fused_k16_e1024", bs=300, k=16, num_experts=1024, h=128),
+    _custom("fused_mask1d", bs=700, mask_ndim=1, mask_false_p=0.3),
+    _custom("fused_mask2d_fp16", bs=513, mask_ndim=2, mask_false_p=0.2, dtype="fp16"),
+    _custom("fused_special", bs=600, zero_expert_num=1, copy_expert_num=1, const_expert_num=1),
+    _custom("fused_empty", bs=0),
+    _custom("fused_fallback_large", bs=2100, h=520),
+    W["special"].scaled(bs=800, h=1040, name="fused_fallback_int8"),
+]
+
+
+@pytest.mark.parametrize("wl", FUSED, ids=lambda w: w.name)
+def test_fused_dispatch(wl):
+    """moe_dispatch (layout + permute, one launch for small batches) against the
+    oracle: counts, prefix sums, assist_info, status and every expanded row bit for
+    bit; ids out of range and repeats are planted in the batches that have rows."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    inp = workloads.generate(wl)
+    if wl.bs > 20:
+        idx = inp["topk_idx"].copy()
+        idx[5, 0] = -3
+        idx[9, wl.k - 1] = idx[9, 0]
+        inp["topk_idx"] = idx
+    counts, send, assist, status = oracle.dispatch_layout(inp["topk_idx"], wl.num_experts,
+                                                          wl.n_ids, wl.a_capacity, inp["mask"])
+    r = int(send[-1])
+    sh = gpu_chain.shape_of(wl)
+    dev, host = gpu_chain.dev, gpu_chain.host
+    lay, ex, sc = moe.dispatch(sh, dev(inp["topk_idx"]), dev(inp["x"], wl.dtype),
+                               x_active_mask=dev(inp["mask"]), comm_quant_mode=wl.quant_mode)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(lay.expert_token_nums), counts)
+    assert np.array_equal(host(lay.ep_send_counts), send)
+    assert np.array_equal(host(lay.assist_info), assist)
+    assert int(host(lay.dev_status)[0]) & 3 == status
+    if wl.quant_mode == 2:
+        q, s = oracle.dispatch_permute_quant(inp["x"], assist, wl.k, wl.a_capacity, wl.dtype)
+        assert np.array_equal(host(ex)[:r], q[:r])
+        assert np.array_equal(host(sc)[:r].view(np.uint32), s[:r].view(np.uint32))
+    else:
+        want = oracle.dispatch_permute(inp["x"], assist, wl.k, wl.a_capacity)
+        assert np.array_equal(host(ex)[:r], want[:r])

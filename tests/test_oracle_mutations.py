@@ -49,7 +49,7 @@ MUTATIONS = [
      "      if (row[k] >= num_experts)"),
     ("int8_roundtrip_skipped",
      "  if (amax == 0.0f) return 0.0f;\n  const float scale = amax / 127.0f;",
-     "  if (amax >= 0.0f) return load16(row, j, dtype);\n  const float scale = amax / 127.0f;"),
+     "  if (amax >= 0.0f) return y;\n  const float scale = amax / 127.0f;"),
     ("duplicate_ids_accepted",
      "    if (row[j] == id) return ST_DUP_ID;", "    if (false) return ST_DUP_ID;"),
 ]
