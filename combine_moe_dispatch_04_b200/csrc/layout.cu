@@ -296,29 +296,26 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutA
   if (threadIdx.x == 0) ws.status[blockIdx.x] = status;
 }
 
-// Phase 2: the tile's first slot per expert, from the count matrix
-// (prefix over earlier tiles + exclusive scan of the expert totals), then the
-// slots of every pair of the tile and -1 for the unused slots [R, A).
-// Dynamic shared memory: words[kTileWarps][E], base[E], total[E], and two
+// Phase 2 for one 256-token tile, run by a whole CTA: the tile's first slot
+// per expert from the count matrix (prefix over earlier tiles + exclusive
+// scan of the expert totals), then slot[] of this thread's token (t < BS).
+// The CTA with first_cta writes the counts, prefix sums and status word.
+// Shared memory (dynamic): words[kTileWarps][E], base[E], total[E], and two
 // [G][E] partial-sum arrays (G * E <= blockDim).
-__global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
-  extern __shared__ uint32_t smem[];
-  __shared__ int warp_sums[32];
-  __shared__ uint32_t status;
+__device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile, bool first_cta,
+                                           uint32_t* smem, int* warp_sums, uint32_t* status,
+                                           int (&e)[kMaxK], int (&slot)[kMaxK], int* grand_out) {
   const int E = a.E;
   uint32_t* words = smem;
   int* base = reinterpret_cast<int*>(smem + kTileWarps * E);
   int* total = base + E;
-  pdl_trigger();
-  pdl_wait();
   for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
-  if (threadIdx.x == 0) status = 0;
+  if (threadIdx.x == 0) *status = 0;
   const TileWs ws = tile_ws(a, T);
-  const int tile = blockIdx.x;
   // Sum the count matrix over tiles: G groups of E threads split the tiles
   // (G = 1 when E >= blockDim), then one thread per expert adds the groups.
   const int G = E < static_cast<int>(blockDim.x) ? blockDim.x / E : 1;
-  int* part_before = total + E;       // [G][E]
+  int* part_before = total + E;         // [G][E]
   int* part_all = part_before + G * E;  // [G][E]
   if (G > 1) {
     const int g = threadIdx.x / E, ex = threadIdx.x - g * E;
@@ -356,10 +353,10 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
       total[ex] = all;
     }
   }
-  if (blockIdx.x == 0) {
+  if (first_cta) {
     uint32_t st = 0;
     for (int i = threadIdx.x; i < T; i += blockDim.x) st |= ws.status[i];
-    if (st) atomicOr(&status, st);
+    if (st) atomicOr(status, st);
   }
   __syncthreads();
   // exclusive scan of total[0, E): each thread owns a contiguous run of experts
@@ -371,34 +368,91 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
   int off = block_exclusive_scan(run, warp_sums, &grand);
   for (int ex = e0; ex < e1; ++ex) {
     const int c = total[ex];
-    if (blockIdx.x == 0) {
+    if (first_cta) {
       a.expert_token_nums[ex] = c;
       a.ep_send_counts[ex] = off;
     }
     base[ex] += off;
     off += c;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
+  if (first_cta && threadIdx.x == 0) {
     a.ep_send_counts[E] = grand;
-    if (a.dev_status) *a.dev_status = status;
+    if (a.dev_status) *a.dev_status = *status;
   }
   const int t = tile * kLayoutTileTokens + threadIdx.x;
-  int e[kMaxK];
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) e[k] = -1;
   if (t < a.bs) {
     classify_row(a, t, e);
     mark_words(words, E, e, a.K);
   }
   __syncthreads();
-  if (t < a.bs) {
-    int slot[kMaxK];
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k)
-      slot[k] = (k < a.K && e[k] >= 0) ? base[e[k]] + tile_rank(words, E, e[k]) : -1;
-    write_slots(a, t, e, slot);
-  }
+  for (int k = 0; k < kMaxK; ++k)
+    slot[k] = (t < a.bs && k < a.K && e[k] >= 0) ? base[e[k]] + tile_rank(words, E, e[k]) : -1;
+  *grand_out = grand;
+}
+
+// Phase 2 as its own launch: every tile's slots, and -1 for the unused
+// slots [R, A).
+__global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
+  extern __shared__ uint32_t smem[];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t status;
+  pdl_trigger();
+  pdl_wait();
+  int e[kMaxK], slot[kMaxK], grand;
+  tile_slots(a, T, blockIdx.x, blockIdx.x == 0, smem, warp_sums, &status, e, slot, &grand);
+  const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
+  if (t < a.bs) write_slots(a, t, e, slot);
   for (int s = grand + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
        s += gridDim.x * blockDim.x)
     a.assist[s] = -1;
+}
+
+// Phase 2 fused with the permute (no quantisation): CTA (tile, sub) of a
+// grid of T * S computes its tile's slots; sub-CTA 0 writes the tile's
+// assist_info and its share of [R, A); every CTA then copies the rows of its
+// 256 / S tokens of the tile to their slots (one thread per 16-byte vector,
+// read once, stored K times).
+__global__ void __launch_bounds__(kLayoutTileTokens) dispatch_tiled_kernel(LayoutArgs a, int T,
+                                                                           int S, const uint4* x,
+                                                                           uint4* expand_x, int V) {
+  extern __shared__ uint32_t smem[];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t status;
+  __shared__ int slot_sh[kLayoutTileTokens][kMaxK];
+  pdl_trigger();
+  pdl_wait();
+  const int tile = blockIdx.x / S, sub = blockIdx.x - tile * S;
+  int e[kMaxK], slot[kMaxK], grand;
+  tile_slots(a, T, tile, blockIdx.x == 0, smem, warp_sums, &status, e, slot, &grand);
+  const int t = tile * kLayoutTileTokens + threadIdx.x;
+  const int per = (kLayoutTileTokens + S - 1) / S;
+  const int l0 = sub * per, l1 = min(kLayoutTileTokens, l0 + per);
+  if (t < a.bs) {
+    if (sub == 0) write_slots(a, t, e, slot);
+    if (static_cast<int>(threadIdx.x) >= l0 && static_cast<int>(threadIdx.x) < l1) {
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k)
+        if (k < a.K) slot_sh[threadIdx.x][k] = slot[k];
+    }
+  }
+  if (sub == 0)
+    for (int s = grand + tile * blockDim.x + threadIdx.x; s < a.A; s += T * blockDim.x)
+      a.assist[s] = -1;
+  __syncthreads();
+  const int tend = min(l1, a.bs - tile * kLayoutTileTokens);
+  const int n = (tend - l0) * V;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int tl = l0 + i / V;
+    const int v = i - (tl - l0) * V;
+    const uint4 val = ld_nc_v4(x + static_cast<size_t>(tile * kLayoutTileTokens + tl) * V + v);
+    for (int k = 0; k < a.K; ++k) {
+      const int s = slot_sh[tl][k];
+      if (s >= 0) st_v4(expand_x + static_cast<size_t>(s) * V + v, val);
+    }
+  }
 }
 
 }  // namespace
@@ -422,6 +476,28 @@ cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expa
   }
   return launch_pdl(dispatch_small_kernel, dim3(blocks), dim3(1024), smem, st, a,
                     static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
+}
+
+cudaError_t launch_dispatch_tiled(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                  cudaStream_t st) {
+  const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
+  const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
+  const size_t smem_scatter =
+      smem_count + 2u * a.E * sizeof(int) + 2u * kLayoutTileTokens * sizeof(int);
+  cudaError_t err = launch_pdl(layout_count_kernel, dim3(T), dim3(kLayoutTileTokens), smem_count,
+                               st, a, T);
+  if (err != cudaSuccess) return err;
+  // enough CTAs for about four per SM, at least one per tile, at most one per 8 tokens
+  int S = (4 * sm_count() + T - 1) / T;
+  S = S < 1 ? 1 : S > kLayoutTileTokens / 8 ? kLayoutTileTokens / 8 : S;
+  if (smem_scatter > 24 * 1024) {  // plus 16 KB of static slots: opt in above 48 KB
+    err = cudaFuncSetAttribute(dispatch_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_scatter));
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(dispatch_tiled_kernel, dim3(T * S), dim3(kLayoutTileTokens), smem_scatter,
+                    st, a, T, S, static_cast<const uint4*>(x), static_cast<uint4*>(expand_x),
+                    H / kVecElems);
 }
 
 size_t layout_workspace_bytes(int bs, int E) {

@@ -164,8 +164,14 @@ FUSED = [
     _custom("fused_mask2d_fp16", bs=513, mask_ndim=2, mask_false_p=0.2, dtype="fp16"),
     _custom("fused_special", bs=600, zero_expert_num=1, copy_expert_num=1, const_expert_num=1),
     _custom("fused_empty", bs=0),
-    _custom("fused_fallback_large", bs=2100, h=520),
+    _custom("fused_tiled_ragged", bs=2100, h=520),
+    _custom("fused_tiled_k16_e1024", bs=1500, k=16, num_experts=1024, h=128),
+    _custom("fused_tiled_one_tile_tail", bs=1025, h=64),
+    W["uniform"],
+    W["mixtral"],
+    W["dsv3"].scaled(bs=3000, h=1024, name="fused_tiled_zipf"),
     W["special"].scaled(bs=800, h=1040, name="fused_fallback_int8"),
+    W["special"].scaled(bs=2600, h=1040, quant_mode=0, name="fused_tiled_special"),
 ]
 
 
