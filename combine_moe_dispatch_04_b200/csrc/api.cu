@@ -146,7 +146,7 @@ moe_status moe_dispatch(const moe_shape* s, const int32_t* topk_idx, const uint8
                         size_t workspace_bytes, void* stream) {
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
-  const bool fused = comm_quant_mode == 0;
+  const bool fused = comm_quant_mode == 0 && s->bs <= moe::kLayoutSmallMaxTokens;
   if (!fused) {
     st = moe_dispatch_layout(s, topk_idx, x_active_mask, expert_token_nums, ep_send_counts,
                              assist_info, dev_status, workspace, workspace_bytes, stream);
@@ -173,14 +173,9 @@ moe_status moe_dispatch(const moe_shape* s, const int32_t* topk_idx, const uint8
   a.ep_send_counts = ep_send_counts;
   a.assist = assist_info;
   a.dev_status = dev_status;
-  a.workspace = workspace;
-  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (s->bs <= moe::kLayoutSmallMaxTokens)
-    return cuda_status(moe::launch_dispatch_small(a, x, expand_x, s->h, cs));
-  const size_t need = moe::layout_workspace_bytes(s->bs, s->num_experts);
-  if (workspace == nullptr || workspace_bytes < need) return MOE_ERR_CAPACITY;
-  if (!aligned16(workspace)) return MOE_ERR_ALIGN;
-  return cuda_status(moe::launch_dispatch_tiled(a, x, expand_x, s->h, cs));
+  a.workspace = nullptr;
+  return cuda_status(
+      moe::launch_dispatch_small(a, x, expand_x, s->h, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine_fwd(const moe_shape* s, const void* expand_x, const int32_t* topk_idx,

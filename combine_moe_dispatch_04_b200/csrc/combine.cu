@@ -279,9 +279,10 @@ __global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
           float y[8];
           widen8<T16>(__ldg(Y + static_cast<size_t>(pm.row) * V + v), y);
           const float scale = __fdiv_rn(mx, 127.0f);
+          const float inv_scale = 1.0f / scale;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            float q = mx == 0.0f ? 0.0f : rintf(__fdiv_rn(y[i], scale));
+            float q = mx == 0.0f ? 0.0f : quant_code(y[i], scale, inv_scale);
             q = fminf(127.0f, fmaxf(-127.0f, q));
             m[i] = __fmul_rn(q, scale);
           }

@@ -102,6 +102,19 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// rne(fl32(y / scale)) for |y| <= max|row| and scale = fl32(max|row| / 127),
+// so |y / scale| <= 127 (1 + 2^-23). r = y * fl32(1 / scale) and the IEEE
+// quotient fl32(y / scale) both lie within 127 * 3 * 2^-24 < 2^-15 of the
+// exact quotient; when r is at least 2^-14 away from every half-integer, both
+// round to the same integer, so rint(r) is the answer. Otherwise (rare: near
+// a rounding tie) the IEEE division decides.
+__device__ __forceinline__ float quant_code(float y, float scale, float inv_scale) {
+  const float r = y * inv_scale;
+  const float frac = r - floorf(r);
+  if (fabsf(frac - 0.5f) > 0.00006103515625f) return rintf(r);  // 2^-14
+  return rintf(__fdiv_rn(y, scale));
+}
+
 // Whether pair (t, k) is active under x_active_mask (1-D per token, 2-D per pair).
 __device__ __forceinline__ bool pair_active(const uint8_t* mask, int mask_ndim, int t, int k,
                                             int K) {

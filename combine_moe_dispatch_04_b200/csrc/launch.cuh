@@ -40,10 +40,6 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
 // Layout and the plain (no quantisation) permute in one launch, BS <= kLayoutSmallMaxTokens.
 cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
                                   cudaStream_t st);
-// Layout and the plain permute in two launches (count; slots fused with the row copies),
-// BS > kLayoutSmallMaxTokens; needs the layout workspace.
-cudaError_t launch_dispatch_tiled(const LayoutArgs& a, const void* x, void* expand_x, int H,
-                                  cudaStream_t st);
 
 struct CombineArgs {
   const void* expand_x;  // (A, H): expert outputs, or slot gradients for dispatch bwd

@@ -410,51 +410,6 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
     a.assist[s] = -1;
 }
 
-// Phase 2 fused with the permute (no quantisation): CTA (tile, sub) of a
-// grid of T * S computes its tile's slots; sub-CTA 0 writes the tile's
-// assist_info and its share of [R, A); every CTA then copies the rows of its
-// 256 / S tokens of the tile to their slots (one thread per 16-byte vector,
-// read once, stored K times).
-__global__ void __launch_bounds__(kLayoutTileTokens) dispatch_tiled_kernel(LayoutArgs a, int T,
-                                                                           int S, const uint4* x,
-                                                                           uint4* expand_x, int V) {
-  extern __shared__ uint32_t smem[];
-  __shared__ int warp_sums[32];
-  __shared__ uint32_t status;
-  __shared__ int slot_sh[kLayoutTileTokens][kMaxK];
-  pdl_trigger();
-  pdl_wait();
-  const int tile = blockIdx.x / S, sub = blockIdx.x - tile * S;
-  int e[kMaxK], slot[kMaxK], grand;
-  tile_slots(a, T, tile, blockIdx.x == 0, smem, warp_sums, &status, e, slot, &grand);
-  const int t = tile * kLayoutTileTokens + threadIdx.x;
-  const int per = (kLayoutTileTokens + S - 1) / S;
-  const int l0 = sub * per, l1 = min(kLayoutTileTokens, l0 + per);
-  if (t < a.bs) {
-    if (sub == 0) write_slots(a, t, e, slot);
-    if (static_cast<int>(threadIdx.x) >= l0 && static_cast<int>(threadIdx.x) < l1) {
-#pragma unroll
-      for (int k = 0; k < kMaxK; ++k)
-        if (k < a.K) slot_sh[threadIdx.x][k] = slot[k];
-    }
-  }
-  if (sub == 0)
-    for (int s = grand + tile * blockDim.x + threadIdx.x; s < a.A; s += T * blockDim.x)
-      a.assist[s] = -1;
-  __syncthreads();
-  const int tend = min(l1, a.bs - tile * kLayoutTileTokens);
-  const int n = (tend - l0) * V;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int tl = l0 + i / V;
-    const int v = i - (tl - l0) * V;
-    const uint4 val = ld_nc_v4(x + static_cast<size_t>(tile * kLayoutTileTokens + tl) * V + v);
-    for (int k = 0; k < a.K; ++k) {
-      const int s = slot_sh[tl][k];
-      if (s >= 0) st_v4(expand_x + static_cast<size_t>(s) * V + v, val);
-    }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
@@ -476,28 +431,6 @@ cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expa
   }
   return launch_pdl(dispatch_small_kernel, dim3(blocks), dim3(1024), smem, st, a,
                     static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
-}
-
-cudaError_t launch_dispatch_tiled(const LayoutArgs& a, const void* x, void* expand_x, int H,
-                                  cudaStream_t st) {
-  const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
-  const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
-  const size_t smem_scatter =
-      smem_count + 2u * a.E * sizeof(int) + 2u * kLayoutTileTokens * sizeof(int);
-  cudaError_t err = launch_pdl(layout_count_kernel, dim3(T), dim3(kLayoutTileTokens), smem_count,
-                               st, a, T);
-  if (err != cudaSuccess) return err;
-  // enough CTAs for about four per SM, at least one per tile, at most one per 8 tokens
-  int S = (4 * sm_count() + T - 1) / T;
-  S = S < 1 ? 1 : S > kLayoutTileTokens / 8 ? kLayoutTileTokens / 8 : S;
-  if (smem_scatter > 24 * 1024) {  // plus 16 KB of static slots: opt in above 48 KB
-    err = cudaFuncSetAttribute(dispatch_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_scatter));
-    if (err != cudaSuccess) return err;
-  }
-  return launch_pdl(dispatch_tiled_kernel, dim3(T * S), dim3(kLayoutTileTokens), smem_scatter,
-                    st, a, T, S, static_cast<const uint4*>(x), static_cast<uint4*>(expand_x),
-                    H / kVecElems);
 }
 
 size_t layout_workspace_bytes(int bs, int E) {

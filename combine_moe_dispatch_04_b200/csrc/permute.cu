@@ -41,9 +41,9 @@ __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
   }
 }
 
-constexpr int kQuantChunksPerThread = 4;  // 16-element chunks per thread
-
-template <typename T16>
+// CPT 16-element chunks per thread (1, 2 or 4), chosen by the launcher so a
+// row fits the CTA with as few registers as possible.
+template <typename T16, int CPT>
 __global__ void __launch_bounds__(256) permute_quant_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
     float* __restrict__ scales, int bs, int K, int H, int A) {
@@ -55,10 +55,12 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
   const int nwarps = blockDim.x >> 5;
   for (int t = blockIdx.x; t < bs; t += gridDim.x) {
     const uint4* xr = x + static_cast<size_t>(t) * (H / 8);
-    float f[kQuantChunksPerThread][16];
+    const int32_t* slots = assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K;
+    const int my_slot = threadIdx.x < K ? __ldg(slots + threadIdx.x) : -1;
+    float f[CPT][16];
     float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kQuantChunksPerThread; ++j) {
+    for (int j = 0; j < CPT; ++j) {
       const int c = threadIdx.x + j * blockDim.x;
       if (c < C) {
         float lo[8], hi[8];
@@ -80,9 +82,9 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
     for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, warp_max[w]);
     __syncthreads();  // warp_max is reused by the next token
     const float scale = __fdiv_rn(amax, 127.0f);
-    const int32_t* slots = assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K;
+    const float inv_scale = 1.0f / scale;
 #pragma unroll
-    for (int j = 0; j < kQuantChunksPerThread; ++j) {
+    for (int j = 0; j < CPT; ++j) {
       const int c = threadIdx.x + j * blockDim.x;
       if (c >= C) continue;
       uint32_t packed[4];
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
         for (int b = 0; b < 4; ++b) {
           int q = 0;
           if (amax != 0.0f) {
-            float r = rintf(__fdiv_rn(f[j][w4 * 4 + b], scale));
+            float r = quant_code(f[j][w4 * 4 + b], scale, inv_scale);
             r = fminf(127.0f, fmaxf(-127.0f, r));
             q = __float2int_rn(r);
           }
@@ -103,14 +105,11 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
       }
       const uint4 val = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       for (int k = 0; k < K; ++k) {
-        const int s = __ldg(slots + k);
+        const int s = __shfl_sync(0xFFFFFFFFu, my_slot, k);
         if (s >= 0) st_v4(out + static_cast<size_t>(s) * C + c, val);
       }
     }
-    if (threadIdx.x < K) {
-      const int s = __ldg(slots + threadIdx.x);
-      if (s >= 0) scales[s] = scale;
-    }
+    if (threadIdx.x < K && my_slot >= 0) scales[my_slot] = scale;
   }
 }
 
@@ -127,16 +126,28 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
                       static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
                       a.bs, a.K, V, a.A);
   }
-  // One chunk per thread up to 256 threads, then up to 4 chunks per thread
+  // One 16-value chunk per thread up to 256 threads, then 2 or 4 per thread
   // (H <= 16384, checked by the caller).
   const int C = a.H / 16;
   int threads = (C + 31) / 32 * 32;
   threads = threads > 256 ? 256 : threads;
-  const int cap = sm_count() * 16;
+  const int cpt = (C + threads - 1) / threads;
+  const int cap = sm_count() * (2048 / threads);
   const int blocks = a.bs < cap ? a.bs : cap;
-  auto kernel = a.dtype == MOE_BF16 ? permute_quant_kernel<Bf16> : permute_quant_kernel<Fp16>;
-  return launch_pdl(kernel, dim3(blocks), dim3(threads), 0, st, static_cast<const uint4*>(a.x),
-                    a.assist, static_cast<uint4*>(a.expand_x), a.scales, a.bs, a.K, a.H, a.A);
+  const uint4* x = static_cast<const uint4*>(a.x);
+  uint4* out = static_cast<uint4*>(a.expand_x);
+  const bool bf = a.dtype == MOE_BF16;
+  if (cpt <= 1)
+    return launch_pdl(bf ? permute_quant_kernel<Bf16, 1> : permute_quant_kernel<Fp16, 1>,
+                      dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales, a.bs, a.K,
+                      a.H, a.A);
+  if (cpt <= 2)
+    return launch_pdl(bf ? permute_quant_kernel<Bf16, 2> : permute_quant_kernel<Fp16, 2>,
+                      dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales, a.bs, a.K,
+                      a.H, a.A);
+  return launch_pdl(bf ? permute_quant_kernel<Bf16, 4> : permute_quant_kernel<Fp16, 4>,
+                    dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales, a.bs, a.K,
+                    a.H, a.A);
 }
 
 }  // namespace moe

@@ -133,13 +133,11 @@ moe_status moe_dispatch_permute(const moe_shape* shape, const void* x,
 /*
  * moe_dispatch — moe_dispatch_layout followed by moe_dispatch_permute, in one
  * call (the dispatch of the [combine] Example: low_latency_dispatch returns
- * the expanded rows, the counts and assist_info together). Without
- * quantisation the row copies are fused into the layout: for BS <= 1024 one
- * launch (every CTA rebuilds the small layout in shared memory and copies its
- * share of rows), above that two (the count kernel, then one kernel that
- * computes each tile's slots and copies the tile's rows). With
- * comm_quant_mode 2 it runs the two separate calls. Arguments and results as
- * in those calls; the workspace may be NULL when BS <= 1024.
+ * the expanded rows, the counts and assist_info together). For BS <= 1024
+ * without quantisation both run in one launch (every CTA rebuilds the small
+ * layout in shared memory and copies its share of rows); otherwise the
+ * launches of the two separate calls. Arguments and results as in those
+ * calls; the workspace may be NULL when BS <= 1024.
  */
 moe_status moe_dispatch(const moe_shape* shape, const int32_t* topk_idx,
                         const uint8_t* x_active_mask, const void* x, int comm_quant_mode,

@@ -209,3 +209,39 @@ def test_fused_dispatch(wl):
     else:
         want = oracle.dispatch_permute(inp["x"], assist, wl.k, wl.a_capacity)
         assert np.array_equal(host(ex)[:r], want[:r])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_int8_quant_rounding_ties(dtype):
+    """Rows whose quotients x / scale are exact half-integers (ties, decided by
+    round-half-even) or lie next to them: the kernel's quantisation must match the
+    oracle's IEEE division and rounding code for code."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+    from golden_io import read
+
+    h = 64
+    rows = []
+    g = read("quant_rows.txt")
+    for r in g["x"]:
+        rows.append(np.pad(np.array(r, np.float64), (0, h - len(r))))
+    rng = np.random.default_rng(17)
+    for amax in (127.0, 63.5, 31.75, 100.0, 3.0, 0.01):
+        ties = (rng.integers(-126, 126, h) + 0.5) * (amax / 127.0)
+        ties[0] = amax
+        rows.append(ties)
+        near = ties * (1 + rng.choice([-1, 1], h) * rng.uniform(0, 4e-3, h))
+        near[0] = amax
+        rows.append(near)
+    x = workloads.encode16(np.array(rows), dtype)
+    bs = len(rows)
+    idx = np.zeros((bs, 1), np.int32)
+    _, send, assist, _ = oracle.dispatch_layout(idx, 1, 1, bs)
+    q, sc = oracle.dispatch_permute_quant(x, assist, 1, bs, dtype)
+    sh = moe.Shape(bs=bs, k=1, h=h, num_experts=1, dtype=workloads.DTYPE_CODES[dtype])
+    lay = moe.dispatch_layout(sh, gpu_chain.dev(idx))
+    qd, scd = moe.dispatch_permute(sh, gpu_chain.dev(x, dtype), lay, 2)
+    torch.cuda.synchronize()
+    assert np.array_equal(gpu_chain.host(qd), q)
+    assert np.array_equal(gpu_chain.host(scd).view(np.uint32), sc.view(np.uint32))
