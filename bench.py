@@ -17,6 +17,7 @@ timing use the process group.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime as _dt
 import hashlib
 import json
@@ -39,7 +40,8 @@ METRIC = "dispatch+combine fwd+bwd tokens/s and achieved HBM GB/s (% of 8 TB/s),
 DEFAULT_WORKLOAD = "uniform_bs8192_h1536_k8_e64"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-KERNELS = ("layout", "permute", "combine_fwd", "combine_bwd", "dispatch_bwd")
+KERNELS = ("layout", "permute", "combine_fwd", "combine_bwd", "combine_bwd_special",
+           "dispatch_bwd")
 DOM_EVERY = 4
 
 
@@ -63,6 +65,12 @@ def byte_model(wl: workloads.Workload, r: int, ori_tokens: int) -> dict:
                         + 3 * wl.const_expert_num * row + bs * row)
     if wl.backward:
         m["combine_bwd"] = bs * row + 2 * r * row + 4 * pairs + slot_map + 4 * pairs + mask
+        if wl.copy_expert_num + wl.const_expert_num:
+            # grad_out and ori_x of the tokens with a copy/const pair, grad_ori_x of
+            # every token, ids and weights, the const rows and their gradients
+            m["combine_bwd_special"] = (2 * ori_tokens * row + bs * row + 8 * pairs + mask
+                                        + 3 * wl.const_expert_num * row
+                                        + 3 * wl.const_expert_num * h * 4)
         m["dispatch_bwd"] = r * row + bs * row + slot_map + mask
     return m
 
@@ -167,7 +175,7 @@ def measured_hbm_peak():
 
 
 KERNEL_SOURCES = {"layout": "layout.cu", "dispatch": "layout.cu", "permute": "permute.cu",
-                  "combine_fwd": "combine.cu",
+                  "combine_fwd": "combine.cu", "combine_bwd_special": "special_bwd.cu",
                   "combine_bwd": "combine.cu", "dispatch_bwd": "combine.cu"}
 
 
@@ -298,10 +306,16 @@ def main():
                     help="layout + permute through the single moe_dispatch call")
     ap.add_argument("--combine-comm-quant", type=int, default=0, choices=[0, 2],
                     help="combine forward with comm_quant_mode 2 (int8 round trip)")
+    ap.add_argument("--with-backward", action="store_true",
+                    help="add the backward steps to a forward-only workload")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step eagerly instead of replaying a CUDA graph of it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     wl = workloads.BY_NAME[args.workload]
+    if args.with_backward and not wl.backward:
+        wl = wl.scaled(backward=True, name=wl.name + "+backward")
     if args.impl == "reference":
         return run_reference(args, wl)
     if args.warmup < 3:
@@ -374,68 +388,104 @@ def main():
         ori_tokens = int(np.any(ids >= lo, axis=1).sum())
     bytes_per = byte_model(wl, r, ori_tokens)
     kernels = [k for k in KERNELS if k in bytes_per]
+    sp_ws = sp_out = None
+    if "combine_bwd_special" in bytes_per:
+        n_ws = moe.moe_combine_bwd_special_workspace_bytes(ctypes.byref(sh.c()))
+        sp_ws = torch.empty(max(n_ws, 16), dtype=torch.uint8, device=dev) if n_ws else None
+        _, *sp_out = moe.combine_bwd_special(
+            sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
+            x_active_mask=d["mask"], const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
+            const_v=d["v"], grad_w=gw, workspace=sp_ws)
+        torch.cuda.synchronize()
 
     cq = args.combine_comm_quant
     if args.fused_dispatch:
-        calls = [("dispatch", lambda: moe.dispatch(
+        calls = [("dispatch", lambda st: moe.dispatch(
             sh, d["topk_idx"], d["x"], x_active_mask=d["mask"], comm_quant_mode=qm,
-            workspace=ws, layout=lay, expand_x=expand, dynamic_scales=scales, stream=stream))]
+            workspace=ws, layout=lay, expand_x=expand, dynamic_scales=scales, stream=st))]
         bytes_per["dispatch"] = bytes_per.pop("layout") + bytes_per.pop("permute")
         kernels = ["dispatch"] + [k for k in kernels if k not in ("layout", "permute")]
     else:
         calls = [
-            ("layout", lambda: moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws,
-                                                   out=lay, stream=stream)),
-            ("permute", lambda: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
-                                                     dynamic_scales=scales, stream=stream)),
+            ("layout", lambda st: moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws,
+                                                   out=lay, stream=st)),
+            ("permute", lambda st: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
+                                                     dynamic_scales=scales, stream=st)),
         ]
     calls += [
-        ("combine_fwd", lambda: moe.combine_fwd(
+        ("combine_fwd", lambda st: moe.combine_fwd(
             sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
             shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
             const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, out=out,
-            stream=stream)),
+            stream=st)),
     ]
     if wl.backward:
         calls += [
-            ("combine_bwd", lambda: moe.combine_bwd(
+            ("combine_bwd", lambda st: moe.combine_bwd(
                 sh, d["grad_out"], y, d["topk_weights"], lay, x_active_mask=d["mask"],
-                grad_expand=gexp, grad_w=gw, stream=stream)),
-            ("dispatch_bwd", lambda: moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"],
-                                                      grad_x=gx, stream=stream)),
+                grad_expand=gexp, grad_w=gw, stream=st)),
+        ]
+        if "combine_bwd_special" in bytes_per:
+            calls += [("combine_bwd_special", lambda st: moe.combine_bwd_special(
+                sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
+                x_active_mask=d["mask"], const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
+                const_v=d["v"], grad_w=gw, workspace=sp_ws, out=sp_out, stream=st))]
+        calls += [
+            ("dispatch_bwd", lambda st: moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"],
+                                                      grad_x=gx, stream=st)),
         ]
     # the kernel that moves the most bytes; the timed steps bracket it with events
     dominant = max((k for k in kernels if k not in ("layout", "dispatch")),
                    key=lambda k: bytes_per[k])
 
-    def step(marks=None):
-        """One pass of the path. `marks` maps "start"/"end" to an event and kernel
-        names to (before, after) event pairs; kernels without events keep their
-        programmatic-launch overlap with their neighbours."""
-        if marks is not None:
-            marks["start"].record(stream)
+    def run_calls(st, marks=None):
         for name, fn in calls:
             if marks is not None and name in marks:
-                marks[name][0].record(stream)
-            fn()
+                marks[name][0].record(st)
+            fn(st)
             if marks is not None and name in marks:
-                marks[name][1].record(stream)
-        if marks is not None:
-            marks["end"].record(stream)
+                marks[name][1].record(st)
 
-    def new_marks(names):
-        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    def new_marks(names, external=False):
+        ev = lambda: torch.cuda.Event(enable_timing=True, external=external)  # noqa: E731
         m = {"start": ev(), "end": ev()}
         for n_ in names:
             m[n_] = (ev(), ev())
         return m
+
+    # CUDA graphs of the step: one plain, and one per sampled step with timing
+    # events (graph event-record nodes) around the dominant kernel.
+    graphs = {}
+
+    def capture(marks=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_calls(torch.cuda.current_stream(), marks)
+        return g
+
+    def step(marks=None, graph=None):
+        """One pass of the path. `marks` maps "start"/"end" to an event and kernel
+        names to (before, after) event pairs; kernels without events keep their
+        programmatic-launch overlap with their neighbours. With `graph`, the
+        pass is that captured graph (whose own events are already inside)."""
+        if marks is not None:
+            marks["start"].record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            run_calls(stream, marks)
+        if marks is not None:
+            marks["end"].record(stream)
 
     tiled = wl.bs > moe_layout_small_max_tokens()
     if args.fused_dispatch and not tiled and qm == 0:
         dispatch_launches = 1
     else:
         dispatch_launches = (2 if tiled else 1) + 1
-    launches_per_step = dispatch_launches + 1 + (2 if wl.backward else 0)
+    special_bwd_launches = 0
+    if "combine_bwd_special" in bytes_per:
+        special_bwd_launches = 2 + (2 if wl.const_expert_num else 0)
+    launches_per_step = dispatch_launches + 1 + (2 if wl.backward else 0) + special_bwd_launches
 
     # L2 flush between steps: write a buffer twice the size of L2
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
@@ -449,8 +499,27 @@ def main():
     # Every DOM_EVERY-th timed step also brackets the dominant kernel with events
     # (an event between two kernels costs both their launch overlap, so the
     # other steps carry only the step's own start/end events).
-    marks = [new_marks([dominant] if i % DOM_EVERY == DOM_EVERY - 1 else [])
-             for i in range(args.steps)]
+    sampled = [i % DOM_EVERY == DOM_EVERY - 1 for i in range(args.steps)]
+    use_graph = not args.no_graph
+    marks, step_graphs = [], []
+    if use_graph:
+        plain = capture()
+        for i in range(args.steps):
+            m = new_marks([])
+            if sampled[i]:
+                inner = new_marks([dominant], external=True)
+                m[dominant] = inner[dominant]
+                step_graphs.append(capture({dominant: inner[dominant]}))
+            else:
+                step_graphs.append(plain)
+            marks.append(m)
+        for _ in range(2):  # warm the graphs
+            flush.zero_()
+            step(graph=plain)
+        torch.cuda.synchronize()
+    else:
+        marks = [new_marks([dominant] if sampled[i] else []) for i in range(args.steps)]
+        step_graphs = [None] * args.steps
     uuid = None
     try:
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -465,7 +534,10 @@ def main():
     t0 = time.time()
     for i in range(args.steps):
         flush.zero_()
-        step(marks[i])
+        if step_graphs[i] is not None:
+            step({"start": marks[i]["start"], "end": marks[i]["end"]}, graph=step_graphs[i])
+        else:
+            step(marks[i])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -544,6 +616,7 @@ def main():
                        "a_capacity": wl.a_capacity, "parallelism": "replicas",
                        "fused_dispatch": bool(args.fused_dispatch),
                        "combine_comm_quant_mode": cq,
+                       "launch": "CUDA graph of the step" if use_graph else "eager launches",
                        "l2": "flushed before every step (write of 2x L2), outside the step events"},
             "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
             "hbm_frac_of_measured": round(gbs / peak, 4),

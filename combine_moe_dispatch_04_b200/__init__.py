@@ -26,7 +26,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_layout_workspace_bytes", "moe_dispatch_layout", "moe_dispatch_permute",
            "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd",
            "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes",
-           "moe_combine_fwd_comm_quant", "moe_dispatch")
+           "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
+           "moe_combine_bwd_special_workspace_bytes")
 
 
 class MoeShape(ctypes.Structure):
@@ -61,6 +62,10 @@ def _load():
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_combine_fwd_comm_quant.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P]
     L.moe_dispatch.argtypes = [S, P, P, P, I, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_combine_bwd_special.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                          ctypes.c_size_t, P]
+    L.moe_combine_bwd_special_workspace_bytes.argtypes = [S]
+    L.moe_combine_bwd_special_workspace_bytes.restype = ctypes.c_size_t
     L.moe_combine_bwd.argtypes = [S, P, P, P, P, P, P, P, P, P]
     L.moe_dispatch_bwd.argtypes = [S, P, P, P, P, P]
     L.moe_dispatch_layout_noalloc.argtypes = [S, P, P, P, P, P, P, P]
@@ -68,7 +73,7 @@ def _load():
     L.moe_layout_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
               "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
-              "moe_combine_fwd_comm_quant", "moe_dispatch"):
+              "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special"):
         getattr(L, n).restype = I
     return L
 
@@ -88,6 +93,8 @@ moe_dispatch_bwd = _lib.moe_dispatch_bwd
 moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
 moe_combine_fwd_comm_quant = _lib.moe_combine_fwd_comm_quant
 moe_dispatch = _lib.moe_dispatch
+moe_combine_bwd_special = _lib.moe_combine_bwd_special
+moe_combine_bwd_special_workspace_bytes = _lib.moe_combine_bwd_special_workspace_bytes
 moe_layout_noalloc_max_workspace_bytes = _lib.moe_layout_noalloc_max_workspace_bytes
 
 
@@ -278,6 +285,38 @@ def combine_bwd(shape: Shape, grad_out, expand_x, topk_weights, layout: Layout, 
         _ptr(topk_weights), _ptr(layout.assist_info), _ptr(x_active_mask), _ptr(grad_expand),
         _ptr(grad_w), _stream(stream)))
     return grad_expand, grad_w
+
+
+def combine_bwd_special(shape: Shape, grad_out, topk_idx, topk_weights, ori_x, *,
+                        x_active_mask=None, const_alpha_1=None, const_alpha_2=None,
+                        const_v=None, grad_w=None, workspace=None, out=None, stream=None):
+    """Backward of the copy/const experts. Fills the copy/const entries of grad_w (a new
+    zero tensor when None) and returns (grad_w, grad_ori_x, grad_alpha_1, grad_alpha_2,
+    grad_v); the last three are None without const experts. `out` may hold the last
+    four tensors, preallocated."""
+    import torch
+
+    dev = grad_out.device
+    if grad_w is None:
+        grad_w = torch.zeros(shape.bs, shape.k, dtype=torch.float32, device=dev)
+    if out is not None:
+        grad_ori, ga1, ga2, gv = out
+    else:
+        grad_ori = torch.empty(shape.bs, shape.h, dtype=_torch_dtype(shape), device=dev)
+        ga1 = ga2 = gv = None
+        if shape.const_expert_num:
+            ga1, ga2, gv = (torch.empty(shape.const_expert_num, shape.h, dtype=torch.float32,
+                                        device=dev) for _ in range(3))
+    if workspace is None:
+        n = moe_combine_bwd_special_workspace_bytes(ctypes.byref(shape.c()))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("moe_combine_bwd_special", moe_combine_bwd_special(
+        ctypes.byref(shape.c()), _ptr(grad_out), _ptr(topk_idx), _ptr(topk_weights),
+        _ptr(x_active_mask), _ptr(ori_x), _ptr(const_alpha_1), _ptr(const_alpha_2),
+        _ptr(const_v), _ptr(grad_w), _ptr(grad_ori), _ptr(ga1), _ptr(ga2), _ptr(gv),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+    return grad_w, grad_ori, ga1, ga2, gv
 
 
 def dispatch_bwd(shape: Shape, grad_expand_in, layout: Layout, *, x_active_mask=None,

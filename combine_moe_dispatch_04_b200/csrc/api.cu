@@ -273,6 +273,41 @@ moe_status moe_combine_bwd(const moe_shape* s, const void* grad_out, const void*
   return cuda_status(moe::launch_combine_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t moe_combine_bwd_special_workspace_bytes(const moe_shape* s) {
+  if (s == nullptr || check_shape(s) != MOE_OK) return 0;
+  return moe::special_bwd_workspace_bytes(s->bs, s->h, s->const_expert_num);
+}
+
+moe_status moe_combine_bwd_special(const moe_shape* s, const void* grad_out,
+                                   const int32_t* topk_idx, const float* topk_weights,
+                                   const uint8_t* x_active_mask, const void* ori_x,
+                                   const void* const_alpha_1, const void* const_alpha_2,
+                                   const void* const_v, float* grad_w, void* grad_ori_x,
+                                   float* grad_alpha_1, float* grad_alpha_2, float* grad_v,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if ((st = check_mask(s, x_active_mask)) != MOE_OK) return st;
+  const bool consts = s->const_expert_num > 0;
+  if (s->bs > 0 && (grad_out == nullptr || topk_idx == nullptr || topk_weights == nullptr ||
+                    ori_x == nullptr || grad_w == nullptr || grad_ori_x == nullptr))
+    return MOE_ERR_ARG;
+  if (consts && (const_alpha_1 == nullptr || const_alpha_2 == nullptr || const_v == nullptr ||
+                 grad_alpha_1 == nullptr || grad_alpha_2 == nullptr || grad_v == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(grad_out) || !aligned16(ori_x) || !aligned16(grad_ori_x) ||
+      !aligned16(const_alpha_1) || !aligned16(const_alpha_2) || !aligned16(const_v))
+    return MOE_ERR_ALIGN;
+  const size_t need = moe::special_bwd_workspace_bytes(s->bs, s->h, s->const_expert_num);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return MOE_ERR_CAPACITY;
+  if (need > 0 && !aligned16(workspace)) return MOE_ERR_ALIGN;
+  return cuda_status(moe::launch_special_bwd(
+      grad_out, topk_idx, topk_weights, x_active_mask, s->mask_ndim, ori_x, const_alpha_1,
+      const_alpha_2, const_v, grad_w, grad_ori_x, grad_alpha_1, grad_alpha_2, grad_v, workspace,
+      s->bs, s->k, s->h, s->num_experts, s->zero_expert_num, s->copy_expert_num,
+      s->const_expert_num, s->dtype, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_dispatch_bwd(const moe_shape* s, const void* grad_expand_in,
                             const int32_t* assist_info, const uint8_t* x_active_mask,
                             void* grad_x, void* stream) {

@@ -197,20 +197,15 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
       if (kind[u][j] == kSkip) continue;
       float m[8];
       pair_values<T16, SPECIAL>(a, kind[u][j], row[u][j], V, v, val[u][j], ori, m);
-      if (UNIT) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], m[i]);
-      } else {
-        const float w = wt[u][j];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, m[i]));
-      }
+      if (UNIT)
+        add8_rn(acc, m);
+      else
+        axpy8_rn(acc, wt[u][j], m);
     }
     if (!UNIT && a.shared != nullptr) {
       float sh[8];
       widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], sh[i]);
+      add8_rn(acc, sh);
     }
     st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
   }
@@ -342,10 +337,12 @@ __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pa
       float gf[8], yf[8], o[8];
       widen8<T16>(gv[u], gf);
       widen8<T16>(yv[u], yf);
+      const unsigned long long ww = pack2(w, w);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        d[i] = __fmaf_rn(gf[i], yf[i], d[i]);
-        o[i] = __fmul_rn(w, gf[i]);
+      for (int i = 0; i < 8; i += 2) {
+        const unsigned long long g2 = pack2(gf[i], gf[i + 1]);
+        unpack2(fma2_rn(g2, pack2(yf[i], yf[i + 1]), pack2(d[i], d[i + 1])), d[i], d[i + 1]);
+        unpack2(mul2_rn(ww, g2), o[i], o[i + 1]);
       }
       st_v4(ge + v, narrow8<T16>(o));
     }

@@ -53,6 +53,53 @@ __device__ __forceinline__ uint4 narrow8(const float (&f)[8]) {
   return v;
 }
 
+// ---- packed fp32 pairs (sm_100: one instruction, each lane rounded as the
+// scalar op would be) ----
+
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ void unpack2(unsigned long long v, float& lo, float& hi) {
+  lo = __uint_as_float(static_cast<uint32_t>(v));
+  hi = __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+__device__ __forceinline__ unsigned long long mul2_rn(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2_rn(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fma2_rn(unsigned long long a, unsigned long long b,
+                                                       unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// acc[i] = acc[i] + w * m[i] for 8 values, product and sum each rounded once.
+// The products are scalar __fmul_rn: a packed multiply followed by a packed
+// add was observed to lose the separate product rounding on B200 (outputs one
+// ulp off), while the scalar .rn multiply is never contracted. A lone add has
+// nothing to fuse with, so the sums are packed.
+__device__ __forceinline__ void axpy8_rn(float (&acc)[8], float w, const float (&m)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const unsigned long long p = pack2(__fmul_rn(w, m[i]), __fmul_rn(w, m[i + 1]));
+    unpack2(add2_rn(pack2(acc[i], acc[i + 1]), p), acc[i], acc[i + 1]);
+  }
+}
+
+// acc[i] = acc[i] + m[i] for 8 values.
+__device__ __forceinline__ void add8_rn(float (&acc)[8], const float (&m)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2)
+    unpack2(add2_rn(pack2(acc[i], acc[i + 1]), pack2(m[i], m[i + 1])), acc[i], acc[i + 1]);
+}
+
 // ---- global memory access ----
 
 // Read-only 16-byte load through the non-coherent path, not kept in L1.

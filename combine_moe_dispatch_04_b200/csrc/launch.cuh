@@ -73,6 +73,15 @@ struct CombineBwdArgs {
 };
 cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st);
 
+size_t special_bwd_workspace_bytes(int bs, int H, int Q);
+cudaError_t launch_special_bwd(const void* grad_out, const int32_t* topk_idx,
+                               const float* weights, const uint8_t* mask, int mask_ndim,
+                               const void* ori_x, const void* alpha1, const void* alpha2,
+                               const void* const_v, float* grad_w, void* grad_ori_x,
+                               float* grad_alpha1, float* grad_alpha2, float* grad_v,
+                               void* workspace, int bs, int K, int H, int E, int Z, int C, int Q,
+                               int dtype, cudaStream_t st);
+
 int sm_count();
 
 // Records err as the thread's last CUDA error; returns MOE_ERR_CUDA (MOE_OK for success).

@@ -24,13 +24,14 @@ namespace {
 
 // Classifies the K pairs of token t: e[k] = expert id of a routed active
 // pair, else -1. Returns the MOE_DEV_* bits of the row.
-__device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int (&e)[kMaxK]) {
+template <int KM>
+__device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int (&e)[KM]) {
   const int32_t* row = a.topk_idx + static_cast<size_t>(t) * a.K;
-  int ids[kMaxK];
+  int ids[KM];
   if ((a.K & 3) == 0 && (reinterpret_cast<uintptr_t>(a.topk_idx) & 15) == 0) {
     // rows of a multiple of 4 ids: 16-byte loads
 #pragma unroll
-    for (int q = 0; q < kMaxK / 4; ++q) {
+    for (int q = 0; q < KM / 4; ++q) {
       int4 v = make_int4(-1, -1, -1, -1);
       if (4 * q < a.K) v = __ldg(reinterpret_cast<const int4*>(row) + q);
       ids[4 * q] = v.x;
@@ -40,11 +41,11 @@ __device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int
     }
   } else {
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k) ids[k] = k < a.K ? __ldg(row + k) : -1;
+    for (int k = 0; k < KM; ++k) ids[k] = k < a.K ? __ldg(row + k) : -1;
   }
   uint32_t st = 0;
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k) {
+  for (int k = 0; k < KM; ++k) {
     e[k] = -1;
     if (k >= a.K) continue;
     const int id = ids[k];
@@ -65,11 +66,12 @@ __device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int
 }
 
 // words[warp * E + e] |= bit of this lane, for each routed pair of the lane.
-__device__ __forceinline__ void mark_words(uint32_t* words, int E, const int (&e)[kMaxK], int K) {
+template <int KM>
+__device__ __forceinline__ void mark_words(uint32_t* words, int E, const int (&e)[KM], int K) {
   const int warp = threadIdx.x >> 5;
   const uint32_t bit = 1u << (threadIdx.x & 31);
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k)
+  for (int k = 0; k < KM; ++k)
     if (k < K && e[k] >= 0) atomicOr(&words[warp * E + e[k]], bit);
 }
 
@@ -110,11 +112,12 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
 }
 
 // Writes both halves of assist_info for token t's pairs given their slots.
-__device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const int (&e)[kMaxK],
-                                            const int (&slot)[kMaxK]) {
+template <int KM>
+__device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const int (&e)[KM],
+                                            const int (&slot)[KM]) {
   const size_t A = static_cast<size_t>(a.A);
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k) {
+  for (int k = 0; k < KM; ++k) {
     if (k >= a.K) continue;
     const int tk = t * a.K + k;
     if (e[k] >= 0) a.assist[slot[k]] = tk;
@@ -125,6 +128,7 @@ __device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const in
 // ---------------------------------------------------------------------------
 // One-CTA layout for BS <= 1024: 32 warps, one token per thread.
 // Dynamic shared memory: words[32][E].
+template <int KM>
 __global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
   extern __shared__ uint32_t words[];
   __shared__ int offs[1024];
@@ -138,14 +142,14 @@ __global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
   __syncthreads();
 
   const int t = threadIdx.x;
-  int e[kMaxK];
+  int e[KM];
   uint32_t st = 0;
   if (t < a.bs) {
-    st = classify_row(a, t, e);
-    mark_words(words, E, e, a.K);
+    st = classify_row<KM>(a, t, e);
+    mark_words<KM>(words, E, e, a.K);
   } else {
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k) e[k] = -1;
+    for (int k = 0; k < KM; ++k) e[k] = -1;
   }
   if (st) atomicOr(&status, st);
   __syncthreads();
@@ -164,11 +168,11 @@ __global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
   __syncthreads();
 
   if (t < a.bs) {
-    int slot[kMaxK];
+    int slot[KM];
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k)
+    for (int k = 0; k < KM; ++k)
       slot[k] = (k < a.K && e[k] >= 0) ? offs[e[k]] + tile_rank(words, E, e[k]) : -1;
-    write_slots(a, t, e, slot);
+    write_slots<KM>(a, t, e, slot);
   }
   for (int s = total + threadIdx.x; s < a.A; s += blockDim.x) a.assist[s] = -1;
   if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
@@ -181,13 +185,14 @@ __global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
 // layout's outputs, and CTA c copies the rows of tokens [c * per, (c+1) * per)
 // to their slots: one thread per 16-byte vector, read once, stored K times.
 // Dynamic shared memory: words[32][E].
+template <int KM>
 __global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, const uint4* x,
                                                               uint4* expand_x, int V, int per) {
   extern __shared__ uint32_t words[];
   __shared__ int offs[1024];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
-  __shared__ int slot_sh[kLayoutSmallMaxTokens / 8][kMaxK];  // slots of this CTA's tokens
+  __shared__ int slot_sh[kLayoutSmallMaxTokens / 8][KM];  // slots of this CTA's tokens
   pdl_trigger();
   pdl_wait();
   const int E = a.E;
@@ -196,14 +201,14 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, cons
   if (threadIdx.x == 0) status = 0;
   __syncthreads();
   const int t = threadIdx.x;
-  int e[kMaxK];
+  int e[KM];
   uint32_t st = 0;
   if (t < a.bs) {
-    st = classify_row(a, t, e);
-    mark_words(words, E, e, a.K);
+    st = classify_row<KM>(a, t, e);
+    mark_words<KM>(words, E, e, a.K);
   } else {
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k) e[k] = -1;
+    for (int k = 0; k < KM; ++k) e[k] = -1;
   }
   if (st) atomicOr(&status, st);
   __syncthreads();
@@ -223,14 +228,14 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, cons
   __syncthreads();
   const int t0 = blockIdx.x * per;
   if (t < a.bs) {
-    int slot[kMaxK];
+    int slot[KM];
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k)
+    for (int k = 0; k < KM; ++k)
       slot[k] = (k < a.K && e[k] >= 0) ? offs[e[k]] + tile_rank(words, E, e[k]) : -1;
-    if (writer) write_slots(a, t, e, slot);
+    if (writer) write_slots<KM>(a, t, e, slot);
     if (t >= t0 && t < t0 + per) {
 #pragma unroll
-      for (int k = 0; k < kMaxK; ++k)
+      for (int k = 0; k < KM; ++k)
         if (k < a.K) slot_sh[t - t0][k] = slot[k];
     }
   }
@@ -269,6 +274,7 @@ __device__ __forceinline__ TileWs tile_ws(const LayoutArgs& a, int T) {
 constexpr int kTileWarps = kLayoutTileTokens / 32;
 
 // Phase 1: per-tile expert counts and status bits.
+template <int KM>
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutArgs a, int T) {
   extern __shared__ uint32_t words[];  // [kTileWarps][E]
   __shared__ uint32_t status;
@@ -280,9 +286,9 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutA
   __syncthreads();
   const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
   if (t < a.bs) {
-    int e[kMaxK];
-    const uint32_t st = classify_row(a, t, e);
-    mark_words(words, E, e, a.K);
+    int e[KM];
+    const uint32_t st = classify_row<KM>(a, t, e);
+    mark_words<KM>(words, E, e, a.K);
     if (st) atomicOr(&status, st);
   }
   __syncthreads();
@@ -302,15 +308,22 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutA
 // The CTA with first_cta writes the counts, prefix sums and status word.
 // Shared memory (dynamic): words[kTileWarps][E], base[E], total[E], and two
 // [G][E] partial-sum arrays (G * E <= blockDim).
+template <int KM>
 __device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile, bool first_cta,
                                            uint32_t* smem, int* warp_sums, uint32_t* status,
-                                           int (&e)[kMaxK], int (&slot)[kMaxK], int* grand_out) {
+                                           int (&e)[KM], int (&slot)[KM], int* grand_out) {
   const int E = a.E;
   uint32_t* words = smem;
   int* base = reinterpret_cast<int*>(smem + kTileWarps * E);
   int* total = base + E;
   for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
   if (threadIdx.x == 0) *status = 0;
+  // this thread's token: its ids are loaded now, so their latency overlaps
+  // the count-matrix loads below
+  const int t = tile * kLayoutTileTokens + threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < KM; ++k) e[k] = -1;
+  if (t < a.bs) classify_row<KM>(a, t, e);
   const TileWs ws = tile_ws(a, T);
   // Sum the count matrix over tiles: G groups of E threads split the tiles
   // (G = 1 when E >= blockDim), then one thread per expert adds the groups.
@@ -379,41 +392,35 @@ __device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile,
     a.ep_send_counts[E] = grand;
     if (a.dev_status) *a.dev_status = *status;
   }
-  const int t = tile * kLayoutTileTokens + threadIdx.x;
-#pragma unroll
-  for (int k = 0; k < kMaxK; ++k) e[k] = -1;
-  if (t < a.bs) {
-    classify_row(a, t, e);
-    mark_words(words, E, e, a.K);
-  }
+  if (t < a.bs) mark_words<KM>(words, E, e, a.K);  // words were zeroed before the syncs above
   __syncthreads();
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k)
+  for (int k = 0; k < KM; ++k)
     slot[k] = (t < a.bs && k < a.K && e[k] >= 0) ? base[e[k]] + tile_rank(words, E, e[k]) : -1;
   *grand_out = grand;
 }
 
 // Phase 2 as its own launch: every tile's slots, and -1 for the unused
 // slots [R, A).
+template <int KM>
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
   extern __shared__ uint32_t smem[];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
   pdl_trigger();
   pdl_wait();
-  int e[kMaxK], slot[kMaxK], grand;
-  tile_slots(a, T, blockIdx.x, blockIdx.x == 0, smem, warp_sums, &status, e, slot, &grand);
+  int e[KM], slot[KM], grand;
+  tile_slots<KM>(a, T, blockIdx.x, blockIdx.x == 0, smem, warp_sums, &status, e, slot, &grand);
   const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
-  if (t < a.bs) write_slots(a, t, e, slot);
+  if (t < a.bs) write_slots<KM>(a, t, e, slot);
   for (int s = grand + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
        s += gridDim.x * blockDim.x)
     a.assist[s] = -1;
 }
 
-}  // namespace
-
-cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
-                                  cudaStream_t st) {
+template <int KM>
+cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                    cudaStream_t st) {
   const int V = H / kVecElems;
   // at most kLayoutSmallMaxTokens / 8 tokens per CTA (the slot buffer's size)
   int blocks = sm_count();
@@ -423,14 +430,47 @@ cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expa
   if (per < 1) per = 1;
   blocks = a.bs > 0 ? (a.bs + per - 1) / per : 1;
   const size_t smem = 32u * a.E * sizeof(uint32_t);
-  if (smem > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel,
+  if (smem > 32 * 1024) {  // with the static buffers: opt in before the total passes 48 KB
+    cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel<KM>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  return launch_pdl(dispatch_small_kernel, dim3(blocks), dim3(1024), smem, st, a,
+  return launch_pdl(dispatch_small_kernel<KM>, dim3(blocks), dim3(1024), smem, st, a,
                     static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
+}
+
+template <int KM>
+cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t st) {
+  if (a.bs <= kLayoutSmallMaxTokens) {
+    const size_t smem = 32u * a.E * sizeof(uint32_t);
+    if (smem > 32 * 1024) {
+      cudaError_t err = cudaFuncSetAttribute(layout_small_kernel<KM>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+      if (err != cudaSuccess) return err;
+    }
+    return launch_pdl(layout_small_kernel<KM>, dim3(1), dim3(1024), smem, st, a);
+  }
+  const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
+  const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
+  const size_t smem_scatter =
+      smem_count + 2u * a.E * sizeof(int) + 2u * kLayoutTileTokens * sizeof(int);
+  cudaError_t err = launch_pdl(layout_count_kernel<KM>, dim3(T), dim3(kLayoutTileTokens),
+                               smem_count, st, a, T);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(layout_scatter_kernel<KM>, dim3(T), dim3(kLayoutTileTokens), smem_scatter,
+                    st, a, T);
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                  cudaStream_t st) {
+  if (a.K <= 2) return launch_dispatch_small_k<2>(a, x, expand_x, H, st);
+  if (a.K <= 4) return launch_dispatch_small_k<4>(a, x, expand_x, H, st);
+  if (a.K <= 8) return launch_dispatch_small_k<8>(a, x, expand_x, H, st);
+  return launch_dispatch_small_k<16>(a, x, expand_x, H, st);
 }
 
 size_t layout_workspace_bytes(int bs, int E) {
@@ -440,24 +480,10 @@ size_t layout_workspace_bytes(int bs, int E) {
 }
 
 cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st) {
-  if (a.bs <= kLayoutSmallMaxTokens) {
-    const size_t smem = 32u * a.E * sizeof(uint32_t);
-    if (smem > 48 * 1024) {
-      cudaError_t err = cudaFuncSetAttribute(layout_small_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-      if (err != cudaSuccess) return err;
-    }
-    return launch_pdl(layout_small_kernel, dim3(1), dim3(1024), smem, st, a);
-  }
-  const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
-  const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
-  const size_t smem_scatter = smem_count + 2u * a.E * sizeof(int) + 2u * kLayoutTileTokens * sizeof(int);
-  cudaError_t err = launch_pdl(layout_count_kernel, dim3(T), dim3(kLayoutTileTokens), smem_count,
-                               st, a, T);
-  if (err != cudaSuccess) return err;
-  return launch_pdl(layout_scatter_kernel, dim3(T), dim3(kLayoutTileTokens), smem_scatter, st,
-                    a, T);
+  if (a.K <= 2) return launch_layout_k<2>(a, st);
+  if (a.K <= 4) return launch_layout_k<4>(a, st);
+  if (a.K <= 8) return launch_layout_k<8>(a, st);
+  return launch_layout_k<16>(a, st);
 }
 
 }  // namespace moe

@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
   for (int t = blockIdx.x; t < bs; t += gridDim.x) {
     const uint4* xr = x + static_cast<size_t>(t) * (H / 8);
     const int32_t* slots = assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K;
-    const int my_slot = threadIdx.x < K ? __ldg(slots + threadIdx.x) : -1;
+    const int my_slot = lane < K ? __ldg(slots + lane) : -1;  // every warp holds the K slots
     float f[CPT][16];
     float amax = 0.0f;
 #pragma unroll
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       const int c = threadIdx.x + j * blockDim.x;
-      if (c >= C) continue;
+      const bool mine = c < C;  // every lane still takes part in the shuffles below
       uint32_t packed[4];
 #pragma unroll
       for (int w4 = 0; w4 < 4; ++w4) {
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           int q = 0;
-          if (amax != 0.0f) {
+          if (mine && amax != 0.0f) {
             float r = quant_code(f[j][w4 * 4 + b], scale, inv_scale);
             r = fminf(127.0f, fmaxf(-127.0f, r));
             q = __float2int_rn(r);
@@ -106,11 +106,21 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
       const uint4 val = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       for (int k = 0; k < K; ++k) {
         const int s = __shfl_sync(0xFFFFFFFFu, my_slot, k);
-        if (s >= 0) st_v4(out + static_cast<size_t>(s) * C + c, val);
+        if (mine && s >= 0) st_v4(out + static_cast<size_t>(s) * C + c, val);
       }
     }
-    if (threadIdx.x < K && my_slot >= 0) scales[my_slot] = scale;
+    if (warp == 0 && lane < K && my_slot >= 0) scales[my_slot] = scale;
   }
+}
+
+// Threads and 16-element chunks per thread for the int8 kernels: one chunk
+// per thread up to 256 threads, then 2 or 4 (H <= 16384, checked by the caller).
+void quant_shape(int H, int* threads, int* cpt) {
+  const int C = H / 16;
+  int t = (C + 31) / 32 * 32;
+  t = t > 256 ? 256 : t;
+  *threads = t;
+  *cpt = (C + t - 1) / t;
 }
 
 }  // namespace
@@ -126,12 +136,8 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
                       static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
                       a.bs, a.K, V, a.A);
   }
-  // One 16-value chunk per thread up to 256 threads, then 2 or 4 per thread
-  // (H <= 16384, checked by the caller).
-  const int C = a.H / 16;
-  int threads = (C + 31) / 32 * 32;
-  threads = threads > 256 ? 256 : threads;
-  const int cpt = (C + threads - 1) / threads;
+  int threads, cpt;
+  quant_shape(a.H, &threads, &cpt);
   const int cap = sm_count() * (2048 / threads);
   const int blocks = a.bs < cap ? a.bs : cap;
   const uint4* x = static_cast<const uint4*>(a.x);

@@ -206,6 +206,34 @@ moe_status moe_combine_bwd(const moe_shape* shape, const void* grad_out, const v
                            void* grad_expand, float* grad_w, void* stream);
 
 /*
+ * moe_combine_bwd_special — gradient of the combine Formula through the copy
+ * and const experts ([combine] Function, special expert use cases: copy
+ * Moe(ori_x) = ori_x, const Moe(ori_x) = alpha_1 * ori_x + alpha_2 * v), the
+ * part moe_combine_bwd leaves out. With g = grad_out[t], c = fl(w[t,k] * g):
+ *   grad_w[t,k]     = sum_h g * M(t,k)   (fp32) for copy and const pairs only;
+ *                     other entries of grad_w are not written (run
+ *                     moe_combine_bwd first for the routed pairs)
+ *   grad_ori_x[t]   = round16( sum over copy/const k, ascending, of c (copy)
+ *                     or fl(c * alpha_1[j]) (const) ), (BS, H) dtype; 0 for
+ *                     tokens without such pairs
+ *   grad_alpha_1[j] = sum over pairs of const j of c * ori_x[t]  (Q, H) fp32
+ *   grad_alpha_2[j] = S_j * v[j],  grad_v[j] = S_j * alpha_2[j],
+ *                     S_j = sum over pairs of const j of c        (Q, H) fp32
+ * Sums over tokens run in a fixed order (chunks of 256 tokens, then the
+ * chunks in order), so results are deterministic. ori_x is required; the
+ * const tensors and their gradients when Q > 0. workspace: device scratch of
+ * moe_combine_bwd_special_workspace_bytes() bytes (0 when Q = 0).
+ */
+size_t moe_combine_bwd_special_workspace_bytes(const moe_shape* shape);
+moe_status moe_combine_bwd_special(const moe_shape* shape, const void* grad_out,
+                                   const int32_t* topk_idx, const float* topk_weights,
+                                   const uint8_t* x_active_mask, const void* ori_x,
+                                   const void* const_alpha_1, const void* const_alpha_2,
+                                   const void* const_v, float* grad_w, void* grad_ori_x,
+                                   float* grad_alpha_1, float* grad_alpha_2, float* grad_v,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * moe_dispatch_bwd — gradient of the permute: every token gathers the
  * gradients of its slots, unweighted, summed in fp32 in ascending k:
  *   grad_x[t] = round16( sum_{k with a slot, active} grad_expand_in[slot(t,k)] )

@@ -59,6 +59,9 @@ def lib():
         L.oracle_combine_fwd.restype = None
         L.oracle_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, i, P, P, P]
         L.oracle_combine_bwd.restype = None
+        L.oracle_combine_bwd_special.argtypes = [i, i, i, i, i, i, i, i, P, P, P, P, i, P, P, P,
+                                                 P, P, P, P, P, P, P, P, P, P]
+        L.oracle_combine_bwd_special.restype = None
         L.oracle_dispatch_bwd.argtypes = [i, i, i, i, i, P, P, P, i, P]
         L.oracle_dispatch_bwd.restype = None
         _lib = L
@@ -169,6 +172,34 @@ def combine_bwd(grad_out, expand_x, topk_weights, assist_info, *, k, a_capacity,
                              _p(_c(topk_weights, np.float32)), _p(_c(assist_info, np.int32)),
                              _p(m), 0 if m is None else m.ndim, _p(ge), _p(gw), _p(mag))
     return ge, gw, mag
+
+
+def combine_bwd_special(grad_out, topk_idx, topk_weights, *, num_experts, dtype,
+                        zero_expert_num=0, copy_expert_num=0, const_expert_num=0, mask=None,
+                        ori_x=None, alpha1=None, alpha2=None, const_v=None):
+    """Backward of the copy/const experts. Returns a dict with grad_w (BS, K; entries
+    of other pairs are 0), abs_sum, grad_ori_x (BS, H) 16-bit, grad_alpha1/2, grad_v
+    (Q, H) fp32 and their abs sums."""
+    g = _c(grad_out, np.uint16)
+    bs, h = g.shape
+    idx = _c(topk_idx, np.int32)
+    k = idx.shape[1]
+    q = const_expert_num
+    m = _c(mask, np.uint8)
+    r = {"grad_w": np.zeros((bs, k), np.float32), "abs_sum": np.zeros((bs, k)),
+         "grad_ori_x": np.zeros((bs, h), np.uint16)}
+    for n in ("grad_alpha1", "grad_alpha2", "grad_v"):
+        r[n] = np.zeros((q, h), np.float32)
+    for n in ("abs_alpha1", "abs_alpha2", "abs_v"):
+        r[n] = np.zeros((q, h))
+    lib().oracle_combine_bwd_special(
+        bs, k, h, num_experts, zero_expert_num, copy_expert_num, q, DTYPE_CODES[dtype], _p(g),
+        _p(idx), _p(_c(topk_weights, np.float32)), _p(m), 0 if m is None else m.ndim,
+        _p(_c(ori_x, np.uint16)), _p(_c(alpha1, np.uint16)), _p(_c(alpha2, np.uint16)),
+        _p(_c(const_v, np.uint16)), _p(r["grad_w"]), _p(r["abs_sum"]), _p(r["grad_ori_x"]),
+        _p(r["grad_alpha1"]), _p(r["grad_alpha2"]), _p(r["grad_v"]), _p(r["abs_alpha1"]),
+        _p(r["abs_alpha2"]), _p(r["abs_v"]))
+    return r
 
 
 def dispatch_bwd(grad_in, assist_info, *, bs, k, a_capacity, dtype, mask=None):

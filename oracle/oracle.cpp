@@ -39,6 +39,14 @@
 //   R10 an id outside [0, N) or a repeat of an id earlier in its row makes the
 //      pair invalid: it is flagged in the status word and takes no part.
 //   R11 grad_w of a pair without a slot (masked, invalid or special) is 0.
+//   R17 backward of the special experts (same Formula, local terms): for a
+//      copy pair grad_w = <g, ori_x[t]>, for a const pair j
+//      grad_w = <g, alpha_1[j] ori_x[t] + alpha_2[j] v[j]> (m as in the forward);
+//      grad_ori_x[t] = round16(sum over copy/const pairs, k ascending, of
+//      c = fl(w g) for copy and fl(c alpha_1[j]) for const, accumulated in
+//      fp32); grad_alpha_1[j] = sum_{t,k} fl(w g) ori_x[t], grad_alpha_2[j] =
+//      sum_{t,k} fl(w g) v[j], grad_v[j] = sum_{t,k} fl(w g) alpha_2[j]
+//      (fp32 results of double sums). Zero experts contribute nothing.
 //   R15 combine with comm_quant_mode 2: each expanded row that returns to its
 //      token is quantised as in R9 (per row, scale = max|y| / 127) and used as
 //      the fp32 value q * scale; special experts and shared_expert_x are local
@@ -343,6 +351,91 @@ void oracle_combine_bwd(int bs, int K, int h, int a_capacity, int dtype,
       grad_w[tk] = static_cast<float>(dot);
       if (abs_sum) abs_sum[tk] = mag;
     }
+  }
+}
+
+// Backward of the special experts (reading R17). [combine] Function
+// (special expert use cases: copy Moe(ori_x) = ori_x, const Moe(ori_x) =
+// alpha_1 ori_x + alpha_2 v) differentiated through the weighted sum of the
+// Formula. grad_w gets entries only for copy and const pairs (others are left
+// as they are); abs_sum bounds the rounding error of grad_w as in the routed
+// backward. grad_ori_x is 16-bit; the alpha/v gradients are fp32 (Q, H) with
+// their abs sums for the tolerance.
+void oracle_combine_bwd_special(int bs, int K, int h, int num_experts, int zero_num, int copy_num,
+                                int const_num, int dtype, const uint16_t* grad_out,
+                                const int32_t* topk_idx, const float* topk_weights,
+                                const uint8_t* mask, int mask_ndim, const uint16_t* ori_x,
+                                const uint16_t* alpha1, const uint16_t* alpha2,
+                                const uint16_t* const_v, float* grad_w, double* abs_sum,
+                                uint16_t* grad_ori_x, float* grad_alpha1, float* grad_alpha2,
+                                float* grad_v, double* abs_alpha1, double* abs_alpha2,
+                                double* abs_v) {
+  const int n_ids = num_experts + zero_num + copy_num + const_num;
+  const int zero_end = num_experts + zero_num, copy_end = zero_end + copy_num;
+  const size_t qh = static_cast<size_t>(const_num) * h;
+  std::vector<double> ga1(qh, 0.0), ga2(qh, 0.0), gv(qh, 0.0), aa1(qh, 0.0), aa2(qh, 0.0),
+      av(qh, 0.0);
+  for (int t = 0; t < bs; ++t) {
+    const int32_t* row = topk_idx + static_cast<size_t>(t) * K;
+    const uint16_t* g = grad_out + static_cast<size_t>(t) * h;
+    const uint16_t* ox = ori_x ? ori_x + static_cast<size_t>(t) * h : nullptr;
+    for (int k = 0; k < K; ++k) {
+      const size_t tk = static_cast<size_t>(t) * K + k;
+      if (pair_problem(row, k, n_ids) || !pair_active(mask, mask_ndim, t, k, K)) continue;
+      const int32_t id = row[k];
+      if (id < zero_end) continue;  // routed (handled elsewhere) or zero expert
+      const float w = topk_weights[tk];
+      double dot = 0.0, mag = 0.0;
+      const size_t q = static_cast<size_t>(id - copy_end);
+      for (int j = 0; j < h; ++j) {
+        const float gj = load16(g, j, dtype), xj = load16(ox, j, dtype);
+        float m;
+        if (id < copy_end) {
+          m = xj;
+        } else {
+          const float p1 = load16(alpha1, q * h + j, dtype) * xj;
+          const float p2 = load16(alpha2, q * h + j, dtype) * load16(const_v, q * h + j, dtype);
+          m = p1 + p2;
+          const double c = static_cast<double>(w * gj);
+          ga1[q * h + j] += c * xj;
+          aa1[q * h + j] += std::fabs(c * xj);
+          ga2[q * h + j] += c * load16(const_v, q * h + j, dtype);
+          aa2[q * h + j] += std::fabs(c * load16(const_v, q * h + j, dtype));
+          gv[q * h + j] += c * load16(alpha2, q * h + j, dtype);
+          av[q * h + j] += std::fabs(c * load16(alpha2, q * h + j, dtype));
+        }
+        const double term = static_cast<double>(gj) * static_cast<double>(m);
+        dot += term;
+        mag += std::fabs(term);
+      }
+      grad_w[tk] = static_cast<float>(dot);
+      if (abs_sum) abs_sum[tk] = mag;
+    }
+    for (int j = 0; j < h; ++j) {
+      float acc = 0.0f;
+      const float gj = load16(g, j, dtype);
+      for (int k = 0; k < K; ++k) {
+        if (pair_problem(row, k, n_ids) || !pair_active(mask, mask_ndim, t, k, K)) continue;
+        const int32_t id = row[k];
+        if (id < zero_end) continue;
+        const float c = topk_weights[static_cast<size_t>(t) * K + k] * gj;
+        if (id < copy_end) {
+          acc = acc + c;
+        } else {
+          const size_t q = static_cast<size_t>(id - copy_end);
+          acc = acc + c * load16(alpha1, q * h + j, dtype);
+        }
+      }
+      if (grad_ori_x) grad_ori_x[static_cast<size_t>(t) * h + j] = store16(acc, dtype);
+    }
+  }
+  for (size_t i = 0; i < qh; ++i) {
+    grad_alpha1[i] = static_cast<float>(ga1[i]);
+    grad_alpha2[i] = static_cast<float>(ga2[i]);
+    grad_v[i] = static_cast<float>(gv[i]);
+    if (abs_alpha1) abs_alpha1[i] = aa1[i];
+    if (abs_alpha2) abs_alpha2[i] = aa2[i];
+    if (abs_v) abs_v[i] = av[i];
   }
 }
 

@@ -102,6 +102,11 @@ def test_other_entry_points_check_first():
     assert moe.moe_combine_fwd_comm_quant(s, *args2, 1, p, None) == moe.MOE_ERR_ARG
     assert moe.moe_combine_bwd(s, None, p, None, p, p, None, p, p, None) == moe.MOE_ERR_ARG
     assert moe.moe_dispatch_bwd(s, p, None, None, p, None) == moe.MOE_ERR_ARG
+    # special-expert backward: ori_x required; const tensors with const experts
+    assert moe.moe_combine_bwd_special(ctypes.byref(sp.c()), p, p, p, None, None, p, p, p, p, p,
+                                       p, p, p, p, 1 << 20, None) == moe.MOE_ERR_ARG
+    assert moe.moe_combine_bwd_special(ctypes.byref(sp.c()), p, p, p, None, p, None, p, p, p, p,
+                                       p, p, p, p, 1 << 20, None) == moe.MOE_ERR_ARG
 
 
 def test_sizes():

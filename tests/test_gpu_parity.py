@@ -245,3 +245,52 @@ def test_int8_quant_rounding_ties(dtype):
     torch.cuda.synchronize()
     assert np.array_equal(gpu_chain.host(qd), q)
     assert np.array_equal(gpu_chain.host(scd).view(np.uint32), sc.view(np.uint32))
+
+
+SPECIAL_BWD = [
+    W["special"].scaled(backward=True, name="special_full_bwd"),
+    W["special"].scaled(bs=1500, h=520, backward=True, mask_ndim=2, mask_false_p=0.2,
+                        name="special_mask_bwd"),
+    _custom("special_fp16_k16_bwd", bs=900, k=16, num_experts=24, zero_expert_num=2,
+            copy_expert_num=3, const_expert_num=4, h=264, dtype="fp16"),
+    _custom("special_copy_only_bwd", bs=700, k=4, num_experts=8, copy_expert_num=2, h=136),
+]
+
+
+@pytest.mark.parametrize("wl", SPECIAL_BWD, ids=lambda w: w.name)
+def test_special_expert_backward(wl):
+    """Backward through the copy/const experts against the oracle: grad_w of those
+    pairs within 1e-5 of max(|ref|, sum |terms|), grad_ori_x within one ulp, and the
+    alpha / v gradients within 1e-5 of their sums of |terms|."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    inp = workloads.generate(wl)
+    inp["ori_x"] = inp["x"]
+    dt = wl.dtype
+    ref = oracle.combine_bwd_special(
+        inp["grad_out"], inp["topk_idx"], inp["topk_weights"], num_experts=wl.num_experts,
+        dtype=dt, zero_expert_num=wl.zero_expert_num, copy_expert_num=wl.copy_expert_num,
+        const_expert_num=wl.const_expert_num, mask=inp["mask"], ori_x=inp["ori_x"],
+        alpha1=inp["alpha1"], alpha2=inp["alpha2"], const_v=inp["v"])
+    sh = gpu_chain.shape_of(wl)
+    dev, host = gpu_chain.dev, gpu_chain.host
+    gw, gox, ga1, ga2, gv = moe.combine_bwd_special(
+        sh, dev(inp["grad_out"], dt), dev(inp["topk_idx"]), dev(inp["topk_weights"]),
+        dev(inp["x"], dt), x_active_mask=dev(inp["mask"]), const_alpha_1=dev(inp["alpha1"], dt),
+        const_alpha_2=dev(inp["alpha2"], dt), const_v=dev(inp["v"], dt))
+    torch.cuda.synchronize()
+
+    def close(got, want, mag, name):
+        err = np.abs(got.astype(np.float64) - want.astype(np.float64))
+        bound = 1e-5 * np.maximum(np.abs(want.astype(np.float64)), mag)
+        assert np.all(err <= bound), (name, float((err / np.maximum(bound, 1e-30)).max()))
+
+    close(host(gw), ref["grad_w"], ref["abs_sum"], "grad_w")
+    d = gpu_chain.ulp_dist(host(gox), ref["grad_ori_x"])
+    assert d.max() <= 1 and (d == 0).mean() == 1.0
+    if wl.const_expert_num:
+        close(host(ga1), ref["grad_alpha1"], ref["abs_alpha1"], "grad_alpha1")
+        close(host(ga2), ref["grad_alpha2"], ref["abs_alpha2"], "grad_alpha2")
+        close(host(gv), ref["grad_v"], ref["abs_v"], "grad_v")

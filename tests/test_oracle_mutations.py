@@ -12,7 +12,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.cpp")
 PIN_TESTS = ["tests/test_oracle_layout.py", "tests/test_oracle_quant.py",
-             "tests/test_oracle_combine.py"]
+             "tests/test_oracle_combine.py", "tests/test_oracle_special_bwd.py"]
 
 # (name, text in oracle.cpp, replacement)
 MUTATIONS = [
@@ -20,10 +20,10 @@ MUTATIONS = [
      "if (shared_x) acc = acc + load16(shared_x",
      "if (false) acc = acc + load16(shared_x"),
     ("const_sign",
-     "m = p1 + p2;", "m = p1 - p2;"),
+     "m = p1 + p2;\n        }\n        float prod", "m = p1 - p2;\n        }\n        float prod"),
     ("const_operand_swapped",
-     "float p1 = load16(alpha1, q * h + j, dtype) *",
-     "float p1 = load16(alpha2, q * h + j, dtype) *"),
+     "float p1 = load16(alpha1, q * h + j, dtype) *\n                     load16(ori_x",
+     "float p1 = load16(alpha2, q * h + j, dtype) *\n                     load16(ori_x"),
     ("unstable_segment_order",
      "[](const Pair& a, const Pair& b) { return a.e < b.e; }",
      "[](const Pair& a, const Pair& b) { return a.e < b.e || (a.e == b.e && a.t > b.t); }"),
@@ -37,7 +37,8 @@ MUTATIONS = [
      "      for (int k = 0; k < K; ++k) {\n        if (pair_problem(row, k, n_ids)) continue;",
      "      for (int k = K - 1; k >= 0; --k) {\n        if (pair_problem(row, k, n_ids)) continue;"),
     ("grad_w_weighted",
-     "dot += term;", "dot += w * term;"),
+     "        dot += term;\n        mag += std::fabs(term);\n      }\n      grad_w[tk] = static_cast<float>(dot);\n      if (abs_sum) abs_sum[tk] = mag;\n    }\n  }\n}",
+     "        dot += w * term;\n        mag += std::fabs(term);\n      }\n      grad_w[tk] = static_cast<float>(dot);\n      if (abs_sum) abs_sum[tk] = mag;\n    }\n  }\n}"),
     ("scan_off_by_one",
      "ep_send_counts[e + 1] = ep_send_counts[e] + expert_token_nums[e];",
      "ep_send_counts[e + 1] = ep_send_counts[e] + expert_token_nums[e] + (e == 0);"),
@@ -50,6 +51,12 @@ MUTATIONS = [
     ("int8_roundtrip_skipped",
      "  if (amax == 0.0f) return 0.0f;\n  const float scale = amax / 127.0f;",
      "  if (amax >= 0.0f) return y;\n  const float scale = amax / 127.0f;"),
+    ("special_bwd_alpha1_dropped",
+     "          acc = acc + c * load16(alpha1, q * h + j, dtype);",
+     "          acc = acc + c;"),
+    ("special_bwd_v_grad_operand",
+     "          gv[q * h + j] += c * load16(alpha2, q * h + j, dtype);",
+     "          gv[q * h + j] += c * load16(const_v, q * h + j, dtype);"),
     ("duplicate_ids_accepted",
      "    if (row[j] == id) return ST_DUP_ID;", "    if (false) return ST_DUP_ID;"),
 ]
