@@ -54,6 +54,8 @@ def lib():
         L.oracle_dispatch_permute.restype = None
         L.oracle_dispatch_permute_quant.argtypes = [i, i, i, i, i, P, P, P, P]
         L.oracle_dispatch_permute_quant.restype = None
+        L.oracle_dispatch_permute_quant_smooth.argtypes = [i, i, i, i, i, P, P, P, P, P, P]
+        L.oracle_dispatch_permute_quant_smooth.restype = None
         L.oracle_combine_fwd.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, i,
                                          P, P, P, P, P, i, P]
         L.oracle_combine_fwd.restype = None
@@ -132,6 +134,19 @@ def dispatch_permute_quant(x, assist_info, k, a_capacity, dtype):
     sc = np.zeros(a_capacity, np.float32)
     lib().oracle_dispatch_permute_quant(bs, k, h, a_capacity, DTYPE_CODES[dtype], _p(x),
                                         _p(_c(assist_info, np.int32)), _p(q), _p(sc))
+    return q, sc
+
+
+def dispatch_permute_quant_smooth(x, topk_idx, smooth_scales, assist_info, a_capacity, dtype):
+    """int8 permute of x[t] * smooth_scales[e] per routed pair: (codes (A, H), scales (A,))."""
+    x = _c(x, np.uint16)
+    bs, h = x.shape
+    idx = _c(topk_idx, np.int32)
+    q = np.zeros((a_capacity, h), np.int8)
+    sc = np.zeros(a_capacity, np.float32)
+    lib().oracle_dispatch_permute_quant_smooth(
+        bs, idx.shape[1], h, a_capacity, DTYPE_CODES[dtype], _p(x), _p(idx),
+        _p(_c(smooth_scales, np.float32)), _p(_c(assist_info, np.int32)), _p(q), _p(sc))
     return q, sc
 
 

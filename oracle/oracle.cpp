@@ -47,6 +47,9 @@
 //      fp32); grad_alpha_1[j] = sum_{t,k} fl(w g) ori_x[t], grad_alpha_2[j] =
 //      sum_{t,k} fl(w g) v[j], grad_v[j] = sum_{t,k} fl(w g) alpha_2[j]
 //      (fp32 results of double sums). Zero experts contribute nothing.
+//   R18 dispatch quantisation with smooth scales (E, H) fp32: the row of pair
+//      (t, k) routed to expert e is y = fl(x[t] * scales[e]) (fp32 product),
+//      then quantised per row as in R9; each slot has its own codes and scale.
 //   R15 combine with comm_quant_mode 2: each expanded row that returns to its
 //      token is quantised as in R9 (per row, scale = max|y| / 127) and used as
 //      the fp32 value q * scale; special experts and shared_expert_x are local
@@ -255,6 +258,43 @@ static float int8_roundtrip(float y, float amax) {
   float q = std::nearbyint(y / scale);
   q = std::min(127.0f, std::max(-127.0f, q));
   return q * scale;
+}
+
+// Dispatch permute with int8 quantisation of smooth-scaled rows (reading
+// R18; [combine] Example, graph mode: quant_mode 2 with a scales tensor of
+// shape (E, H)).
+void oracle_dispatch_permute_quant_smooth(int bs, int K, int h, int a_capacity, int dtype,
+                                          const uint16_t* x, const int32_t* topk_idx,
+                                          const float* smooth_scales,
+                                          const int32_t* assist_info, int8_t* expand_q,
+                                          float* dynamic_scales) {
+  std::fesetround(FE_TONEAREST);
+  const size_t A = static_cast<size_t>(a_capacity);
+  std::vector<float> y(h);
+  for (int t = 0; t < bs; ++t) {
+    const uint16_t* xr = x + static_cast<size_t>(t) * h;
+    for (int k = 0; k < K; ++k) {
+      const int32_t s = assist_info[A + static_cast<size_t>(t) * K + k];
+      if (s < 0) continue;
+      const int32_t e = topk_idx[static_cast<size_t>(t) * K + k];
+      const float* se = smooth_scales + static_cast<size_t>(e) * h;
+      float amax = 0.0f;
+      for (int j = 0; j < h; ++j) {
+        y[j] = load16(xr, j, dtype) * se[j];
+        amax = std::max(amax, std::fabs(y[j]));
+      }
+      const float scale = amax / 127.0f;
+      for (int j = 0; j < h; ++j) {
+        float r = 0.0f;
+        if (amax != 0.0f) {
+          r = std::nearbyint(y[j] / scale);
+          r = std::min(127.0f, std::max(-127.0f, r));
+        }
+        expand_q[static_cast<size_t>(s) * h + j] = static_cast<int8_t>(r);
+      }
+      dynamic_scales[s] = scale;
+    }
+  }
 }
 
 // Combine forward. [combine] Function (Formula: weighted sum of the returned

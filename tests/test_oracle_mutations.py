@@ -57,6 +57,12 @@ MUTATIONS = [
     ("special_bwd_v_grad_operand",
      "          gv[q * h + j] += c * load16(alpha2, q * h + j, dtype);",
      "          gv[q * h + j] += c * load16(const_v, q * h + j, dtype);"),
+    ("smooth_expert_of_first_k",
+     "const int32_t e = topk_idx[static_cast<size_t>(t) * K + k];\n      const float* se",
+     "const int32_t e = topk_idx[static_cast<size_t>(t) * K];\n      const float* se"),
+    ("smooth_amax_unscaled",
+     "        amax = std::max(amax, std::fabs(y[j]));",
+     "        amax = std::max(amax, std::fabs(load16(xr, j, dtype)));"),
     ("duplicate_ids_accepted",
      "    if (row[j] == id) return ST_DUP_ID;", "    if (false) return ST_DUP_ID;"),
 ]
