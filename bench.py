@@ -55,7 +55,10 @@ def byte_model(wl: workloads.Workload, r: int, ori_tokens: int) -> dict:
     slot_map = 4 * pairs
     m = {}
     m["layout"] = 4 * pairs + mask + 4 * (wl.a_capacity + pairs) + 4 * (2 * wl.num_experts + 1)
-    if wl.quant_mode == 2:
+    if wl.quant_mode == 2 and wl.smooth:
+        # x once, the smooth factors once, per slot its pair, id, int8 row and scale
+        m["permute"] = bs * row + 4 * wl.num_experts * h + 8 * r + r * h + 4 * r
+    elif wl.quant_mode == 2:
         m["permute"] = bs * row + slot_map + r * h + 4 * r
     else:
         m["permute"] = bs * row + slot_map + r * row
@@ -225,7 +228,12 @@ def oracle_chain_timed(inputs: dict, sample_tokens: int) -> tuple[float, int]:
     counts, send, assist, _ = oracle.dispatch_layout(inp["topk_idx"], sub.num_experts, sub.n_ids,
                                                      sub.a_capacity, inp["mask"])
     if sub.quant_mode == 2:
-        q, sc = oracle.dispatch_permute_quant(inp["x"], assist, sub.k, sub.a_capacity, sub.dtype)
+        if sub.smooth:
+            q, sc = oracle.dispatch_permute_quant_smooth(inp["x"], inp["topk_idx"], inp["smooth"],
+                                                         assist, sub.a_capacity, sub.dtype)
+        else:
+            q, sc = oracle.dispatch_permute_quant(inp["x"], assist, sub.k, sub.a_capacity,
+                                                  sub.dtype)
         secs += time.perf_counter() - t
         y = workloads.expert_forward(inp, q, sc)
     else:
@@ -308,6 +316,8 @@ def main():
                     help="combine forward with comm_quant_mode 2 (int8 round trip)")
     ap.add_argument("--with-backward", action="store_true",
                     help="add the backward steps to a forward-only workload")
+    ap.add_argument("--smooth-quant", action="store_true",
+                    help="int8 dispatch of x * smooth_scales[e] (int8 workloads only)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step eagerly instead of replaying a CUDA graph of it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -316,6 +326,10 @@ def main():
     wl = workloads.BY_NAME[args.workload]
     if args.with_backward and not wl.backward:
         wl = wl.scaled(backward=True, name=wl.name + "+backward")
+    if args.smooth_quant:
+        if wl.quant_mode != 2 or args.fused_dispatch:
+            ap.error("--smooth-quant needs an int8 workload and the separate permute call")
+        wl = wl.scaled(smooth=True, name=wl.name + "+smooth")
     if args.impl == "reference":
         return run_reference(args, wl)
     if args.warmup < 3:
@@ -356,11 +370,14 @@ def main():
                    const_expert_num=wl.const_expert_num, a_capacity=wl.a_capacity,
                    dtype=workloads.DTYPE_CODES[dt], mask_ndim=wl.mask_ndim)
     d = {k: up(inputs[k]) for k in ("topk_idx", "topk_weights", "x", "mask", "shared", "ori_x",
-                                     "alpha1", "alpha2", "v", "grad_out")}
+                                     "alpha1", "alpha2", "v", "grad_out", "smooth")}
     ws = moe.layout_workspace(sh, dev)
     lay = moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws)
     qm = wl.quant_mode
-    expand, scales = moe.dispatch_permute(sh, d["x"], lay, qm)
+    if wl.smooth:
+        expand, scales = moe.dispatch_permute_smooth(sh, d["x"], d["topk_idx"], lay, d["smooth"])
+    else:
+        expand, scales = moe.dispatch_permute(sh, d["x"], lay, qm)
     torch.cuda.synchronize()
     r = int(lay.ep_send_counts[-1].item())
     # untimed expert stand-ins, computed once on the host from the GPU's dispatch output
@@ -412,6 +429,10 @@ def main():
             ("permute", lambda st: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
                                                      dynamic_scales=scales, stream=st)),
         ]
+        if wl.smooth:
+            calls[1] = ("permute", lambda st: moe.dispatch_permute_smooth(
+                sh, d["x"], d["topk_idx"], lay, d["smooth"], expand_x=expand,
+                dynamic_scales=scales, stream=st))
     calls += [
         ("combine_fwd", lambda st: moe.combine_fwd(
             sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
@@ -484,15 +505,24 @@ def main():
         dispatch_launches = (2 if tiled else 1) + 1
     special_bwd_launches = 0
     if "combine_bwd_special" in bytes_per:
-        special_bwd_launches = 2 + (2 if wl.const_expert_num else 0)
+        special_bwd_launches = 1 + (2 if wl.const_expert_num else 0)
     launches_per_step = dispatch_launches + 1 + (2 if wl.backward else 0) + special_bwd_launches
 
-    # L2 flush between steps: write a buffer twice the size of L2
+    # L2 flush between steps: write a buffer twice the size of L2, then read
+    # another one as large, so the step starts with none of its data in L2 and
+    # without the flush's dirty lines, whose write-back would otherwise be
+    # billed to the step. Both run before the step's start event.
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
     flush = torch.empty(2 * l2 // 4, dtype=torch.int32, device=dev)
+    sweep = torch.zeros(2 * l2 // 4, dtype=torch.int32, device=dev)
+    sweep_out = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        torch.sum(sweep, dim=0, dtype=torch.int64, out=sweep_out)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize()
 
@@ -514,7 +544,7 @@ def main():
                 step_graphs.append(plain)
             marks.append(m)
         for _ in range(2):  # warm the graphs
-            flush.zero_()
+            flush_l2()
             step(graph=plain)
         torch.cuda.synchronize()
     else:
@@ -533,7 +563,7 @@ def main():
     torch.cuda.synchronize()
     t0 = time.time()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         if step_graphs[i] is not None:
             step({"start": marks[i]["start"], "end": marks[i]["end"]}, graph=step_graphs[i])
         else:
@@ -555,7 +585,7 @@ def main():
     # events around every kernel, which costs each kernel its launch overlap.
     diag = [new_marks(kernels) for _ in range(min(args.steps, 20))]
     for m in diag:
-        flush.zero_()
+        flush_l2()
         step(m)
     torch.cuda.synchronize()
     per_kernel_ms = {k: [m[k][0].elapsed_time(m[k][1]) for m in diag] for k in kernels}
@@ -615,9 +645,12 @@ def main():
                        "num_experts": wl.num_experts, "routed_pairs": r,
                        "a_capacity": wl.a_capacity, "parallelism": "replicas",
                        "fused_dispatch": bool(args.fused_dispatch),
+                       "smooth_quant": bool(wl.smooth),
                        "combine_comm_quant_mode": cq,
                        "launch": "CUDA graph of the step" if use_graph else "eager launches",
-                       "l2": "flushed before every step (write of 2x L2), outside the step events"},
+                       "l2": "flushed before every step (write of 2x L2, then a read of another 2x L2 so "
+                             "no dirty flush lines are written back inside the step), outside "
+                             "the step events"},
             "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
             "hbm_frac_of_measured": round(gbs / peak, 4),
             "algorithmic_bytes_per_step": bytes_step,

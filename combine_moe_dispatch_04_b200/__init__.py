@@ -27,7 +27,7 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd",
            "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes",
            "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
-           "moe_combine_bwd_special_workspace_bytes")
+           "moe_combine_bwd_special_workspace_bytes", "moe_dispatch_permute_smooth")
 
 
 class MoeShape(ctypes.Structure):
@@ -59,6 +59,7 @@ def _load():
     L.moe_layout_workspace_bytes.restype = ctypes.c_size_t
     L.moe_dispatch_layout.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_dispatch_permute.argtypes = [S, P, P, P, I, P, P, P]
+    L.moe_dispatch_permute_smooth.argtypes = [S, P, P, P, P, P, P, P, P]
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_combine_fwd_comm_quant.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P]
     L.moe_dispatch.argtypes = [S, P, P, P, I, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -87,6 +88,7 @@ moe_assist_info_elems = _lib.moe_assist_info_elems
 moe_layout_workspace_bytes = _lib.moe_layout_workspace_bytes
 moe_dispatch_layout = _lib.moe_dispatch_layout
 moe_dispatch_permute = _lib.moe_dispatch_permute
+moe_dispatch_permute_smooth = _lib.moe_dispatch_permute_smooth
 moe_combine_fwd = _lib.moe_combine_fwd
 moe_combine_bwd = _lib.moe_combine_bwd
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
@@ -248,6 +250,22 @@ def dispatch_permute(shape: Shape, x, layout: Layout, comm_quant_mode: int = 0, 
     _check("moe_dispatch_permute", moe_dispatch_permute(
         ctypes.byref(shape.c()), _ptr(x), _ptr(layout.assist_info), _ptr(layout.ep_send_counts),
         comm_quant_mode, _ptr(expand_x), _ptr(dynamic_scales), _stream(stream)))
+    return expand_x, dynamic_scales
+
+
+def dispatch_permute_smooth(shape: Shape, x, topk_idx, layout: Layout, smooth_scales, *,
+                            expand_x=None, dynamic_scales=None, stream=None):
+    """int8 dispatch of x[t] * smooth_scales[e] per slot: (expand_x (A, H) int8, scales (A,))."""
+    import torch
+
+    if expand_x is None:
+        expand_x = torch.empty(shape.A, shape.h, dtype=torch.int8, device=x.device)
+    if dynamic_scales is None:
+        dynamic_scales = torch.empty(shape.A, dtype=torch.float32, device=x.device)
+    _check("moe_dispatch_permute_smooth", moe_dispatch_permute_smooth(
+        ctypes.byref(shape.c()), _ptr(x), _ptr(topk_idx), _ptr(layout.assist_info),
+        _ptr(layout.ep_send_counts), _ptr(smooth_scales), _ptr(expand_x), _ptr(dynamic_scales),
+        _stream(stream)))
     return expand_x, dynamic_scales
 
 

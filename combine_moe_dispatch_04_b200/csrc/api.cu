@@ -139,6 +139,35 @@ moe_status moe_dispatch_permute(const moe_shape* s, const void* x, const int32_t
   return cuda_status(moe::launch_permute(a, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_dispatch_permute_smooth(const moe_shape* s, const void* x,
+                                       const int32_t* topk_idx, const int32_t* assist_info,
+                                       const int32_t* ep_send_counts, const float* smooth_scales,
+                                       void* expand_x, float* dynamic_scales, void* stream) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (s->bs > 0 && (x == nullptr || topk_idx == nullptr || assist_info == nullptr ||
+                    ep_send_counts == nullptr || smooth_scales == nullptr ||
+                    expand_x == nullptr || dynamic_scales == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(expand_x) || !aligned16(smooth_scales)) return MOE_ERR_ALIGN;
+  if (s->h % 16 != 0) return MOE_ERR_ALIGN;
+  if (s->h > 16384) return MOE_ERR_UNSUPPORTED;
+  moe::PermuteArgs a;
+  a.x = x;
+  a.assist = assist_info;
+  a.expand_x = expand_x;
+  a.scales = dynamic_scales;
+  a.bs = s->bs;
+  a.K = s->k;
+  a.H = s->h;
+  a.A = s->a_capacity;
+  a.dtype = s->dtype;
+  a.quant_mode = 2;
+  return cuda_status(moe::launch_permute_smooth(a, topk_idx, smooth_scales, ep_send_counts,
+                                                s->num_experts,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_dispatch(const moe_shape* s, const int32_t* topk_idx, const uint8_t* x_active_mask,
                         const void* x, int comm_quant_mode, int32_t* expert_token_nums,
                         int32_t* ep_send_counts, int32_t* assist_info, uint32_t* dev_status,

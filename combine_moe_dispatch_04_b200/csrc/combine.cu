@@ -276,11 +276,7 @@ __global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
           const float scale = __fdiv_rn(mx, 127.0f);
           const float inv_scale = 1.0f / scale;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float q = mx == 0.0f ? 0.0f : quant_code(y[i], scale, inv_scale);
-            q = fminf(127.0f, fmaxf(-127.0f, q));
-            m[i] = __fmul_rn(q, scale);
-          }
+          for (int i = 0; i < 8; ++i) m[i] = quant_roundtrip(y[i], mx, scale, inv_scale);
         } else {
           pair_values<T16, SPECIAL>(a, pm.kind, pm.row, V, v, make_uint4(0, 0, 0, 0), ori, m);
         }
@@ -296,6 +292,117 @@ __global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
       st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
     }
     __syncthreads();  // meta, red and rmax are reused by the next token
+  }
+}
+
+// The same round trip with the token's rows held in registers: one CTA per
+// token (grid-stride), thread v owning vector v of every row (V <= 512,
+// K <= 8). Every warp classifies the token's pairs itself (lanes 0..K-1) and
+// spreads them by shuffle; all routed rows are loaded at once, each row's
+// max|y| is reduced (shuffles, then one shared-memory step), and the same
+// registers are dequantised and accumulated in ascending k. Shared arrays are
+// double-buffered by token parity, so two barriers per token suffice.
+constexpr int kQ8rMaxVectors = 512;
+
+template <typename T16, int KMAX, bool SPECIAL>
+__global__ void __launch_bounds__(kQ8rMaxVectors, 1) combine_fwd_q8r_kernel(CombineArgs a) {
+  __shared__ float red[2][kQ8rMaxVectors / 32][KMAX];
+  __shared__ float rmax[2][KMAX];
+  pdl_trigger();
+  pdl_wait();
+  const int V = a.H / kVecElems;
+  const int K = a.K;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int v = threadIdx.x;
+  const bool act = v < V;
+  const uint4* Y = static_cast<const uint4*>(a.expand_x);
+  int buf = 0;
+  for (int t = blockIdx.x; t < a.bs; t += gridDim.x) {
+    PairMeta pm{kSkip, 0, 1.0f};
+    if (lane < K) pm = classify_pair<SPECIAL, false, false>(a, t, lane);
+    if (SPECIAL) {
+      // a repeat of an id held by an earlier lane takes no part
+      const int id = lane < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + lane) : -1;
+      bool dup = false;
+#pragma unroll
+      for (int jj = 0; jj < KMAX; ++jj) {
+        const int other = __shfl_sync(0xFFFFFFFFu, id, jj);
+        dup |= jj < lane && other == id;
+      }
+      if (dup) pm.kind = kSkip;
+    }
+    int kind[KMAX], row[KMAX];
+    float w[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      kind[j] = __shfl_sync(0xFFFFFFFFu, pm.kind, j);
+      row[j] = __shfl_sync(0xFFFFFFFFu, pm.row, j);
+      w[j] = __shfl_sync(0xFFFFFFFFu, pm.w, j);
+      if (j >= K) kind[j] = kSkip;
+    }
+    uint4 val[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      val[j] = make_uint4(0, 0, 0, 0);
+      if (act && kind[j] == kRouted) val[j] = ld_nc_v4(Y + static_cast<size_t>(row[j]) * V + v);
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (kind[j] != kRouted) continue;  // CTA-uniform
+      float f[8];
+      widen8<T16>(val[j], f);
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(f[i]));
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+      if (lane == 0) red[buf][warp][j] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x < K) {
+      float mx = 0.0f;
+      for (int ww = 0; ww < nwarps; ++ww) mx = fmaxf(mx, red[buf][ww][threadIdx.x]);
+      rmax[buf][threadIdx.x] = mx;
+    }
+    __syncthreads();
+    if (act) {
+      const size_t item = static_cast<size_t>(t) * V + v;
+      float ori[8];
+      if (SPECIAL) {
+        bool need = false;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) need |= kind[j] == kCopy || kind[j] == kConst;
+        if (need) widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
+      }
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (kind[j] == kSkip) continue;
+        float m[8];
+        if (kind[j] == kRouted) {
+          const float mx = rmax[buf][j];
+          const float scale = __fdiv_rn(mx, 127.0f);
+          const float inv_scale = 1.0f / scale;
+          float y[8];
+          widen8<T16>(val[j], y);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m[i] = quant_roundtrip(y[i], mx, scale, inv_scale);
+        } else {
+          pair_values<T16, SPECIAL>(a, kind[j], row[j], V, v, val[j], ori, m);
+        }
+        axpy8_rn(acc, w[j], m);
+      }
+      if (a.shared != nullptr) {
+        float sh[8];
+        widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
+        add8_rn(acc, sh);
+      }
+      st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
+    }
+    buf ^= 1;
   }
 }
 
@@ -364,18 +471,21 @@ __global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(CombineBwdArgs
     combine_bwd_pair<T16>(a, pair, lane);
 }
 
-// Resident blocks per SM of a kernel (occupancy API), cached per kernel.
+// Resident blocks per SM of a kernel (occupancy API), cached per kernel and
+// block size (a multiple of 32, at most 1024); each kernel is always launched
+// with the same shared memory size.
 template <auto Kernel>
 int blocks_per_sm(int threads, size_t smem) {
-  static int cached = 0;
-  if (cached == 0) {
+  static int cached[33] = {};
+  const int slot = threads >= 1024 ? 32 : threads / 32;
+  if (cached[slot] == 0) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
         n < 1)
       n = 1;
-    cached = n;
+    cached[slot] = n;
   }
-  return cached;
+  return cached[slot];
 }
 
 template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
@@ -406,9 +516,24 @@ cudaError_t launch_fwd_t(const CombineArgs& a, cudaStream_t st) {
   return launch_fwd_k<T16, false, false>(a, st);
 }
 
+template <typename T16, bool SPECIAL, int KMAX>
+cudaError_t launch_fwd_q8r(const CombineArgs& a, cudaStream_t st) {
+  const int V = a.H / kVecElems;
+  const int threads = (V + 31) / 32 * 32;
+  constexpr auto kernel = combine_fwd_q8r_kernel<T16, KMAX, SPECIAL>;
+  const int cap = sm_count() * blocks_per_sm<kernel>(threads, 0);
+  const int blocks = a.bs < cap ? a.bs : cap;
+  return launch_pdl(kernel, dim3(blocks), dim3(threads), 0, st, a);
+}
+
 template <typename T16, bool SPECIAL>
 cudaError_t launch_fwd_q8_t(const CombineArgs& a, cudaStream_t st) {
   const int V = a.H / kVecElems;
+  if (V <= kQ8rMaxVectors && a.K <= 8) {
+    if (a.K <= 2) return launch_fwd_q8r<T16, SPECIAL, 2>(a, st);
+    if (a.K <= 4) return launch_fwd_q8r<T16, SPECIAL, 4>(a, st);
+    return launch_fwd_q8r<T16, SPECIAL, 8>(a, st);
+  }
   const int threads = V < 256 ? (V + 31) / 32 * 32 : 256;
   const int cap = sm_count() * (2048 / threads);
   const int blocks = a.bs < cap ? a.bs : cap;

@@ -149,17 +149,59 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// rne(fl32(y / scale)) for |y| <= max|row| and scale = fl32(max|row| / 127),
-// so |y / scale| <= 127 (1 + 2^-23). r = y * fl32(1 / scale) and the IEEE
-// quotient fl32(y / scale) both lie within 127 * 3 * 2^-24 < 2^-15 of the
-// exact quotient; when r is at least 2^-14 away from every half-integer, both
-// round to the same integer, so rint(r) is the answer. Otherwise (rare: near
-// a rounding tie) the IEEE division decides.
-__device__ __forceinline__ float quant_code(float y, float scale, float inv_scale) {
-  const float r = y * inv_scale;
-  const float frac = r - floorf(r);
-  if (fabsf(frac - 0.5f) > 0.00006103515625f) return rintf(r);  // 2^-14
-  return rintf(__fdiv_rn(y, scale));
+// Integer rounding on the FMA pipe: for |r| <= 2^22, r + 1.5 * 2^23 lies in
+// [2^23, 2^24), where fp32 values are spaced 1 apart, so the add itself rounds
+// r to an integer n (round-to-nearest-even), and n sits in the low mantissa
+// bits: for |n| <= 127 the low byte is n in two's complement.
+constexpr float kRoundBias = 12582912.0f;        // 1.5 * 2^23
+constexpr float kTieGuard = 0.49993896484375f;   // 0.5 - 2^-14
+constexpr float kMinNormal = 1.17549435e-38f;    // 2^-126
+
+// The int8 code clamp(rne(fl32(y / scale)), -127, 127), returned biased (as
+// code + 1.5 * 2^23, see above), for scale = fl32(max|row| / 127) > 0 and
+// |y| <= max|row|, so |y / scale| <= 127 (1 + 2^-23). With fast set (scale
+// normal, inv_scale = fl32(1 / scale)), r = y * inv_scale and the IEEE quotient
+// fl32(y / scale) both lie within 127 * 3 * 2^-24 < 2^-15 of the exact
+// quotient; when r, clamped to [-127, 127], is more than 2^-14 from every
+// half-integer, both round and clamp to the same integer (the bounds are
+// integers, so clamping before or after rounding agrees). Otherwise (rare:
+// near a rounding tie) the IEEE division decides.
+__device__ __forceinline__ float quant_code_biased(float y, float scale, float inv_scale,
+                                                   bool fast) {
+  if (fast) {
+    const float r = fminf(127.0f, fmaxf(-127.0f, __fmul_rn(y, inv_scale)));
+    const float b = __fadd_rn(r, kRoundBias);
+    const float d = __fsub_rn(r, __fsub_rn(b, kRoundBias));
+    if (fabsf(d) < kTieGuard) return b;
+  }
+  return __fadd_rn(fminf(127.0f, fmaxf(-127.0f, __fdiv_rn(y, scale))), kRoundBias);
+}
+
+// Sixteen int8 codes of one row chunk (see quant_code_biased) as one 16-byte
+// vector, element i in byte i; an all-zero row (amax == 0) gives zero codes.
+__device__ __forceinline__ uint4 pack_codes16(const float (&y)[16], float amax, float scale,
+                                              float inv_scale) {
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  if (amax != 0.0f) {
+    const bool fast = scale >= kMinNormal;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t u[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        u[b] = __float_as_uint(quant_code_biased(y[4 * k + b], scale, inv_scale, fast));
+      w[k] = __byte_perm(__byte_perm(u[0], u[1], 0x0040), __byte_perm(u[2], u[3], 0x0040), 0x5410);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The fp32 value q * scale of the round trip of y (0 for an all-zero row).
+__device__ __forceinline__ float quant_roundtrip(float y, float amax, float scale,
+                                                 float inv_scale) {
+  if (amax == 0.0f) return 0.0f;
+  const float b = quant_code_biased(y, scale, inv_scale, scale >= kMinNormal);
+  return __fmul_rn(__fsub_rn(b, kRoundBias), scale);
 }
 
 // Whether pair (t, k) is active under x_active_mask (1-D per token, 2-D per pair).

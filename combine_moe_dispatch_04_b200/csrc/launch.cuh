@@ -36,6 +36,11 @@ struct PermuteArgs {
   int bs, K, H, A, dtype, quant_mode;
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
+// int8 permute of x[t] * smooth[e] per slot (H <= 16384, multiple of 16; smooth 16-byte
+// aligned); reads the total R from send[E].
+cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
+                                  const float* smooth, const int32_t* send, int E,
+                                  cudaStream_t st);
 
 // Layout and the plain (no quantisation) permute in one launch, BS <= kLayoutSmallMaxTokens.
 cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,

@@ -7,7 +7,8 @@
 //
 // int8: one CTA per token (grid-stride); each thread keeps 16-element chunks
 // of the row in registers, the CTA reduces max|x|, and every chunk becomes one
-// 16-byte int8 store per slot.
+// 16-byte int8 store per slot. With smooth scales (E, H) every slot has its
+// own row x[t] * smooth[e] and is quantised on its own, one warp per slot.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -87,29 +88,129 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
     for (int j = 0; j < CPT; ++j) {
       const int c = threadIdx.x + j * blockDim.x;
       const bool mine = c < C;  // every lane still takes part in the shuffles below
-      uint32_t packed[4];
-#pragma unroll
-      for (int w4 = 0; w4 < 4; ++w4) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          int q = 0;
-          if (mine && amax != 0.0f) {
-            float r = quant_code(f[j][w4 * 4 + b], scale, inv_scale);
-            r = fminf(127.0f, fmaxf(-127.0f, r));
-            q = __float2int_rn(r);
-          }
-          word |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * b);
-        }
-        packed[w4] = word;
-      }
-      const uint4 val = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      const uint4 val = mine ? pack_codes16(f[j], amax, scale, inv_scale) : make_uint4(0, 0, 0, 0);
       for (int k = 0; k < K; ++k) {
         const int s = __shfl_sync(0xFFFFFFFFu, my_slot, k);
         if (mine && s >= 0) st_v4(out + static_cast<size_t>(s) * C + c, val);
       }
     }
     if (warp == 0 && lane < K && my_slot >= 0) scales[my_slot] = scale;
+  }
+}
+
+// Smooth-scaled int8 (reading R18): the row of slot s is y = x[t] * smooth[e]
+// for its pair (t, k) and expert e, quantised on its own. One warp per slot,
+// slots taken in order (a contiguous run per warp), so the warps of an SM keep
+// re-reading one expert's smooth row from L1 and write their int8 rows back to
+// back; each token row is gathered K times, from L2 after its first touch.
+// Lane i loads the pair and expert of slot i of each batch of 32 and the warp
+// walks the batch by shuffle, so only the first slot of a batch waits on the
+// index loads. max|y| is a warp reduction: no barriers. With CPL > 0 a lane
+// keeps its CPL chunks of y in registers (C <= 32 * CPL); with CPL == 0 it
+// streams the row twice, the second pass served mostly by L1.
+template <typename T16>
+__device__ __forceinline__ void smooth_chunk(const uint4* xr, const float4* sr, int c,
+                                             float (&y)[16]) {
+  float v[16];
+  widen8<T16>(__ldg(xr + 2 * c), reinterpret_cast<float(&)[8]>(v[0]));
+  widen8<T16>(__ldg(xr + 2 * c + 1), reinterpret_cast<float(&)[8]>(v[8]));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 m = __ldg(sr + 4 * c + q);
+    y[4 * q + 0] = __fmul_rn(v[4 * q + 0], m.x);
+    y[4 * q + 1] = __fmul_rn(v[4 * q + 1], m.y);
+    y[4 * q + 2] = __fmul_rn(v[4 * q + 2], m.z);
+    y[4 * q + 3] = __fmul_rn(v[4 * q + 3], m.w);
+  }
+}
+
+constexpr int kSmoothThreads = 256;
+constexpr int kSmoothStream = 4;  // chunks per lane in flight when streaming
+
+template <typename T16, int CPL>
+__global__ void __launch_bounds__(kSmoothThreads) permute_quant_smooth_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
+    const float4* __restrict__ smooth, const int32_t* __restrict__ assist,
+    const int32_t* __restrict__ send, uint4* __restrict__ out, float* __restrict__ scales, int K,
+    int H, int A, int E) {
+  pdl_trigger();
+  pdl_wait();
+  const int C = H / 16;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * (kSmoothThreads / 32);
+  const int gw = blockIdx.x * (kSmoothThreads / 32) + (threadIdx.x >> 5);
+  const int R = min(max(__ldg(send + E), 0), A);
+  const int per = (R + nwarps - 1) / nwarps;
+  const int lo = gw * per;
+  const int hi = min(R, lo + per);
+  for (int b = lo; b < hi; b += 32) {
+    int my_pair = -1, my_e = -1;
+    if (b + lane < hi) {
+      my_pair = __ldg(assist + b + lane);
+      if (my_pair >= 0) my_e = __ldg(topk_idx + my_pair);
+    }
+    const int n = min(32, hi - b);
+    for (int j = 0; j < n; ++j) {
+      const int pair = __shfl_sync(0xFFFFFFFFu, my_pair, j);
+      const int e = __shfl_sync(0xFFFFFFFFu, my_e, j);
+      if (pair < 0 || static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
+      const int s = b + j;
+      const uint4* xr = x + static_cast<size_t>(pair / K) * (H / 8);
+      const float4* sr = smooth + static_cast<size_t>(e) * (H / 4);
+      uint4* orow = out + static_cast<size_t>(s) * C;
+      float amax = 0.0f;
+      if constexpr (CPL > 0) {
+        float y[CPL][16];
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+          const int c = lane + 32 * u;
+          if (c < C) {
+            smooth_chunk<T16>(xr, sr, c, y[u]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[u][i]));
+          }
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+        const float scale = __fdiv_rn(amax, 127.0f);
+        const float inv_scale = 1.0f / scale;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+          const int c = lane + 32 * u;
+          if (c < C) st_v4(orow + c, pack_codes16(y[u], amax, scale, inv_scale));
+        }
+        if (lane == 0) scales[s] = scale;
+      } else {
+        for (int c0 = lane; c0 < C; c0 += 32 * kSmoothStream) {
+#pragma unroll
+          for (int u = 0; u < kSmoothStream; ++u) {
+            const int c = c0 + 32 * u;
+            if (c < C) {
+              float y[16];
+              smooth_chunk<T16>(xr, sr, c, y);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
+            }
+          }
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+        const float scale = __fdiv_rn(amax, 127.0f);
+        const float inv_scale = 1.0f / scale;
+        for (int c0 = lane; c0 < C; c0 += 32 * kSmoothStream) {
+#pragma unroll
+          for (int u = 0; u < kSmoothStream; ++u) {
+            const int c = c0 + 32 * u;
+            if (c < C) {
+              float y[16];
+              smooth_chunk<T16>(xr, sr, c, y);
+              st_v4(orow + c, pack_codes16(y, amax, scale, inv_scale));
+            }
+          }
+        }
+        if (lane == 0) scales[s] = scale;
+      }
+    }
   }
 }
 
@@ -124,6 +225,32 @@ void quant_shape(int H, int* threads, int* cpt) {
 }
 
 }  // namespace
+
+cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
+                                  const float* smooth, const int32_t* send, int E,
+                                  cudaStream_t st) {
+  if (a.bs == 0 || a.A == 0) return cudaSuccess;
+  const int C = a.H / 16;
+  const bool bf = a.dtype == MOE_BF16;
+  auto kern = bf ? permute_quant_smooth_kernel<Bf16, 0> : permute_quant_smooth_kernel<Fp16, 0>;
+  if (C <= 32)
+    kern = bf ? permute_quant_smooth_kernel<Bf16, 1> : permute_quant_smooth_kernel<Fp16, 1>;
+  else if (C <= 64)
+    kern = bf ? permute_quant_smooth_kernel<Bf16, 2> : permute_quant_smooth_kernel<Fp16, 2>;
+  else if (C <= 128)
+    kern = bf ? permute_quant_smooth_kernel<Bf16, 4> : permute_quant_smooth_kernel<Fp16, 4>;
+  int per_sm = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSmoothThreads, 0);
+  if (err != cudaSuccess) return err;
+  const long long want = (static_cast<long long>(a.A) + kSmoothThreads / 32 - 1) /
+                         (kSmoothThreads / 32);
+  const long long cap = static_cast<long long>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(kern, dim3(blocks), dim3(kSmoothThreads), 0, st,
+                    static_cast<const uint4*>(a.x), topk_idx,
+                    reinterpret_cast<const float4*>(smooth), a.assist, send,
+                    static_cast<uint4*>(a.expand_x), a.scales, a.K, a.H, a.A, E);
+}
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;

@@ -8,9 +8,9 @@
 //   S[j]             = sum_{pairs of const j} c,   grad_alpha1[j] = sum c ori_x[t]
 //   grad_alpha2[j]   = fl(S[j] v[j]),   grad_v[j] = fl(S[j] alpha2[j])
 //
-// Four launches: warp-per-pair dots (fixed butterfly), thread-per-vector
-// grad_ori_x, per-(token chunk, const expert) partial sums into the workspace,
-// and one fixed-order sum over the chunks. Every result is deterministic.
+// Three launches: warp-per-token grad_w dots (fixed butterfly) and grad_ori_x,
+// per-(token chunk, const expert) partial sums into the workspace, and one
+// fixed-order sum over the chunks. Every result is deterministic.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -18,7 +18,7 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunkTokens = 256;  // tokens per partial sum of the alpha / v gradients
+constexpr int kChunkTokens = 64;  // tokens per partial sum of the alpha / v gradients
 
 struct SpecialBwdArgs {
   const void* grad_out;
@@ -39,125 +39,178 @@ struct SpecialBwdArgs {
   int bs, K, H, E, Z, C, Q;
 };
 
-// Kind of pair (t, k): 0 none (routed, zero, masked, invalid), 1 copy, 2 const
-// (row q of the const tensors in *q).
-__device__ __forceinline__ int special_kind(const SpecialBwdArgs& a, int t, int k, int* q) {
-  const int32_t* ids = a.topk_idx + static_cast<size_t>(t) * a.K;
-  const int id = __ldg(ids + k);
-  const int lo = a.E + a.Z;
-  if (id < lo || id >= lo + a.C + a.Q) return 0;
-  for (int j = 0; j < k; ++j)
-    if (__ldg(ids + j) == id) return 0;
-  if (!pair_active(a.mask, a.mask_ndim, t, k, a.K)) return 0;
-  if (id < lo + a.C) return 1;
-  *q = id - lo - a.C;
-  return 2;
-}
-
-template <typename T16>
-__device__ __forceinline__ void const_m(const SpecialBwdArgs& a, int q, int V, int v,
-                                        const float (&x)[8], float (&m)[8]) {
-  const size_t r = static_cast<size_t>(q) * V + v;
-  float a1[8], a2[8], cv[8];
-  widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + r), a1);
-  widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + r), a2);
-  widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + r), cv);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(__fmul_rn(a1[i], x[i]), __fmul_rn(a2[i], cv[i]));
-}
-
-// grad_w of copy/const pairs: one warp per (token, k), persistent grid.
-template <typename T16>
-__global__ void __launch_bounds__(kThreads) special_dot_kernel(SpecialBwdArgs a) {
+// grad_w of the copy/const pairs and grad_ori_x: one warp per token on a
+// persistent grid. Lanes 0..K-1 classify the token's pairs (a repeat of an id
+// held by an earlier lane takes no part); the warp walks the ballot of those
+// pairs, taking each pair's kind, weight and const row by shuffle. A token
+// without such pairs only writes its zero grad_ori_x row. Otherwise the warp
+// writes grad_ori_x (pairs in ascending k), then makes one pass over the row
+// per pair for its dot (grad_out[t] and ori_x[t] from L1 after the first
+// touch), reduced with a fixed butterfly.
+template <typename T16, int KMAX>
+__global__ void __launch_bounds__(kThreads) special_token_kernel(SpecialBwdArgs a) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int V = a.H / kVecElems;
-  const int n_pairs = a.bs * a.K;
-  for (int pair = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); pair < n_pairs;
-       pair += gridDim.x * (kThreads / 32)) {
-    const int t = pair / a.K, k = pair - t * a.K;
-    int q = 0;
-    const int kind = special_kind(a, t, k, &q);  // warp-uniform
-    if (kind == 0) continue;
+  const int K = a.K;
+  const int lo = a.E + a.Z;
+  const int nw = gridDim.x * (kThreads / 32);
+  for (int t = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < a.bs; t += nw) {
+    const int id = lane < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + lane) : -1;
+    bool dup = false;
+#pragma unroll
+    for (int jj = 0; jj < KMAX; ++jj) {
+      const int other = __shfl_sync(0xFFFFFFFFu, id, jj);
+      dup |= jj < lane && other == id;
+    }
+    int my_kind = 0, my_q = 0;
+    float my_w = 0.0f;
+    if (lane < K && !dup && id >= lo && id < lo + a.C + a.Q &&
+        pair_active(a.mask, a.mask_ndim, t, lane, K)) {
+      my_kind = id < lo + a.C ? 1 : 2;
+      my_q = id - lo - a.C;
+      my_w = __ldg(a.weights + static_cast<size_t>(t) * K + lane);
+    }
+    uint4* go = static_cast<uint4*>(a.grad_ori_x) + static_cast<size_t>(t) * V;
+    const unsigned spec = __ballot_sync(0xFFFFFFFFu, my_kind != 0);
     const uint4* g = static_cast<const uint4*>(a.grad_out) + static_cast<size_t>(t) * V;
     const uint4* x = static_cast<const uint4*>(a.ori_x) + static_cast<size_t>(t) * V;
-    float d[8];
+    // grad_ori_x, pairs in ascending k (a token without such pairs gets zeros)
+    // (every lane runs every iteration: the shuffles below need the whole warp)
+    for (int v0 = 0; v0 < V; v0 += 32) {
+      const int v = v0 + lane;
+      const bool in = v < V;
+      float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) d[i] = 0.0f;
-    for (int v = lane; v < V; v += 32) {
-      float gf[8], xf[8], m[8];
-      widen8<T16>(__ldg(g + v), gf);
-      widen8<T16>(__ldg(x + v), xf);
-      if (kind == 1) {
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      if (spec != 0) {
+        float gf[8];
+        widen8<T16>(in ? __ldg(g + v) : make_uint4(0, 0, 0, 0), gf);  // kept in L1 for the dots
+        for (unsigned m = spec; m != 0; m &= m - 1) {
+          const int j = __ffs(m) - 1;
+          const int kind = __shfl_sync(0xFFFFFFFFu, my_kind, j);
+          const float w = __shfl_sync(0xFFFFFFFFu, my_w, j);
+          const int q = __shfl_sync(0xFFFFFFFFu, my_q, j);
+          if (kind == 1) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m[i] = xf[i];
-      } else {
-        const_m<T16>(a, q, V, v, xf, m);
+            for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, gf[i]));
+          } else {
+            float a1[8];
+            widen8<T16>(in ? __ldg(static_cast<const uint4*>(a.alpha1) +
+                                   static_cast<size_t>(q) * V + v)
+                           : make_uint4(0, 0, 0, 0),
+                        a1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[i] = __fadd_rn(acc[i], __fmul_rn(__fmul_rn(w, gf[i]), a1[i]));
+          }
+        }
+      }
+      if (in) st_v4(go + v, narrow8<T16>(acc));
+    }
+    // grad_w: one pass over the row per copy/const pair, then a fixed butterfly
+    for (unsigned m = spec; m != 0; m &= m - 1) {
+      const int j = __ffs(m) - 1;
+      const int kind = __shfl_sync(0xFFFFFFFFu, my_kind, j);
+      const int q = __shfl_sync(0xFFFFFFFFu, my_q, j);
+      float d = 0.0f;
+      for (int v = lane; v < V; v += 32) {
+        float gf[8], xf[8];
+        widen8<T16>(__ldg(g + v), gf);
+        widen8<T16>(__ldg(x + v), xf);
+        if (kind == 1) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) d = __fmaf_rn(gf[i], xf[i], d);
+        } else {
+          const size_t r = static_cast<size_t>(q) * V + v;
+          float a1[8], a2[8], cv[8];
+          widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + r), a1);
+          widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + r), a2);
+          widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + r), cv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d = __fmaf_rn(gf[i], __fadd_rn(__fmul_rn(a1[i], xf[i]), __fmul_rn(a2[i], cv[i])), d);
+        }
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) d[i] = __fmaf_rn(gf[i], m[i], d[i]);
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xFFFFFFFFu, d, off);
+      if (lane == 0) a.grad_w[static_cast<size_t>(t) * K + j] = d;
     }
-    float dot = ((d[0] + d[1]) + (d[2] + d[3])) + ((d[4] + d[5]) + (d[6] + d[7]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, off);
-    if (lane == 0) a.grad_w[pair] = dot;
   }
 }
 
-// grad_ori_x: one thread per 16-byte vector of (BS, H).
-template <typename T16>
-__global__ void __launch_bounds__(kThreads) special_ori_kernel(SpecialBwdArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  const int V = a.H / kVecElems;
-  const int item = blockIdx.x * kThreads + threadIdx.x;
-  if (item >= a.bs * V) return;
-  const int t = item / V, v = item - t * V;
-  float gf[8], acc[8];
-  widen8<T16>(__ldg(static_cast<const uint4*>(a.grad_out) + item), gf);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-  for (int k = 0; k < a.K; ++k) {
-    int q = 0;
-    const int kind = special_kind(a, t, k, &q);
-    if (kind == 0) continue;
-    const float w = __ldg(a.weights + static_cast<size_t>(t) * a.K + k);
-    float a1[8];
-    if (kind == 2)
-      widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + static_cast<size_t>(q) * V + v), a1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float c = __fmul_rn(w, gf[i]);
-      acc[i] = __fadd_rn(acc[i], kind == 1 ? c : __fmul_rn(c, a1[i]));
-    }
-  }
-  st_v4(static_cast<uint4*>(a.grad_ori_x) + item, narrow8<T16>(acc));
-}
-
-// Partial sums over one chunk of tokens for one const expert q: thread per
-// 16-byte vector of the row, tokens in ascending order.
+// Partial sums over one chunk of tokens for one const expert q. The first
+// threads find, per token of the chunk, the pair of q (its first occurrence
+// in the row, if active) and the CTA compacts those tokens in ascending order
+// into shared memory; then every thread (one 16-byte vector of the row) walks
+// the list, a few tokens' loads in flight at a time.
 template <typename T16>
 __global__ void __launch_bounds__(kThreads) special_partial_kernel(SpecialBwdArgs a) {
+  __shared__ int s_tok[kChunkTokens];
+  __shared__ float s_w[kChunkTokens];
+  __shared__ int s_cnt[kChunkTokens / 32];
   pdl_trigger();
   pdl_wait();
   const int V = a.H / kVecElems;
   const int chunk = blockIdx.x, q = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = chunk * kChunkTokens;
+  const int target = a.E + a.Z + a.C + q;
+  bool hit = false;
+  float wt = 0.0f;
+  const int t = t0 + threadIdx.x;
+  if (threadIdx.x < kChunkTokens && t < a.bs) {
+    const int32_t* ids = a.topk_idx + static_cast<size_t>(t) * a.K;
+    for (int k = 0; k < a.K; ++k) {
+      if (__ldg(ids + k) != target) continue;
+      if (pair_active(a.mask, a.mask_ndim, t, k, a.K)) {
+        hit = true;
+        wt = __ldg(a.weights + static_cast<size_t>(t) * a.K + k);
+      }
+      break;  // later occurrences are repeats
+    }
+  }
+  const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
+  if (lane == 0 && warp < kChunkTokens / 32) s_cnt[warp] = __popc(bal);
+  __syncthreads();
+  int n = 0, base = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kChunkTokens / 32; ++w2) {
+    if (w2 < warp) base += s_cnt[w2];
+    n += s_cnt[w2];
+  }
+  if (hit) {
+    const int pos = base + __popc(bal & lanemask_lt());
+    s_tok[pos] = t;
+    s_w[pos] = wt;
+  }
+  __syncthreads();
   const int v = blockIdx.z * kThreads + threadIdx.x;
   if (v >= V) return;
   float s1[8], sc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) s1[i] = sc[i] = 0.0f;
-  const int t1 = min(a.bs, (chunk + 1) * kChunkTokens);
-  for (int t = chunk * kChunkTokens; t < t1; ++t) {
-    for (int k = 0; k < a.K; ++k) {
-      int qq = -1;
-      if (special_kind(a, t, k, &qq) != 2 || qq != q) continue;
-      const float w = __ldg(a.weights + static_cast<size_t>(t) * a.K + k);
+  const uint4* G = static_cast<const uint4*>(a.grad_out);
+  const uint4* X = static_cast<const uint4*>(a.ori_x);
+  constexpr int kU = 4;
+  for (int i0 = 0; i0 < n; i0 += kU) {
+    uint4 gv[kU], xv[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (i0 + u < n) {
+        const size_t r = static_cast<size_t>(s_tok[i0 + u]) * V + v;
+        gv[u] = ld_nc_v4(G + r);
+        xv[u] = ld_nc_v4(X + r);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (i0 + u >= n) break;
+      const float w = s_w[i0 + u];
       float gf[8], xf[8];
-      widen8<T16>(__ldg(static_cast<const uint4*>(a.grad_out) + static_cast<size_t>(t) * V + v),
-                  gf);
-      widen8<T16>(__ldg(static_cast<const uint4*>(a.ori_x) + static_cast<size_t>(t) * V + v), xf);
+      widen8<T16>(gv[u], gf);
+      widen8<T16>(xv[u], xf);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float c = __fmul_rn(w, gf[i]);
@@ -169,11 +222,12 @@ __global__ void __launch_bounds__(kThreads) special_partial_kernel(SpecialBwdArg
   const size_t qh = static_cast<size_t>(a.Q) * a.H;
   float* p1 = a.partials + static_cast<size_t>(chunk) * 2 * qh + static_cast<size_t>(q) * a.H;
   float* pc = p1 + qh;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    p1[v * 8 + i] = s1[i];
-    pc[v * 8 + i] = sc[i];
-  }
+  float4* p1v = reinterpret_cast<float4*>(p1 + static_cast<size_t>(v) * 8);
+  float4* pcv = reinterpret_cast<float4*>(pc + static_cast<size_t>(v) * 8);
+  p1v[0] = make_float4(s1[0], s1[1], s1[2], s1[3]);
+  p1v[1] = make_float4(s1[4], s1[5], s1[6], s1[7]);
+  pcv[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+  pcv[1] = make_float4(sc[4], sc[5], sc[6], sc[7]);
 }
 
 // Sum of the partials over the chunks, in chunk order: grad_alpha1, and the
@@ -190,24 +244,35 @@ __global__ void __launch_bounds__(kThreads) special_final_kernel(SpecialBwdArgs 
     s1 = __fadd_rn(s1, a.partials[static_cast<size_t>(c) * 2 * qh + i]);
     sc = __fadd_rn(sc, a.partials[static_cast<size_t>(c) * 2 * qh + qh + i]);
   }
-  const size_t vi = i / 8, e = i - vi * 8;  // 16-byte vector and lane of element i
-  float a2[8], cv[8];
-  widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + vi), a2);
-  widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + vi), cv);
+  // element i of alpha_2 and v: the pair of 16-bit values holding it, widened
+  const size_t pi = i / 2;
+  const float2 a2 = T16::widen2(__ldg(static_cast<const uint32_t*>(a.alpha2) + pi));
+  const float2 cv = T16::widen2(__ldg(static_cast<const uint32_t*>(a.const_v) + pi));
+  const bool hi = i & 1;
   a.grad_alpha1[i] = s1;
-  a.grad_alpha2[i] = __fmul_rn(sc, cv[e]);
-  a.grad_v[i] = __fmul_rn(sc, a2[e]);
+  a.grad_alpha2[i] = __fmul_rn(sc, hi ? cv.y : cv.x);
+  a.grad_v[i] = __fmul_rn(sc, hi ? a2.y : a2.x);
+}
+
+template <typename T16, int KMAX>
+cudaError_t launch_token(const SpecialBwdArgs& a, cudaStream_t st) {
+  constexpr auto kernel = special_token_kernel<T16, KMAX>;
+  int per_sm = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+  if (err != cudaSuccess) return err;
+  const long long want = (static_cast<long long>(a.bs) + kThreads / 32 - 1) / (kThreads / 32);
+  const long long cap = static_cast<long long>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  return launch_pdl(kernel, dim3(static_cast<int>(want < cap ? want : cap)), dim3(kThreads), 0,
+                    st, a);
 }
 
 template <typename T16>
 cudaError_t launch_t(const SpecialBwdArgs& a, cudaStream_t st) {
   const int V = a.H / kVecElems;
-  cudaError_t err = launch_pdl(special_dot_kernel<T16>, dim3(sm_count() * 4), dim3(kThreads), 0,
-                               st, a);
-  if (err != cudaSuccess) return err;
-  const long long n = static_cast<long long>(a.bs) * V;
-  err = launch_pdl(special_ori_kernel<T16>, dim3(static_cast<int>((n + kThreads - 1) / kThreads)),
-                   dim3(kThreads), 0, st, a);
+  cudaError_t err = a.K <= 2   ? launch_token<T16, 2>(a, st)
+                    : a.K <= 4 ? launch_token<T16, 4>(a, st)
+                    : a.K <= 8 ? launch_token<T16, 8>(a, st)
+                               : launch_token<T16, 16>(a, st);
   if (err != cudaSuccess || a.Q == 0) return err;
   const int chunks = (a.bs + kChunkTokens - 1) / kChunkTokens;
   err = launch_pdl(special_partial_kernel<T16>,

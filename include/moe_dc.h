@@ -131,6 +131,31 @@ moe_status moe_dispatch_permute(const moe_shape* shape, const void* x,
                                 void* stream);
 
 /*
+ * moe_dispatch_permute_smooth — int8 dispatch of smooth-scaled rows: the
+ * graph-mode dispatch of the [combine] Example passes quant_mode 2 with a
+ * scales tensor of shape (E, H), read here as one fp32 factor per expert and
+ * hidden channel applied before the per-row quantisation.
+ *   x                (BS, H) dtype, in
+ *   topk_idx         int32 (BS, K), in: the ids moe_dispatch_layout was given
+ *   assist_info      from moe_dispatch_layout, in
+ *   ep_send_counts   from moe_dispatch_layout, in: the total R = ep_send_counts[E]
+ *                    is read (clamped to [0, A])
+ *   smooth_scales    fp32 (E, H), in, 16-byte aligned
+ *   For slot s of pair (t, k) with expert e = topk_idx[t, k]:
+ *     y = fp32(x[t] * smooth_scales[e]) (one rounding per element),
+ *     scale = max_h |y| / 127 (IEEE division), expand_x[s] =
+ *     int8(clamp(rne(y / scale), -127, 127)), dynamic_scales[s] = scale;
+ *     an all-zero y gives scale 0 and zero codes.
+ *   expand_x         int8 (A, H), out; dynamic_scales fp32 (A,), out. Rows
+ *                    s >= R are not written. H must be a multiple of 16 and at
+ *                    most 16384 (MOE_ERR_ALIGN / MOE_ERR_UNSUPPORTED).
+ */
+moe_status moe_dispatch_permute_smooth(const moe_shape* shape, const void* x,
+                                       const int32_t* topk_idx, const int32_t* assist_info,
+                                       const int32_t* ep_send_counts, const float* smooth_scales,
+                                       void* expand_x, float* dynamic_scales, void* stream);
+
+/*
  * moe_dispatch — moe_dispatch_layout followed by moe_dispatch_permute, in one
  * call (the dispatch of the [combine] Example: low_latency_dispatch returns
  * the expanded rows, the counts and assist_info together). For BS <= 1024
@@ -219,7 +244,7 @@ moe_status moe_combine_bwd(const moe_shape* shape, const void* grad_out, const v
  *   grad_alpha_1[j] = sum over pairs of const j of c * ori_x[t]  (Q, H) fp32
  *   grad_alpha_2[j] = S_j * v[j],  grad_v[j] = S_j * alpha_2[j],
  *                     S_j = sum over pairs of const j of c        (Q, H) fp32
- * Sums over tokens run in a fixed order (chunks of 256 tokens, then the
+ * Sums over tokens run in a fixed order (chunks of 64 tokens, then the
  * chunks in order), so results are deterministic. ori_x is required; the
  * const tensors and their gradients when Q > 0. workspace: device scratch of
  * moe_combine_bwd_special_workspace_bytes() bytes (0 when Q = 0).

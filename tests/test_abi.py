@@ -90,6 +90,16 @@ def test_other_entry_points_check_first():
     # misaligned row pointer
     assert moe.moe_dispatch_permute(s, ctypes.c_void_p(258), p, None, 0, p, None, None) == \
         moe.MOE_ERR_ALIGN
+    # smooth-scaled int8 dispatch: every pointer required, smooth scales 16-byte aligned,
+    # H a multiple of 16 and at most 16384
+    sm = moe.moe_dispatch_permute_smooth
+    assert sm(s, p, p, p, p, None, p, p, None) == moe.MOE_ERR_ARG
+    assert sm(s, p, None, p, p, p, p, p, None) == moe.MOE_ERR_ARG
+    assert sm(s, p, p, p, p, ctypes.c_void_p(260), p, p, None) == moe.MOE_ERR_ALIGN
+    h8 = moe.Shape(bs=16, k=2, h=1032, num_experts=4)
+    assert sm(ctypes.byref(h8.c()), p, p, p, p, p, p, p, None) == moe.MOE_ERR_ALIGN
+    big = moe.Shape(bs=16, k=2, h=16400, num_experts=4)
+    assert sm(ctypes.byref(big.c()), p, p, p, p, p, p, p, None) == moe.MOE_ERR_UNSUPPORTED
     # copy/const experts need ori_x; const experts need alpha_1, alpha_2, v
     sp = moe.Shape(bs=16, k=4, h=1024, num_experts=8, copy_expert_num=1, const_expert_num=1)
     args = [p, p, p, p, None, None, None, None, p, p, p, p, None]

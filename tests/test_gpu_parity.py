@@ -247,6 +247,44 @@ def test_int8_quant_rounding_ties(dtype):
     assert np.array_equal(gpu_chain.host(scd).view(np.uint32), sc.view(np.uint32))
 
 
+SMOOTH = [
+    W["special"],
+    W["special"].scaled(bs=1500, h=528, mask_ndim=2, mask_false_p=0.2, name="special_mask"),
+    W["dsv3"].scaled(bs=700, dtype="fp16", name="dsv3_fp16"),  # rows streamed twice
+    _custom("smooth_h16384", bs=40, k=3, num_experts=5, h=16384, quant_mode=2),
+    _custom("smooth_h16_one_expert", bs=333, k=1, num_experts=1, h=16, quant_mode=2),
+    _custom("smooth_empty", bs=0, quant_mode=2),
+]
+
+
+@pytest.mark.parametrize("wl", SMOOTH, ids=lambda w: w.name)
+def test_dispatch_smooth_quant(wl):
+    """int8 dispatch of x[t] * smooth[e]: codes and scales bit for bit against the
+    oracle; with several experts, expert 0's factors are zero, so its rows give
+    scale 0 and zero codes."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    inp = workloads.generate(wl)
+    sm = workloads.smooth_scales(wl)
+    if wl.num_experts > 1:
+        sm[0] = 0.0
+    _, send, assist, _ = oracle.dispatch_layout(inp["topk_idx"], wl.num_experts, wl.n_ids,
+                                                wl.a_capacity, mask=inp["mask"])
+    r = int(send[-1])
+    q, s = oracle.dispatch_permute_quant_smooth(inp["x"], inp["topk_idx"], sm, assist,
+                                                wl.a_capacity, wl.dtype)
+    sh = gpu_chain.shape_of(wl)
+    dev, host = gpu_chain.dev, gpu_chain.host
+    idx = dev(inp["topk_idx"])
+    lay = moe.dispatch_layout(sh, idx, x_active_mask=dev(inp["mask"]))
+    qd, sd = moe.dispatch_permute_smooth(sh, dev(inp["x"], wl.dtype), idx, lay, dev(sm))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(qd)[:r], q[:r])
+    assert np.array_equal(host(sd)[:r].view(np.uint32), s[:r].view(np.uint32))
+
+
 SPECIAL_BWD = [
     W["special"].scaled(backward=True, name="special_full_bwd"),
     W["special"].scaled(bs=1500, h=520, backward=True, mask_ndim=2, mask_false_p=0.2,

@@ -55,6 +55,7 @@ class Workload:
     mask_ndim: int = 0                # 0 none, 1 (BS,), 2 (BS, K)
     mask_false_p: float = 0.0
     quant_mode: int = 0               # 0 none, 2 dynamic int8 per row
+    smooth: bool = False              # int8 of x * smooth_scales[e] (needs quant_mode 2)
     backward: bool = True
     seed: int = 1
     a_capacity_override: int = 0
@@ -173,7 +174,17 @@ def generate(wl: Workload, seed: int | None = None) -> dict:
         out["expert_factor"] = (1.0 + eps).astype(np.float32)
     out["grad_out"] = (encode16(rng.standard_normal((wl.bs, wl.h)), wl.dtype)
                        if wl.backward else None)
+    out["smooth"] = smooth_scales(wl, seed) if wl.smooth else None
     return out
+
+
+def smooth_scales(wl: Workload, seed: int | None = None) -> np.ndarray:
+    """Per-expert, per-channel smooth-quant factors (E, H) fp32, standard normal
+    like the graph-mode dispatch example's scales; drawn from their own stream so
+    that generate() is unchanged."""
+    rng = np.random.Generator(np.random.PCG64((wl.seed if seed is None else seed) + 7919))
+    return np.ascontiguousarray(
+        rng.standard_normal((wl.num_experts, wl.h)).astype(np.float32))
 
 
 # ---------------------------------------------------------------------------
