@@ -186,7 +186,7 @@ def kernel_source_hash(kernel: str) -> str:
     """Hash of the source file that defines `kernel` and of the shared device helpers."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_moe_dispatch_04_b200", "csrc")
-    for name in (KERNEL_SOURCES[kernel], "common.cuh"):
+    for name in (KERNEL_SOURCES[kernel], "common.cuh", "async.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -416,6 +416,8 @@ def main():
         torch.cuda.synchronize()
 
     cq = args.combine_comm_quant
+    # the profiled kernel differs with the combine's quantisation mode
+    traffic_key = wl.name + ("+comm_quant2" if cq == 2 else "")
     if args.fused_dispatch:
         calls = [("dispatch", lambda st: moe.dispatch(
             sh, d["topk_idx"], d["x"], x_active_mask=d["mask"], comm_quant_mode=qm,
@@ -656,7 +658,7 @@ def main():
             "algorithmic_bytes_per_step": bytes_step,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
-                         "traffic": profiled_traffic(dom, wl.name),
+                         "traffic": profiled_traffic(dom, traffic_key),
                          "algorithmic_bytes": bytes_per[dom], "us_per_launch": round(dom_us, 3),
                          "timed": f"CUDA events around this kernel in every {DOM_EVERY}th timed "
                                   f"step ({len(dom_ms)} launches)"},

@@ -27,7 +27,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_combine_fwd", "moe_combine_bwd", "moe_dispatch_bwd",
            "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes",
            "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
-           "moe_combine_bwd_special_workspace_bytes", "moe_dispatch_permute_smooth")
+           "moe_combine_bwd_special_workspace_bytes", "moe_dispatch_permute_smooth",
+           "moe_async_wait_timeouts")
 
 
 class MoeShape(ctypes.Structure):
@@ -60,6 +61,7 @@ def _load():
     L.moe_dispatch_layout.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_dispatch_permute.argtypes = [S, P, P, P, I, P, P, P]
     L.moe_dispatch_permute_smooth.argtypes = [S, P, P, P, P, P, P, P, P]
+    L.moe_async_wait_timeouts.argtypes, L.moe_async_wait_timeouts.restype = [], ctypes.c_uint32
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_combine_fwd_comm_quant.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P]
     L.moe_dispatch.argtypes = [S, P, P, P, I, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -74,7 +76,8 @@ def _load():
     L.moe_layout_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
               "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
-              "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special"):
+              "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
+              "moe_dispatch_permute_smooth"):
         getattr(L, n).restype = I
     return L
 
@@ -89,6 +92,7 @@ moe_layout_workspace_bytes = _lib.moe_layout_workspace_bytes
 moe_dispatch_layout = _lib.moe_dispatch_layout
 moe_dispatch_permute = _lib.moe_dispatch_permute
 moe_dispatch_permute_smooth = _lib.moe_dispatch_permute_smooth
+moe_async_wait_timeouts = _lib.moe_async_wait_timeouts
 moe_combine_fwd = _lib.moe_combine_fwd
 moe_combine_bwd = _lib.moe_combine_bwd
 moe_dispatch_bwd = _lib.moe_dispatch_bwd

@@ -69,6 +69,14 @@ const char* moe_status_string(int status) {
 
 int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
+uint32_t moe_async_wait_timeouts(void) {
+  unsigned* p = moe::wait_timeout_counter();
+  unsigned v = 0;
+  if (p == nullptr || cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return UINT32_MAX;
+  return v;
+}
+
 size_t moe_assist_info_elems(const moe_shape* s) {
   if (s == nullptr) return 0;
   return static_cast<size_t>(s->a_capacity) + static_cast<size_t>(s->bs) * s->k;

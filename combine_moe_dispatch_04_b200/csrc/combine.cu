@@ -14,10 +14,27 @@
 // share grad_out[t] through L1), writes grad_expand = round16(w * grad_out)
 // and reduces grad_w with eight per-element accumulators per lane and a fixed
 // butterfly, so the result does not depend on scheduling.
+#include "async.cuh"
 #include "common.cuh"
 #include "launch.cuh"
 
 namespace moe {
+
+// CTAs that gave up a bounded wait on an asynchronous copy (0 in normal use).
+__device__ unsigned g_wait_timeouts = 0;
+
+unsigned* wait_timeout_counter() {
+  static unsigned* ptr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<unsigned*>(p);
+  }
+  return ptr[dev];
+}
+
 namespace {
 
 constexpr int kFwdThreads = 256;
@@ -275,8 +292,7 @@ __global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
           widen8<T16>(__ldg(Y + static_cast<size_t>(pm.row) * V + v), y);
           const float scale = __fdiv_rn(mx, 127.0f);
           const float inv_scale = 1.0f / scale;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = quant_roundtrip(y[i], mx, scale, inv_scale);
+          quant_roundtrip8(y, mx, scale, inv_scale, m);
         } else {
           pair_values<T16, SPECIAL>(a, pm.kind, pm.row, V, v, make_uint4(0, 0, 0, 0), ori, m);
         }
@@ -295,34 +311,59 @@ __global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
   }
 }
 
-// The same round trip with the token's rows held in registers: one CTA per
-// token (grid-stride), thread v owning vector v of every row (V <= 512,
-// K <= 8). Every warp classifies the token's pairs itself (lanes 0..K-1) and
-// spreads them by shuffle; all routed rows are loaded at once, each row's
-// max|y| is reduced (shuffles, then one shared-memory step), and the same
-// registers are dequantised and accumulated in ascending k. Shared arrays are
-// double-buffered by token parity, so two barriers per token suffice.
-constexpr int kQ8rMaxVectors = 512;
+// The same round trip with the token's rows staged in shared memory: one CTA
+// per token on a persistent grid, NBUF row buffers. Warp 0 classifies the
+// pairs of the token NBUF - 1 places ahead (lanes 0..K-1, repeats found by
+// shuffle), records them in shared memory and starts one bulk copy per routed
+// row (cp.async.bulk, global -> shared, completing on the buffer's mbarrier),
+// so the rows of the next tokens are in flight while this one is computed and
+// no register holds them. Each row's max|y| is taken on packed 16-bit pairs and
+// reduced by shuffles (the K rows interleaved); after the token's one barrier
+// every warp finishes the K maxima from shared memory itself (lane j: row j,
+// its scale and reciprocal; the array is double-buffered by token parity).
+// Every thread then dequantises its vectors of the rows and accumulates in
+// ascending k. Every wait is bounded: a CTA that gives up counts itself in
+// *timeouts and returns.
+constexpr int kQ8sThreads = 256;
+constexpr int kQ8sWarps = kQ8sThreads / 32;
 
-template <typename T16, int KMAX, bool SPECIAL>
-__global__ void __launch_bounds__(kQ8rMaxVectors, 1) combine_fwd_q8r_kernel(CombineArgs a) {
-  __shared__ float red[2][kQ8rMaxVectors / 32][KMAX];
-  __shared__ float rmax[2][KMAX];
-  pdl_trigger();
-  pdl_wait();
+template <int KMAX, int NBUF>
+struct Q8sLayout {  // byte offsets into the dynamic shared memory
+  static constexpr size_t bars = 0;  // NBUF mbarriers
+  static constexpr size_t meta = 64;
+  static constexpr size_t red = meta + (NBUF * KMAX * sizeof(PairMeta) + 15) / 16 * 16;
+  static constexpr size_t rmax = red + 2 * kQ8sWarps * KMAX * sizeof(float);  // end
+  static constexpr size_t rows = (rmax + 127) / 128 * 128;
+  static size_t bytes(int V) { return rows + static_cast<size_t>(NBUF) * KMAX * V * 16; }
+};
+
+template <typename T16, int KMAX, bool SPECIAL, int NBUF>
+__global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(CombineArgs a,
+                                                                      unsigned* timeouts) {
+  using L = Q8sLayout<KMAX, NBUF>;
+  static_assert(NBUF >= 2 && NBUF * 8 <= 64, "buffers");
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
+  PairMeta* meta = reinterpret_cast<PairMeta*>(smem + L::meta);
+  float* red = reinterpret_cast<float*>(smem + L::red);
+  uint4* rows = reinterpret_cast<uint4*>(smem + L::rows);
   const int V = a.H / kVecElems;
   const int K = a.K;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  const int v = threadIdx.x;
-  const bool act = v < V;
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
-  int buf = 0;
-  for (int t = blockIdx.x; t < a.bs; t += gridDim.x) {
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < NBUF; ++b) mbar_init(bars + b, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+
+  // Warp 0: record token t's pairs in buffer b and start its row copies.
+  auto stage = [&](int t, int b) {
     PairMeta pm{kSkip, 0, 1.0f};
     if (lane < K) pm = classify_pair<SPECIAL, false, false>(a, t, lane);
     if (SPECIAL) {
-      // a repeat of an id held by an earlier lane takes no part
       const int id = lane < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + lane) : -1;
       bool dup = false;
 #pragma unroll
@@ -332,68 +373,131 @@ __global__ void __launch_bounds__(kQ8rMaxVectors, 1) combine_fwd_q8r_kernel(Comb
       }
       if (dup) pm.kind = kSkip;
     }
-    int kind[KMAX], row[KMAX];
-    float w[KMAX];
+    const unsigned routed = __ballot_sync(0xFFFFFFFFu, pm.kind == kRouted);
+    if (lane < KMAX) meta[b * KMAX + lane] = pm;
+    fence_proxy_async_smem();  // the buffer was last read by the CTA's loads
+    if (lane == 0) mbar_arrive_expect_tx(bars + b, __popc(routed) * static_cast<uint32_t>(V) * 16u);
+    __syncwarp();
+    if ((routed >> lane) & 1u)
+      bulk_g2s(rows + (static_cast<size_t>(b) * KMAX + lane) * V,
+               Y + static_cast<size_t>(pm.row) * V, static_cast<uint32_t>(V) * 16u, bars + b);
+  };
+
+  const int stride = gridDim.x;
+  if (warp == 0)
+    for (int p = 0; p < NBUF - 1; ++p)
+      if (blockIdx.x + p * stride < a.bs) stage(blockIdx.x + p * stride, p);
+
+  int it = 0;
+  for (int t = blockIdx.x; t < a.bs; t += stride, ++it) {
+    const int b = it % NBUF;
+    const int rb = it & 1;
+    const bool ok = mbar_wait_bounded(bars + b, (it / NBUF) & 1);
+    const PairMeta* pmeta = meta + b * KMAX;
+    const uint4* brows = rows + static_cast<size_t>(b) * KMAX * V;
+    // this warp's max |y| of every row, the K reductions interleaved
+    // (rows of pairs that are not routed hold stale data: their maxima are
+    // computed without a branch and never used)
+    float mx[KMAX];
+    {
+      uint32_t m2[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      kind[j] = __shfl_sync(0xFFFFFFFFu, pm.kind, j);
-      row[j] = __shfl_sync(0xFFFFFFFFu, pm.row, j);
-      w[j] = __shfl_sync(0xFFFFFFFFu, pm.w, j);
-      if (j >= K) kind[j] = kSkip;
+      for (int j = 0; j < KMAX; ++j) m2[j] = 0;
+      for (int v = threadIdx.x; v < V; v += kQ8sThreads)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) m2[j] = absmax_v4<T16>(m2[j], brows[static_cast<size_t>(j) * V + v]);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) mx[j] = absmax_final<T16>(m2[j]);
     }
-    uint4 val[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      val[j] = make_uint4(0, 0, 0, 0);
-      if (act && kind[j] == kRouted) val[j] = ld_nc_v4(Y + static_cast<size_t>(row[j]) * V + v);
-    }
+    for (int d = 16; d > 0; d >>= 1)
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (kind[j] != kRouted) continue;  // CTA-uniform
-      float f[8];
-      widen8<T16>(val[j], f);
-      float mx = 0.0f;
+      for (int j = 0; j < KMAX; ++j) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xFFFFFFFFu, mx[j], d));
+    if (lane == 0)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(f[i]));
-#pragma unroll
-      for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
-      if (lane == 0) red[buf][warp][j] = mx;
-    }
-    __syncthreads();
-    if (threadIdx.x < K) {
-      float mx = 0.0f;
-      for (int ww = 0; ww < nwarps; ++ww) mx = fmaxf(mx, red[buf][ww][threadIdx.x]);
-      rmax[buf][threadIdx.x] = mx;
-    }
-    __syncthreads();
-    if (act) {
-      const size_t item = static_cast<size_t>(t) * V + v;
-      float ori[8];
-      if (SPECIAL) {
-        bool need = false;
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) need |= kind[j] == kCopy || kind[j] == kConst;
-        if (need) widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
+      for (int j = 0; j < KMAX; ++j) red[(rb * kQ8sWarps + warp) * KMAX + j] = mx[j];
+    // Every thread has finished the previous token here, so its buffer can be
+    // refilled; a CTA whose wait gave up leaves together.
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) {
+        atomicAdd(timeouts, 1u);
+        for (int q = 0; q < NBUF - 1; ++q)  // copies already started: let them land
+          if (t + q * stride < a.bs) mbar_wait_bounded(bars + (it + q) % NBUF, ((it + q) / NBUF) & 1);
       }
+      return;
+    }
+    if (warp == 0 && t + (NBUF - 1) * stride < a.bs) stage(t + (NBUF - 1) * stride, (it + NBUF - 1) % NBUF);
+    // every warp: lane j < K finishes row j's max and takes its scale and reciprocal
+    float rm = 0.0f;
+    if (lane < KMAX)
+#pragma unroll
+      for (int w = 0; w < kQ8sWarps; ++w) rm = fmaxf(rm, red[(rb * kQ8sWarps + w) * KMAX + lane]);
+    const float rs = __fdiv_rn(rm, 127.0f);
+    const float ri = 1.0f / rs;
+    // the fast path's reciprocal: 0 for an all-zero row (its codes are then 0)
+    const float rf = rm == 0.0f ? 0.0f : ri;
+    const bool rfast = rm == 0.0f || rs >= kMinNormal;
+    float rmj[KMAX], rsj[KMAX], rij[KMAX], rfj[KMAX], wj[KMAX];
+    int kindj[KMAX];
+    uint32_t fastj = 0;
+    bool any_special = false;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      rmj[j] = __shfl_sync(0xFFFFFFFFu, rm, j);
+      rsj[j] = __shfl_sync(0xFFFFFFFFu, rs, j);
+      rij[j] = __shfl_sync(0xFFFFFFFFu, ri, j);
+      rfj[j] = __shfl_sync(0xFFFFFFFFu, rf, j);
+      const PairMeta pm = pmeta[j];
+      kindj[j] = j < K ? pm.kind : static_cast<int>(kSkip);
+      wj[j] = pm.w;
+      // zero experts too: their +0 terms can change the sign of a zero sum
+      any_special |= kindj[j] == kZero || kindj[j] == kCopy || kindj[j] == kConst;
+    }
+    fastj = __ballot_sync(0xFFFFFFFFu, rfast);  // bit j: row j may take the fast path
+    for (int v = threadIdx.x; v < V; v += kQ8sThreads) {
+      const size_t item = static_cast<size_t>(t) * V + v;
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      uint32_t redo = any_special ? 1u : 0u;
+      if (!redo) {
+        // Routed rows only: every row computed without a branch, its terms
+        // selected in (unselected ones add -0, which leaves any sum as it is).
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (kind[j] == kSkip) continue;
-        float m[8];
-        if (kind[j] == kRouted) {
-          const float mx = rmax[buf][j];
-          const float scale = __fdiv_rn(mx, 127.0f);
-          const float inv_scale = 1.0f / scale;
-          float y[8];
-          widen8<T16>(val[j], y);
+        for (int j = 0; j < KMAX; ++j) {
+          float y[8], n[8], b[8], prod[8];
+          widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
+          const float dmax = quant_fast8(y, rfj[j], n, b);
+          const bool use = kindj[j] == kRouted;
+          redo |= (use && !(dmax < kTieGuard && ((fastj >> j) & 1u))) ? 1u : 0u;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = quant_roundtrip(y[i], mx, scale, inv_scale);
-        } else {
-          pair_values<T16, SPECIAL>(a, kind[j], row[j], V, v, val[j], ori, m);
+          for (int i = 0; i < 8; ++i) {
+            const float p = __fmul_rn(wj[j], __fmul_rn(n[i], rsj[j]));
+            prod[i] = use ? p : -0.0f;
+          }
+          add8_rn(acc, prod);
         }
-        axpy8_rn(acc, w[j], m);
+      }
+      if (redo) {  // special pairs, or a routed vector near a rounding tie
+        float ori[8];
+        if (SPECIAL && any_special && a.ori_x != nullptr)
+          widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (kindj[j] == kSkip) continue;
+          float m[8];
+          if (kindj[j] == kRouted) {
+            float y[8];
+            widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
+            quant_roundtrip8(y, rmj[j], rsj[j], rij[j], m);
+          } else {
+            pair_values<T16, SPECIAL>(a, kindj[j], pmeta[j].row, V, v, make_uint4(0, 0, 0, 0),
+                                      ori, m);
+          }
+          axpy8_rn(acc, wj[j], m);
+        }
       }
       if (a.shared != nullptr) {
         float sh[8];
@@ -402,7 +506,6 @@ __global__ void __launch_bounds__(kQ8rMaxVectors, 1) combine_fwd_q8r_kernel(Comb
       }
       st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
     }
-    buf ^= 1;
   }
 }
 
@@ -516,24 +619,50 @@ cudaError_t launch_fwd_t(const CombineArgs& a, cudaStream_t st) {
   return launch_fwd_k<T16, false, false>(a, st);
 }
 
-template <typename T16, bool SPECIAL, int KMAX>
-cudaError_t launch_fwd_q8r(const CombineArgs& a, cudaStream_t st) {
+// Shared memory a CTA of the staged kernel may use: two CTAs per SM.
+constexpr size_t kQ8sSmemBudget = 110 * 1024;
+
+template <typename T16, bool SPECIAL, int KMAX, int NBUF>
+cudaError_t launch_fwd_q8s(const CombineArgs& a, cudaStream_t st) {
+  constexpr auto kernel = combine_fwd_q8s_kernel<T16, KMAX, SPECIAL, NBUF>;
   const int V = a.H / kVecElems;
-  const int threads = (V + 31) / 32 * 32;
-  constexpr auto kernel = combine_fwd_q8r_kernel<T16, KMAX, SPECIAL>;
-  const int cap = sm_count() * blocks_per_sm<kernel>(threads, 0);
+  const size_t smem = Q8sLayout<KMAX, NBUF>::bytes(V);
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  unsigned* timeouts = wait_timeout_counter();
+  if (timeouts == nullptr) return cudaErrorInvalidSymbol;
+  int per_sm = 0;  // depends on the row size: not cached
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQ8sThreads, smem);
+  if (err != cudaSuccess) return err;
+  const int cap = sm_count() * (per_sm > 0 ? per_sm : 1);
   const int blocks = a.bs < cap ? a.bs : cap;
-  return launch_pdl(kernel, dim3(blocks), dim3(threads), 0, st, a);
+  return launch_pdl(kernel, dim3(blocks), dim3(kQ8sThreads), smem, st, a, timeouts);
+}
+
+// Staged kernel with three buffers when they fit the budget, else two; false
+// when even two do not fit (the caller then takes the two-pass kernel).
+template <typename T16, bool SPECIAL, int KMAX>
+bool try_launch_fwd_q8s(const CombineArgs& a, cudaStream_t st, cudaError_t* err) {
+  const int V = a.H / kVecElems;
+  if (Q8sLayout<KMAX, 3>::bytes(V) <= kQ8sSmemBudget) {
+    *err = launch_fwd_q8s<T16, SPECIAL, KMAX, 3>(a, st);
+    return true;
+  }
+  if (Q8sLayout<KMAX, 2>::bytes(V) <= kQ8sSmemBudget) {
+    *err = launch_fwd_q8s<T16, SPECIAL, KMAX, 2>(a, st);
+    return true;
+  }
+  return false;
 }
 
 template <typename T16, bool SPECIAL>
 cudaError_t launch_fwd_q8_t(const CombineArgs& a, cudaStream_t st) {
   const int V = a.H / kVecElems;
-  if (V <= kQ8rMaxVectors && a.K <= 8) {
-    if (a.K <= 2) return launch_fwd_q8r<T16, SPECIAL, 2>(a, st);
-    if (a.K <= 4) return launch_fwd_q8r<T16, SPECIAL, 4>(a, st);
-    return launch_fwd_q8r<T16, SPECIAL, 8>(a, st);
-  }
+  cudaError_t err = cudaSuccess;
+  if (a.K <= 2 && try_launch_fwd_q8s<T16, SPECIAL, 2>(a, st, &err)) return err;
+  if (a.K > 2 && a.K <= 4 && try_launch_fwd_q8s<T16, SPECIAL, 4>(a, st, &err)) return err;
+  if (a.K > 4 && a.K <= 8 && try_launch_fwd_q8s<T16, SPECIAL, 8>(a, st, &err)) return err;
   const int threads = V < 256 ? (V + 31) / 32 * 32 : 256;
   const int cap = sm_count() * (2048 / threads);
   const int blocks = a.bs < cap ? a.bs : cap;

@@ -25,6 +25,18 @@ struct Bf16 {
   }
 };
 
+// Running max of |value| over 16-bit pairs, kept packed (one instruction per
+// pair of values); max and abs are exact, so the widened result equals the
+// fp32 max of the widened values.
+struct Bf16Abs {
+  static __device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t v) {
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&acc);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&v);
+    __nv_bfloat162 r = __hmax2(a, __habs2(b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+};
+
 struct Fp16 {
   static __device__ __forceinline__ float2 widen2(uint32_t u) {
     __half2 h = *reinterpret_cast<__half2*>(&u);
@@ -53,15 +65,42 @@ __device__ __forceinline__ uint4 narrow8(const float (&f)[8]) {
   return v;
 }
 
+// Packed running max of |x| over a 16-byte vector (8 values), per dtype.
+template <typename T>
+__device__ __forceinline__ uint32_t absmax_v4(uint32_t acc, const uint4& v);
+template <>
+__device__ __forceinline__ uint32_t absmax_v4<Bf16>(uint32_t acc, const uint4& v) {
+  acc = Bf16Abs::absmax2(acc, v.x);
+  acc = Bf16Abs::absmax2(acc, v.y);
+  acc = Bf16Abs::absmax2(acc, v.z);
+  return Bf16Abs::absmax2(acc, v.w);
+}
+template <>
+__device__ __forceinline__ uint32_t absmax_v4<Fp16>(uint32_t acc, const uint4& v) {
+  __half2 a = *reinterpret_cast<__half2*>(&acc);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a = __hmax2(a, __habs2(*reinterpret_cast<const __half2*>(&w[i])));
+  return *reinterpret_cast<uint32_t*>(&a);
+}
+// The larger of the two packed maxima, widened.
+template <typename T>
+__device__ __forceinline__ float absmax_final(uint32_t acc) {
+  const float2 f = T::widen2(acc);
+  return fmaxf(f.x, f.y);
+}
+
 // ---- packed fp32 pairs (sm_100: one instruction, each lane rounded as the
 // scalar op would be) ----
 
+// A register pair viewed as one 64-bit operand (no data movement).
 __device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
-  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+  unsigned long long v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
 }
 __device__ __forceinline__ void unpack2(unsigned long long v, float& lo, float& hi) {
-  lo = __uint_as_float(static_cast<uint32_t>(v));
-  hi = __uint_as_float(static_cast<uint32_t>(v >> 32));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 __device__ __forceinline__ unsigned long long mul2_rn(unsigned long long a, unsigned long long b) {
   unsigned long long d;
@@ -157,51 +196,107 @@ constexpr float kRoundBias = 12582912.0f;        // 1.5 * 2^23
 constexpr float kTieGuard = 0.49993896484375f;   // 0.5 - 2^-14
 constexpr float kMinNormal = 1.17549435e-38f;    // 2^-126
 
-// The int8 code clamp(rne(fl32(y / scale)), -127, 127), returned biased (as
-// code + 1.5 * 2^23, see above), for scale = fl32(max|row| / 127) > 0 and
-// |y| <= max|row|, so |y / scale| <= 127 (1 + 2^-23). With fast set (scale
-// normal, inv_scale = fl32(1 / scale)), r = y * inv_scale and the IEEE quotient
-// fl32(y / scale) both lie within 127 * 3 * 2^-24 < 2^-15 of the exact
-// quotient; when r, clamped to [-127, 127], is more than 2^-14 from every
-// half-integer, both round and clamp to the same integer (the bounds are
-// integers, so clamping before or after rounding agrees). Otherwise (rare:
-// near a rounding tie) the IEEE division decides.
-__device__ __forceinline__ float quant_code_biased(float y, float scale, float inv_scale,
-                                                   bool fast) {
-  if (fast) {
-    const float r = fminf(127.0f, fmaxf(-127.0f, __fmul_rn(y, inv_scale)));
-    const float b = __fadd_rn(r, kRoundBias);
-    const float d = __fsub_rn(r, __fsub_rn(b, kRoundBias));
-    if (fabsf(d) < kTieGuard) return b;
+// The int8 codes n[i] = rne(fl32(y[i] / scale)) of eight values, as fp32
+// integers n and biased (b = n + 1.5 * 2^23, see above), for
+// scale = fl32(max|row| / 127) > 0 and every |y[i]| <= max|row|. Then
+// |y / scale| <= 127 (1 + 2^-23) and |n| <= 127, so no clamp is needed. With
+// fast set (scale normal and inv_scale = fl32(1 / scale)), r = y * inv_scale
+// and the IEEE quotient fl32(y / scale) both lie within 127 * 3 * 2^-24 <
+// 2^-15 of the exact quotient; when every r is more than 2^-14 from every
+// half-integer, each r rounds to the same integer as its quotient. Otherwise
+// (rare: near a rounding tie) the IEEE divisions decide. Products are scalar
+// .rn multiplies (never contracted); the rest is packed and exact.
+// The fast path alone: n[i] = rint(fl32(y[i] * inv_scale)) (as fp32 integers)
+// and b[i] = n[i] + 1.5 * 2^23; returns max_i |r[i] - n[i]| (a tree of maxima).
+__device__ __forceinline__ float quant_fast8(const float (&y)[8], float inv_scale, float (&n)[8],
+                                             float (&b)[8]) {
+  const unsigned long long bias2 = pack2(kRoundBias, kRoundBias);
+  const unsigned long long nbias2 = pack2(-kRoundBias, -kRoundBias);
+  const unsigned long long neg2 = pack2(-1.0f, -1.0f);
+  float d[8];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const unsigned long long r2 = pack2(__fmul_rn(y[i], inv_scale), __fmul_rn(y[i + 1], inv_scale));
+    const unsigned long long b2 = add2_rn(r2, bias2);
+    const unsigned long long n2 = add2_rn(b2, nbias2);
+    unpack2(fma2_rn(n2, neg2, r2), d[i], d[i + 1]);  // r - n, exact
+    unpack2(b2, b[i], b[i + 1]);
+    unpack2(n2, n[i], n[i + 1]);
   }
-  return __fadd_rn(fminf(127.0f, fmaxf(-127.0f, __fdiv_rn(y, scale))), kRoundBias);
+  return fmaxf(fmaxf(fmaxf(fabsf(d[0]), fabsf(d[1])), fmaxf(fabsf(d[2]), fabsf(d[3]))),
+               fmaxf(fmaxf(fabsf(d[4]), fabsf(d[5])), fmaxf(fabsf(d[6]), fabsf(d[7]))));
 }
 
-// Sixteen int8 codes of one row chunk (see quant_code_biased) as one 16-byte
-// vector, element i in byte i; an all-zero row (amax == 0) gives zero codes.
+__device__ __forceinline__ void quant_codes8(const float (&y)[8], float scale, float inv_scale,
+                                             bool fast, float (&n)[8], float (&b)[8]) {
+  const float dmax = fast ? quant_fast8(y, inv_scale, n, b) : 1.0f;
+  if (!(dmax < kTieGuard)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      b[i] = __fadd_rn(__fdiv_rn(y[i], scale), kRoundBias);
+      n[i] = __fsub_rn(b[i], kRoundBias);
+    }
+  }
+}
+
+// max |y[i]| over eight values, as a tree.
+__device__ __forceinline__ float absmax8(const float (&y)[8]) {
+  return fmaxf(fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3]))),
+               fmaxf(fmaxf(fabsf(y[4]), fabsf(y[5])), fmaxf(fabsf(y[6]), fabsf(y[7]))));
+}
+
+// Sixteen int8 codes of one row chunk as one 16-byte vector, element i in
+// byte i; an all-zero row (amax == 0) gives zero codes.
 __device__ __forceinline__ uint4 pack_codes16(const float (&y)[16], float amax, float scale,
                                               float inv_scale) {
   uint32_t w[4] = {0u, 0u, 0u, 0u};
   if (amax != 0.0f) {
     const bool fast = scale >= kMinNormal;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t u[4];
+    for (int h = 0; h < 2; ++h) {
+      float n[8], b[8];
+      quant_codes8(reinterpret_cast<const float(&)[8]>(y[8 * h]), scale, inv_scale, fast, n, b);
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
-        u[b] = __float_as_uint(quant_code_biased(y[4 * k + b], scale, inv_scale, fast));
-      w[k] = __byte_perm(__byte_perm(u[0], u[1], 0x0040), __byte_perm(u[2], u[3], 0x0040), 0x5410);
+      for (int k = 0; k < 2; ++k) {
+        const uint32_t u0 = __float_as_uint(b[4 * k]), u1 = __float_as_uint(b[4 * k + 1]);
+        const uint32_t u2 = __float_as_uint(b[4 * k + 2]), u3 = __float_as_uint(b[4 * k + 3]);
+        w[2 * h + k] = __byte_perm(__byte_perm(u0, u1, 0x0040), __byte_perm(u2, u3, 0x0040), 0x5410);
+      }
     }
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// The fp32 value q * scale of the round trip of y (0 for an all-zero row).
-__device__ __forceinline__ float quant_roundtrip(float y, float amax, float scale,
-                                                 float inv_scale) {
-  if (amax == 0.0f) return 0.0f;
-  const float b = quant_code_biased(y, scale, inv_scale, scale >= kMinNormal);
-  return __fmul_rn(__fsub_rn(b, kRoundBias), scale);
+// Eight int8 codes (element i in byte i) of one 16-byte vector of a row.
+__device__ __forceinline__ uint2 pack_codes8(const float (&y)[8], float amax, float scale,
+                                             float inv_scale) {
+  if (amax == 0.0f) return make_uint2(0u, 0u);
+  float n[8], b[8];
+  quant_codes8(y, scale, inv_scale, scale >= kMinNormal, n, b);
+  uint32_t w[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t u0 = __float_as_uint(b[4 * k]), u1 = __float_as_uint(b[4 * k + 1]);
+    const uint32_t u2 = __float_as_uint(b[4 * k + 2]), u3 = __float_as_uint(b[4 * k + 3]);
+    w[k] = __byte_perm(__byte_perm(u0, u1, 0x0040), __byte_perm(u2, u3, 0x0040), 0x5410);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// m[i] = n[i] * scale, the fp32 values of the int8 round trip of eight values
+// of a row (0 for an all-zero row), scale = fl32(amax / 127).
+__device__ __forceinline__ void quant_roundtrip8(const float (&y)[8], float amax, float scale,
+                                                 float inv_scale, float (&m)[8]) {
+  if (amax == 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+    return;
+  }
+  float n[8], b[8];
+  quant_codes8(y, scale, inv_scale, scale >= kMinNormal, n, b);
+  const unsigned long long s2 = pack2(scale, scale);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) unpack2(mul2_rn(pack2(n[i], n[i + 1]), s2), m[i], m[i + 1]);
 }
 
 // Whether pair (t, k) is active under x_active_mask (1-D per token, 2-D per pair).

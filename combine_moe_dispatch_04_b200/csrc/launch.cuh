@@ -89,6 +89,10 @@ cudaError_t launch_special_bwd(const void* grad_out, const int32_t* topk_idx,
 
 int sm_count();
 
+// Device address of the counter of CTAs that gave up a bounded wait on an
+// asynchronous copy (this device's; null if it cannot be had).
+unsigned* wait_timeout_counter();
+
 // Records err as the thread's last CUDA error; returns MOE_ERR_CUDA (MOE_OK for success).
 moe_status report_cuda_error(cudaError_t err);
 

@@ -9,6 +9,7 @@
 // of the row in registers, the CTA reduces max|x|, and every chunk becomes one
 // 16-byte int8 store per slot. With smooth scales (E, H) every slot has its
 // own row x[t] * smooth[e] and is quantised on its own, one warp per slot.
+#include "async.cuh"
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -214,6 +215,125 @@ __global__ void __launch_bounds__(kSmoothThreads) permute_quant_smooth_kernel(
   }
 }
 
+// Smooth-scaled int8 with each warp's token rows staged in shared memory: a
+// CTA takes a contiguous run of slots and its warps take them in turn (so
+// they share the current expert's smooth row through L1). Lane 0 of a warp
+// looks up the pair and expert of the slot kSmoothStages - 1 places ahead and
+// starts one bulk copy of its token row into the warp's next buffer
+// (cp.async.bulk on the buffer's mbarrier), so the gather is in flight while
+// the current slot is quantised. Lane l handles 16-byte vectors l, l + 32, ...
+// of the row: one pass for max|x * s| (warp reduction), one for the codes
+// (8 bytes per vector). No CTA barrier; every wait is bounded and a warp that
+// gives up counts itself in *timeouts and returns.
+constexpr int kSmoothStages = 3;
+
+struct SmoothSlot {
+  int e;     // expert of the slot, -1: nothing to do
+  int slot;
+};
+
+__host__ __device__ constexpr size_t smooth_warp_bytes(int H) {
+  return (128 + static_cast<size_t>(kSmoothStages) * H * 2 + 127) / 128 * 128;
+}
+
+template <typename T16>
+__global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
+    const float4* __restrict__ smooth, const int32_t* __restrict__ assist,
+    const int32_t* __restrict__ send, uint2* __restrict__ out, float* __restrict__ scales, int K,
+    int H, int A, int E, unsigned* timeouts) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int V = H / kVecElems;
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+  unsigned char* wbase = smem + static_cast<size_t>(warp) * smooth_warp_bytes(H);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase);
+  SmoothSlot* info = reinterpret_cast<SmoothSlot*>(wbase + 64);
+  uint4* rows = reinterpret_cast<uint4*>(wbase + 128);
+  if (lane == 0) {
+    for (int b = 0; b < kSmoothStages; ++b) mbar_init(bars + b, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  pdl_trigger();
+  pdl_wait();
+  const int R = min(max(__ldg(send + E), 0), A);
+  const int per = (R + gridDim.x - 1) / gridDim.x;
+  const int lo = blockIdx.x * per;
+  const int hi = min(R, lo + per);
+
+  // Lane 0: slot s into buffer b.
+  auto stage = [&](int s, int b) {
+    const int pair = __ldg(assist + s);
+    int e = pair >= 0 ? __ldg(topk_idx + pair) : -1;
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
+    info[b] = SmoothSlot{e, s};
+    fence_proxy_async_smem();  // the buffer was last read by the warp's loads
+    mbar_arrive_expect_tx(bars + b, e >= 0 ? row_bytes : 0u);
+    if (e >= 0)
+      bulk_g2s(rows + static_cast<size_t>(b) * V, x + static_cast<size_t>(pair / K) * V, row_bytes,
+               bars + b);
+  };
+
+  if (lane == 0)
+    for (int p = 0; p < kSmoothStages - 1; ++p)
+      if (lo + warp + p * nwarps < hi) stage(lo + warp + p * nwarps, p);
+  int it = 0;
+  for (int s = lo + warp; s < hi; s += nwarps, ++it) {
+    const int b = it % kSmoothStages;
+    const bool ok = mbar_wait_bounded(bars + b, (it / kSmoothStages) & 1);
+    if (__any_sync(0xFFFFFFFFu, !ok)) {
+      if (lane == 0) {
+        atomicAdd(timeouts, 1u);
+        for (int q = 1; q < kSmoothStages; ++q)  // copies already started: let them land
+          if (s + q * nwarps < hi)
+            mbar_wait_bounded(bars + (it + q) % kSmoothStages, ((it + q) / kSmoothStages) & 1);
+      }
+      return;
+    }
+    // the buffer of the previous slot is free (its reads ended before the
+    // __syncwarp below): refill it with the slot kSmoothStages - 1 ahead
+    const int ahead = s + (kSmoothStages - 1) * nwarps;
+    if (lane == 0 && ahead < hi) stage(ahead, (it + kSmoothStages - 1) % kSmoothStages);
+    const SmoothSlot si = info[b];
+    if (si.e >= 0) {
+      const uint4* xr = rows + static_cast<size_t>(b) * V;
+      const float4* sr = smooth + static_cast<size_t>(si.e) * (H / 4);
+      float amax = 0.0f;
+#pragma unroll 4
+      for (int v = lane; v < V; v += 32) {
+        float y[8];
+        widen8<T16>(xr[v], y);
+        const float4 m0 = __ldg(sr + 2 * v), m1 = __ldg(sr + 2 * v + 1);
+        y[0] = __fmul_rn(y[0], m0.x); y[1] = __fmul_rn(y[1], m0.y);
+        y[2] = __fmul_rn(y[2], m0.z); y[3] = __fmul_rn(y[3], m0.w);
+        y[4] = __fmul_rn(y[4], m1.x); y[5] = __fmul_rn(y[5], m1.y);
+        y[6] = __fmul_rn(y[6], m1.z); y[7] = __fmul_rn(y[7], m1.w);
+        amax = fmaxf(amax, absmax8(y));
+      }
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+      const float scale = __fdiv_rn(amax, 127.0f);
+      const float inv_scale = 1.0f / scale;
+      uint2* orow = out + static_cast<size_t>(si.slot) * V;
+#pragma unroll 4
+      for (int v = lane; v < V; v += 32) {
+        float y[8];
+        widen8<T16>(xr[v], y);
+        const float4 m0 = __ldg(sr + 2 * v), m1 = __ldg(sr + 2 * v + 1);
+        y[0] = __fmul_rn(y[0], m0.x); y[1] = __fmul_rn(y[1], m0.y);
+        y[2] = __fmul_rn(y[2], m0.z); y[3] = __fmul_rn(y[3], m0.w);
+        y[4] = __fmul_rn(y[4], m1.x); y[5] = __fmul_rn(y[5], m1.y);
+        y[6] = __fmul_rn(y[6], m1.z); y[7] = __fmul_rn(y[7], m1.w);
+        orow[v] = pack_codes8(y, amax, scale, inv_scale);
+      }
+      if (lane == 0) scales[si.slot] = scale;
+    }
+    __syncwarp();
+  }
+}
+
 // Threads and 16-element chunks per thread for the int8 kernels: one chunk
 // per thread up to 256 threads, then 2 or 4 (H <= 16384, checked by the caller).
 void quant_shape(int H, int* threads, int* cpt) {
@@ -239,6 +359,28 @@ cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
     kern = bf ? permute_quant_smooth_kernel<Bf16, 2> : permute_quant_smooth_kernel<Fp16, 2>;
   else if (C <= 128)
     kern = bf ? permute_quant_smooth_kernel<Bf16, 4> : permute_quant_smooth_kernel<Fp16, 4>;
+  // Staged kernel when at least four warps' buffers fit in 110 KB (two CTAs per SM).
+  const int staged_warps = static_cast<int>(110 * 1024 / smooth_warp_bytes(a.H));
+  if (staged_warps >= 4) {
+    const int warps = staged_warps < 8 ? staged_warps : 8;
+    const size_t smem = static_cast<size_t>(warps) * smooth_warp_bytes(a.H);
+    auto sk = bf ? permute_smooth_staged_kernel<Bf16> : permute_smooth_staged_kernel<Fp16>;
+    cudaError_t err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    unsigned* timeouts = wait_timeout_counter();
+    if (timeouts == nullptr) return cudaErrorInvalidSymbol;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sk, 32 * warps, smem);
+    if (err != cudaSuccess) return err;
+    const long long want = (static_cast<long long>(a.A) + warps - 1) / warps;
+    const long long cap = static_cast<long long>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+    const int blocks = static_cast<int>(want < cap ? want : cap);
+    return launch_pdl(sk, dim3(blocks), dim3(32 * warps), smem, st,
+                      static_cast<const uint4*>(a.x), topk_idx,
+                      reinterpret_cast<const float4*>(smooth), a.assist, send,
+                      static_cast<uint2*>(a.expand_x), a.scales, a.K, a.H, a.A, E, timeouts);
+  }
   int per_sm = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSmoothThreads, 0);
   if (err != cudaSuccess) return err;

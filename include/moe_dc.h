@@ -75,6 +75,14 @@ const char* moe_status_string(int status);
 /* The CUDA error (cudaError_t value) behind the last MOE_ERR_CUDA on this thread. */
 int moe_last_cuda_error(void);
 
+/*
+ * Number of thread blocks on the current device that gave up a bounded wait
+ * for an asynchronous copy since the library was loaded (0 in normal
+ * operation; such a block leaves its part of the output unwritten).
+ * Synchronises the device. Returns UINT32_MAX if the count cannot be read.
+ */
+uint32_t moe_async_wait_timeouts(void);
+
 /* Elements of the int32 assist_info buffer: A + BS * K. */
 size_t moe_assist_info_elems(const moe_shape* shape);
 

@@ -113,6 +113,8 @@ COMM_QUANT = [
     W["dsv3"].scaled(bs=300, h=7168, name="dsv3_shared_q8"),
     _custom("k16_q8", bs=700, k=16, num_experts=40, h=136, zero_expert_num=2,
             const_expert_num=2, backward=False),
+    _custom("zero_only_q8", bs=900, k=4, num_experts=16, zero_expert_num=3, h=256,
+            backward=False),
     W["special"],  # full size
 ]
 
@@ -153,6 +155,41 @@ def test_combine_comm_quant_mode2(wl):
     d = gpu_chain.ulp_dist(got, want)
     assert d.max() <= gpu_chain.ULP_TOL
     assert (d == 0).mean() == 1.0  # same fp32 operations in the same order
+    assert moe.moe_async_wait_timeouts() == 0  # no staged copy was given up on
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_combine_q8_rounding_ties(dtype):
+    """Returning rows whose values sit exactly on, or one 16-bit step beside,
+    half-integer multiples of their scale: the combine round trip must match the
+    oracle's IEEE division and rounding bit for bit."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    wl = _custom("q8_ties", bs=600, k=4, num_experts=8, h=256, backward=False, dtype=dtype)
+    inp = workloads.generate(wl)
+    _, send, assist, st = oracle.dispatch_layout(inp["topk_idx"], wl.num_experts, wl.n_ids,
+                                                 wl.a_capacity)
+    rng = np.random.default_rng(23)
+    a_rows = wl.a_capacity
+    c = 2.0 ** rng.integers(-6, 3, (a_rows, 1))
+    ties = (rng.integers(-127, 127, (a_rows, wl.h)) + 0.5) * c
+    ties[:, 0] = 127 * c[:, 0]  # the row max, so scale = c exactly
+    y = workloads.encode16(ties, dtype)
+    step = rng.integers(-1, 2, y.shape).astype(np.int32)
+    step[:, 0] = 0
+    y = (y.astype(np.int32) + step * (rng.random(y.shape) < 0.3)).astype(np.uint16)
+    want = oracle.combine_fwd(y, inp["topk_idx"], inp["topk_weights"], assist,
+                              num_experts=wl.num_experts, a_capacity=wl.a_capacity, dtype=dtype,
+                              comm_quant_mode=2)
+    sh = gpu_chain.shape_of(wl)
+    dev = gpu_chain.dev
+    lay = moe.dispatch_layout(sh, dev(inp["topk_idx"]))
+    out = moe.combine_fwd(sh, dev(y, dtype), dev(inp["topk_idx"]), dev(inp["topk_weights"]), lay,
+                          comm_quant_mode=2)
+    torch.cuda.synchronize()
+    assert np.array_equal(gpu_chain.host(out), want)
 
 
 FUSED = [
