@@ -312,38 +312,43 @@ __global__ void __launch_bounds__(1024) combine_fwd_q8_kernel(CombineArgs a) {
 }
 
 // The same round trip with the token's rows staged in shared memory: one CTA
-// per token on a persistent grid, NBUF row buffers. Warp 0 classifies the
-// pairs of the token NBUF - 1 places ahead (lanes 0..K-1, repeats found by
-// shuffle), records them in shared memory and starts one bulk copy per routed
-// row (cp.async.bulk, global -> shared, completing on the buffer's mbarrier),
-// so the rows of the next tokens are in flight while this one is computed and
-// no register holds them. Each row's max|y| is taken on packed 16-bit pairs and
-// reduced by shuffles (the K rows interleaved); after the token's one barrier
-// every warp finishes the K maxima from shared memory itself (lane j: row j,
-// its scale and reciprocal; the array is double-buffered by token parity).
-// Every thread then dequantises its vectors of the rows and accumulates in
-// ascending k. Every wait is bounded: a CTA that gives up counts itself in
-// *timeouts and returns.
-constexpr int kQ8sThreads = 256;
-constexpr int kQ8sWarps = kQ8sThreads / 32;
+// per token on a persistent grid, NBUF row buffers, warp-specialised. A
+// producer warp classifies each token's pairs (lanes 0..K-1, repeats found by
+// shuffle) ahead of time, waits until the consumers have released the
+// buffer, records the pairs in shared memory and starts one bulk copy per
+// routed row (cp.async.bulk, global -> shared, completing on the buffer's
+// "full" mbarrier). Eight consumer warps wait for "full", take each row's
+// max|y| on packed 16-bit pairs (the K reductions interleaved, then one
+// consumer-only named barrier; the array is double-buffered by token parity),
+// finish the K maxima from shared memory (lane j: row j, its scale and
+// reciprocal), dequantise and accumulate in ascending k, and release the
+// buffer on its "empty" mbarrier. The classification's global loads thus
+// never sit on the consumers' path. Every wait is bounded: a block that gives
+// up counts itself in *timeouts, lets its started copies land and returns.
+constexpr int kQ8sConsumerWarps = 8;
+constexpr int kQ8sConsumers = 32 * kQ8sConsumerWarps;
+constexpr int kQ8sThreads = kQ8sConsumers + 32;  // the last warp is the producer
+constexpr int kQ8sWarps = kQ8sConsumerWarps;
 
 template <int KMAX, int NBUF>
 struct Q8sLayout {  // byte offsets into the dynamic shared memory
-  static constexpr size_t bars = 0;  // NBUF mbarriers
+  static constexpr size_t full = 0;    // NBUF mbarriers
+  static constexpr size_t empty = 32;  // NBUF mbarriers
   static constexpr size_t meta = 64;
   static constexpr size_t red = meta + (NBUF * KMAX * sizeof(PairMeta) + 15) / 16 * 16;
-  static constexpr size_t rmax = red + 2 * kQ8sWarps * KMAX * sizeof(float);  // end
-  static constexpr size_t rows = (rmax + 127) / 128 * 128;
+  static constexpr size_t end = red + 2 * kQ8sWarps * KMAX * sizeof(float);
+  static constexpr size_t rows = (end + 127) / 128 * 128;
   static size_t bytes(int V) { return rows + static_cast<size_t>(NBUF) * KMAX * V * 16; }
 };
 
 template <typename T16, int KMAX, bool SPECIAL, int NBUF>
 __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(CombineArgs a,
-                                                                      unsigned* timeouts) {
+                                                                         unsigned* timeouts) {
   using L = Q8sLayout<KMAX, NBUF>;
-  static_assert(NBUF >= 2 && NBUF * 8 <= 64, "buffers");
+  static_assert(NBUF >= 2 && NBUF <= 4, "buffers");
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::full);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::empty);
   PairMeta* meta = reinterpret_cast<PairMeta*>(smem + L::meta);
   float* red = reinterpret_cast<float*>(smem + L::red);
   uint4* rows = reinterpret_cast<uint4*>(smem + L::rows);
@@ -352,47 +357,57 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
   if (threadIdx.x == 0) {
-    for (int b = 0; b < NBUF; ++b) mbar_init(bars + b, 1);
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(full + b, 1);
+      mbar_init(empty + b, kQ8sConsumerWarps);
+    }
     mbar_init_fence();
   }
   __syncthreads();
   pdl_trigger();
   pdl_wait();
-
-  // Warp 0: record token t's pairs in buffer b and start its row copies.
-  auto stage = [&](int t, int b) {
-    PairMeta pm{kSkip, 0, 1.0f};
-    if (lane < K) pm = classify_pair<SPECIAL, false, false>(a, t, lane);
-    if (SPECIAL) {
-      const int id = lane < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + lane) : -1;
-      bool dup = false;
-#pragma unroll
-      for (int jj = 0; jj < KMAX; ++jj) {
-        const int other = __shfl_sync(0xFFFFFFFFu, id, jj);
-        dup |= jj < lane && other == id;
-      }
-      if (dup) pm.kind = kSkip;
-    }
-    const unsigned routed = __ballot_sync(0xFFFFFFFFu, pm.kind == kRouted);
-    if (lane < KMAX) meta[b * KMAX + lane] = pm;
-    fence_proxy_async_smem();  // the buffer was last read by the CTA's loads
-    if (lane == 0) mbar_arrive_expect_tx(bars + b, __popc(routed) * static_cast<uint32_t>(V) * 16u);
-    __syncwarp();
-    if ((routed >> lane) & 1u)
-      bulk_g2s(rows + (static_cast<size_t>(b) * KMAX + lane) * V,
-               Y + static_cast<size_t>(pm.row) * V, static_cast<uint32_t>(V) * 16u, bars + b);
-  };
-
   const int stride = gridDim.x;
-  if (warp == 0)
-    for (int p = 0; p < NBUF - 1; ++p)
-      if (blockIdx.x + p * stride < a.bs) stage(blockIdx.x + p * stride, p);
+
+  if (warp == kQ8sConsumerWarps) {  // producer
+    int q = 0;
+    for (int t = blockIdx.x; t < a.bs; t += stride, ++q) {
+      const int b = q % NBUF;
+      PairMeta pm{kSkip, 0, 1.0f};
+      if (lane < K) pm = classify_pair<SPECIAL, false, false>(a, t, lane);
+      if (SPECIAL) {
+        const int id = lane < K ? __ldg(a.topk_idx + static_cast<size_t>(t) * K + lane) : -1;
+        bool dup = false;
+#pragma unroll
+        for (int jj = 0; jj < KMAX; ++jj) {
+          const int other = __shfl_sync(0xFFFFFFFFu, id, jj);
+          dup |= jj < lane && other == id;
+        }
+        if (dup) pm.kind = kSkip;
+      }
+      const unsigned routed = __ballot_sync(0xFFFFFFFFu, pm.kind == kRouted);
+      if (q >= NBUF) {  // wait until the consumers have released this buffer
+        const bool ok = mbar_wait_bounded(empty + b, ((q / NBUF) - 1) & 1);
+        if (__any_sync(0xFFFFFFFFu, !ok)) {
+          if (lane == 0) atomicAdd(timeouts, 1u);
+          return;
+        }
+      }
+      if (lane < KMAX) meta[b * KMAX + lane] = pm;
+      fence_proxy_async_smem();  // the buffer was last read by the consumers' loads
+      if (lane == 0) mbar_arrive_expect_tx(full + b, __popc(routed) * static_cast<uint32_t>(V) * 16u);
+      __syncwarp();
+      if ((routed >> lane) & 1u)
+        bulk_g2s(rows + (static_cast<size_t>(b) * KMAX + lane) * V,
+                 Y + static_cast<size_t>(pm.row) * V, static_cast<uint32_t>(V) * 16u, full + b);
+    }
+    return;
+  }
 
   int it = 0;
   for (int t = blockIdx.x; t < a.bs; t += stride, ++it) {
     const int b = it % NBUF;
     const int rb = it & 1;
-    const bool ok = mbar_wait_bounded(bars + b, (it / NBUF) & 1);
+    const bool ok = mbar_wait_bounded(full + b, (it / NBUF) & 1);
     const PairMeta* pmeta = meta + b * KMAX;
     const uint4* brows = rows + static_cast<size_t>(b) * KMAX * V;
     // this warp's max |y| of every row, the K reductions interleaved
@@ -403,7 +418,7 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
       uint32_t m2[KMAX];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) m2[j] = 0;
-      for (int v = threadIdx.x; v < V; v += kQ8sThreads)
+      for (int v = threadIdx.x; v < V; v += kQ8sConsumers)
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) m2[j] = absmax_v4<T16>(m2[j], brows[static_cast<size_t>(j) * V + v]);
 #pragma unroll
@@ -416,17 +431,15 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
     if (lane == 0)
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) red[(rb * kQ8sWarps + warp) * KMAX + j] = mx[j];
-    // Every thread has finished the previous token here, so its buffer can be
-    // refilled; a CTA whose wait gave up leaves together.
-    if (__syncthreads_or(!ok)) {
+    // consumers only; a block whose wait gave up leaves together
+    if (named_barrier_or(1, kQ8sConsumers, !ok)) {
       if (threadIdx.x == 0) {
         atomicAdd(timeouts, 1u);
-        for (int q = 0; q < NBUF - 1; ++q)  // copies already started: let them land
-          if (t + q * stride < a.bs) mbar_wait_bounded(bars + (it + q) % NBUF, ((it + q) / NBUF) & 1);
+        for (int q = 0; q < NBUF; ++q)  // copies already started: let them land
+          if (t + q * stride < a.bs) mbar_wait_bounded(full + (it + q) % NBUF, ((it + q) / NBUF) & 1);
       }
       return;
     }
-    if (warp == 0 && t + (NBUF - 1) * stride < a.bs) stage(t + (NBUF - 1) * stride, (it + NBUF - 1) % NBUF);
     // every warp: lane j < K finishes row j's max and takes its scale and reciprocal
     float rm = 0.0f;
     if (lane < KMAX)
@@ -436,25 +449,19 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
     const float ri = 1.0f / rs;
     // the fast path's reciprocal: 0 for an all-zero row (its codes are then 0)
     const float rf = rm == 0.0f ? 0.0f : ri;
-    const bool rfast = rm == 0.0f || rs >= kMinNormal;
-    float rmj[KMAX], rsj[KMAX], rij[KMAX], rfj[KMAX], wj[KMAX];
-    int kindj[KMAX];
-    uint32_t fastj = 0;
-    bool any_special = false;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      rmj[j] = __shfl_sync(0xFFFFFFFFu, rm, j);
-      rsj[j] = __shfl_sync(0xFFFFFFFFu, rs, j);
-      rij[j] = __shfl_sync(0xFFFFFFFFu, ri, j);
-      rfj[j] = __shfl_sync(0xFFFFFFFFu, rf, j);
-      const PairMeta pm = pmeta[j];
-      kindj[j] = j < K ? pm.kind : static_cast<int>(kSkip);
-      wj[j] = pm.w;
-      // zero experts too: their +0 terms can change the sign of a zero sum
-      any_special |= kindj[j] == kZero || kindj[j] == kCopy || kindj[j] == kConst;
-    }
-    fastj = __ballot_sync(0xFFFFFFFFu, rfast);  // bit j: row j may take the fast path
-    for (int v = threadIdx.x; v < V; v += kQ8sThreads) {
+    // lane j also holds pair j's weight and kind; the warp takes them by shuffle
+    const PairMeta lpm = pmeta[lane < KMAX ? lane : 0];
+    const int lkind = lane < K ? lpm.kind : static_cast<int>(kSkip);
+    const float lw = lpm.w;
+    const uint32_t routed = __ballot_sync(0xFFFFFFFFu, lkind == kRouted);
+    // zero experts too: their +0 terms can change the sign of a zero sum
+    const bool any_special = __any_sync(0xFFFFFFFFu, lkind == kZero || lkind == kCopy || lkind == kConst);
+    const uint32_t fastm = __ballot_sync(0xFFFFFFFFu, rm == 0.0f || rs >= kFastMinScale);
+    // Whole warps walk the vectors (the shuffles below need every lane); a lane
+    // past the row end works on vector 0 and stores nothing.
+    for (int v0 = warp * 32; v0 < V; v0 += kQ8sConsumers) {
+      const bool act = v0 + lane < V;
+      const int v = act ? v0 + lane : 0;
       const size_t item = static_cast<size_t>(t) * V + v;
       float acc[8];
 #pragma unroll
@@ -465,40 +472,54 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
         // selected in (unselected ones add -0, which leaves any sum as it is).
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
+          const float rfj = __shfl_sync(0xFFFFFFFFu, rf, j);
+          const float rsj = __shfl_sync(0xFFFFFFFFu, rs, j);
+          const float wj = __shfl_sync(0xFFFFFFFFu, lw, j);
           float y[8], n[8], b[8], prod[8];
           widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
-          const float dmax = quant_fast8(y, rfj[j], n, b);
-          const bool use = kindj[j] == kRouted;
-          redo |= (use && !(dmax < kTieGuard && ((fastj >> j) & 1u))) ? 1u : 0u;
+          quant_codes8<true>(y, rsj, rfj, true, n, b);  // exact, ties included
+          const bool use = (routed >> j) & 1u;
+          redo |= (use && !((fastm >> j) & 1u)) ? 1u : 0u;  // a tiny scale: IEEE divisions
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float p = __fmul_rn(wj[j], __fmul_rn(n[i], rsj[j]));
+            const float p = __fmul_rn(wj, __fmul_rn(n[i], rsj));
             prod[i] = use ? p : -0.0f;
           }
           add8_rn(acc, prod);
         }
       }
-      if (redo) {  // special pairs, or a routed vector near a rounding tie
+      // special pairs, or a row with a tiny scale: the general path
+      // (the shuffles need the whole warp, so every lane walks it when any does)
+      if (__any_sync(0xFFFFFFFFu, redo != 0u)) {
         float ori[8];
         if (SPECIAL && any_special && a.ori_x != nullptr)
           widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
+        float acc2[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-#pragma unroll
+        for (int i = 0; i < 8; ++i) acc2[i] = 0.0f;
+#pragma unroll 1
         for (int j = 0; j < KMAX; ++j) {
-          if (kindj[j] == kSkip) continue;
+          const int kind = __shfl_sync(0xFFFFFFFFu, lkind, j);
+          const float wj = __shfl_sync(0xFFFFFFFFu, lw, j);
+          const float rmj = __shfl_sync(0xFFFFFFFFu, rm, j);
+          const float rsj = __shfl_sync(0xFFFFFFFFu, rs, j);
+          const float rij = __shfl_sync(0xFFFFFFFFu, ri, j);
+          if (kind == kSkip) continue;
           float m[8];
-          if (kindj[j] == kRouted) {
+          if (kind == kRouted) {
             float y[8];
             widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
-            quant_roundtrip8(y, rmj[j], rsj[j], rij[j], m);
+            quant_roundtrip8<true>(y, rmj, rsj, rij, m);
           } else {
-            pair_values<T16, SPECIAL>(a, kindj[j], pmeta[j].row, V, v, make_uint4(0, 0, 0, 0),
-                                      ori, m);
+            pair_values<T16, SPECIAL>(a, kind, pmeta[j].row, V, v, make_uint4(0, 0, 0, 0), ori, m);
           }
-          axpy8_rn(acc, wj[j], m);
+          axpy8_rn(acc2, wj, m);
         }
+        if (redo != 0u)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = acc2[i];
       }
+      if (!act) continue;
       if (a.shared != nullptr) {
         float sh[8];
         widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
@@ -506,6 +527,8 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
       }
       st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + b);  // this warp is done with buffer b
   }
 }
 
@@ -547,12 +570,16 @@ __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pa
       float gf[8], yf[8], o[8];
       widen8<T16>(gv[u], gf);
       widen8<T16>(yv[u], yf);
-      const unsigned long long ww = pack2(w, w);
+      const float2 ww = f2(w, w);
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
-        const unsigned long long g2 = pack2(gf[i], gf[i + 1]);
-        unpack2(fma2_rn(g2, pack2(yf[i], yf[i + 1]), pack2(d[i], d[i + 1])), d[i], d[i + 1]);
-        unpack2(mul2_rn(ww, g2), o[i], o[i + 1]);
+        const float2 g2 = f2(gf[i], gf[i + 1]);
+        const float2 dd = __ffma2_rn(g2, f2(yf[i], yf[i + 1]), f2(d[i], d[i + 1]));
+        d[i] = dd.x;
+        d[i + 1] = dd.y;
+        const float2 oo = __fmul2_rn(ww, g2);
+        o[i] = oo.x;
+        o[i + 1] = oo.y;
       }
       st_v4(ge + v, narrow8<T16>(o));
     }

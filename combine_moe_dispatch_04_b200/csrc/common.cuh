@@ -93,50 +93,33 @@ __device__ __forceinline__ float absmax_final(uint32_t acc) {
 // ---- packed fp32 pairs (sm_100: one instruction, each lane rounded as the
 // scalar op would be) ----
 
-// A register pair viewed as one 64-bit operand (no data movement).
-__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
-  unsigned long long v;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
-  return v;
-}
-__device__ __forceinline__ void unpack2(unsigned long long v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long mul2_rn(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long add2_rn(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long fma2_rn(unsigned long long a, unsigned long long b,
-                                                       unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
+// Packed fp32 pairs: __fadd2_rn / __fmul2_rn / __ffma2_rn, one instruction
+// per pair. A packed product that feeds a packed sum was observed to lose its
+// own rounding on B200 (outputs one ulp off), so every product that is then
+// added is a scalar __fmul_rn (never contracted); packed multiplies only feed
+// other multiplies or stores.
+__device__ __forceinline__ float2 f2(float lo, float hi) { return make_float2(lo, hi); }
 
-// acc[i] = acc[i] + w * m[i] for 8 values, product and sum each rounded once.
-// The products are scalar __fmul_rn: a packed multiply followed by a packed
-// add was observed to lose the separate product rounding on B200 (outputs one
-// ulp off), while the scalar .rn multiply is never contracted. A lone add has
-// nothing to fuse with, so the sums are packed.
+// acc[i] = acc[i] + w * m[i] for 8 values, product and sum each rounded once
+// (scalar products, packed sums).
 __device__ __forceinline__ void axpy8_rn(float (&acc)[8], float w, const float (&m)[8]) {
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
-    const unsigned long long p = pack2(__fmul_rn(w, m[i]), __fmul_rn(w, m[i + 1]));
-    unpack2(add2_rn(pack2(acc[i], acc[i + 1]), p), acc[i], acc[i + 1]);
+    const float2 a =
+        __fadd2_rn(f2(acc[i], acc[i + 1]), f2(__fmul_rn(w, m[i]), __fmul_rn(w, m[i + 1])));
+    acc[i] = a.x;
+    acc[i + 1] = a.y;
   }
 }
 
 // acc[i] = acc[i] + m[i] for 8 values.
 __device__ __forceinline__ void add8_rn(float (&acc)[8], const float (&m)[8]) {
 #pragma unroll
-  for (int i = 0; i < 8; i += 2)
-    unpack2(add2_rn(pack2(acc[i], acc[i + 1]), pack2(m[i], m[i + 1])), acc[i], acc[i + 1]);
+  for (int i = 0; i < 8; i += 2) {
+    const float2 a = __fadd2_rn(f2(acc[i], acc[i + 1]), f2(m[i], m[i + 1]));
+    acc[i] = a.x;
+    acc[i + 1] = a.y;
+  }
 }
 
 // ---- global memory access ----
@@ -194,48 +177,88 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // bits: for |n| <= 127 the low byte is n in two's complement.
 constexpr float kRoundBias = 12582912.0f;        // 1.5 * 2^23
 constexpr float kTieGuard = 0.49993896484375f;   // 0.5 - 2^-14
-constexpr float kMinNormal = 1.17549435e-38f;    // 2^-126
+
+constexpr float kFastMinScale = 7.888609052210118e-31f;  // 2^-100
+
+// The code of one value whose r = fl32(y * inv_scale) lies within 2^-14 of a
+// half-integer h (n = rint(r), d = r - n), decided exactly without a division.
+// Let Q = y / scale. D = y - h * scale is exact in fp32 (for 16-bit y and
+// |Q - h| < 2^-13 it needs at most 11 significant bits), so one fma gives it.
+// fl32(Q) equals h when |Q - h| is at most half the fp32 spacing on that side
+// of h (h, with at most 9 significant bits, wins a tie at exactly half), i.e.
+// when |D| <= spacing / 2 * scale (exact products of powers of two, no
+// underflow for scale >= 2^-100); the spacing toward zero is halved at
+// h = +-0.5, the only power of two among half-integers. The code is then the
+// even one of h -+ 0.5 (round half to even), else the neighbour on Q's side.
+__device__ __forceinline__ float tie_code_inline(float y, float scale, float n, float d) {
+  const float h = n + (d > 0.0f ? 0.5f : -0.5f);
+  const float D = __fmaf_rn(-h, scale, y);
+  const float ah = fabsf(h);
+  const float e = __uint_as_float(__float_as_uint(ah) & 0x7F800000u);  // 2^floor(log2|h|)
+  const float u = e * 1.1920928955078125e-07f;                           // its spacing, 2^-23 e
+  const bool away = D != 0.0f && ((D > 0.0f) == (h > 0.0f));
+  const float lim = ((away || ah != e) ? u * 0.5f : u * 0.25f) * scale;
+  const float lo = h - 0.5f, hi = h + 0.5f;
+  const bool lo_even = (__float_as_uint(lo + kRoundBias) & 1u) == 0u;
+  if (fabsf(D) <= lim) return lo_even ? lo : hi;
+  return (away == (h > 0.0f)) ? hi : lo;
+}
+
+// The same decision as an out-of-line call: for kernels whose unrolled bodies
+// would otherwise carry many inline copies of this rarely taken code.
+static __device__ __noinline__ float tie_code_call(float y, float scale, float n, float d) {
+  return tie_code_inline(y, scale, n, d);
+}
 
 // The int8 codes n[i] = rne(fl32(y[i] / scale)) of eight values, as fp32
 // integers n and biased (b = n + 1.5 * 2^23, see above), for
 // scale = fl32(max|row| / 127) > 0 and every |y[i]| <= max|row|. Then
 // |y / scale| <= 127 (1 + 2^-23) and |n| <= 127, so no clamp is needed. With
-// fast set (scale normal and inv_scale = fl32(1 / scale)), r = y * inv_scale
+// fast set (scale >= 2^-100, inv_scale = fl32(1 / scale)), r = y * inv_scale
 // and the IEEE quotient fl32(y / scale) both lie within 127 * 3 * 2^-24 <
-// 2^-15 of the exact quotient; when every r is more than 2^-14 from every
-// half-integer, each r rounds to the same integer as its quotient. Otherwise
-// (rare: near a rounding tie) the IEEE divisions decide. Products are scalar
-// .rn multiplies (never contracted); the rest is packed and exact.
-// The fast path alone: n[i] = rint(fl32(y[i] * inv_scale)) (as fp32 integers)
-// and b[i] = n[i] + 1.5 * 2^23; returns max_i |r[i] - n[i]| (a tree of maxima).
-__device__ __forceinline__ float quant_fast8(const float (&y)[8], float inv_scale, float (&n)[8],
-                                             float (&b)[8]) {
-  const unsigned long long bias2 = pack2(kRoundBias, kRoundBias);
-  const unsigned long long nbias2 = pack2(-kRoundBias, -kRoundBias);
-  const unsigned long long neg2 = pack2(-1.0f, -1.0f);
-  float d[8];
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    const unsigned long long r2 = pack2(__fmul_rn(y[i], inv_scale), __fmul_rn(y[i + 1], inv_scale));
-    const unsigned long long b2 = add2_rn(r2, bias2);
-    const unsigned long long n2 = add2_rn(b2, nbias2);
-    unpack2(fma2_rn(n2, neg2, r2), d[i], d[i + 1]);  // r - n, exact
-    unpack2(b2, b[i], b[i + 1]);
-    unpack2(n2, n[i], n[i + 1]);
-  }
-  return fmaxf(fmaxf(fmaxf(fabsf(d[0]), fabsf(d[1])), fmaxf(fabsf(d[2]), fabsf(d[3]))),
-               fmaxf(fmaxf(fabsf(d[4]), fabsf(d[5])), fmaxf(fabsf(d[6]), fabsf(d[7]))));
-}
-
+// 2^-15 of the exact quotient; when r is more than 2^-14 from every
+// half-integer, both round to the same integer, and otherwise tie_code
+// decides exactly (inline, or as a call with OUTLINE). Without fast (a tiny
+// scale) the IEEE divisions decide.
+template <bool OUTLINE = false>
 __device__ __forceinline__ void quant_codes8(const float (&y)[8], float scale, float inv_scale,
                                              bool fast, float (&n)[8], float (&b)[8]) {
-  const float dmax = fast ? quant_fast8(y, inv_scale, n, b) : 1.0f;
-  if (!(dmax < kTieGuard)) {
+  if (fast) {
+    const float2 bias2 = f2(kRoundBias, kRoundBias);
+    const float2 nbias2 = f2(-kRoundBias, -kRoundBias);
+    const float2 neg2 = f2(-1.0f, -1.0f);
+    float d[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      b[i] = __fadd_rn(__fdiv_rn(y[i], scale), kRoundBias);
-      n[i] = __fsub_rn(b[i], kRoundBias);
+    for (int i = 0; i < 8; i += 2) {
+      const float2 r2 = f2(__fmul_rn(y[i], inv_scale), __fmul_rn(y[i + 1], inv_scale));
+      const float2 b2 = __fadd2_rn(r2, bias2);
+      const float2 n2 = __fadd2_rn(b2, nbias2);
+      const float2 d2 = __ffma2_rn(n2, neg2, r2);  // r - n, exact
+      b[i] = b2.x;
+      b[i + 1] = b2.y;
+      n[i] = n2.x;
+      n[i + 1] = n2.y;
+      d[i] = d2.x;
+      d[i + 1] = d2.y;
     }
+    const float dmax =
+        fmaxf(fmaxf(fmaxf(fabsf(d[0]), fabsf(d[1])), fmaxf(fabsf(d[2]), fabsf(d[3]))),
+              fmaxf(fmaxf(fabsf(d[4]), fabsf(d[5])), fmaxf(fabsf(d[6]), fabsf(d[7]))));
+    if (dmax >= kTieGuard) {  // one branch per vector, rarely taken
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (fabsf(d[i]) >= kTieGuard) {
+          n[i] = OUTLINE ? tie_code_call(y[i], scale, n[i], d[i])
+                         : tie_code_inline(y[i], scale, n[i], d[i]);
+          b[i] = __fadd_rn(n[i], kRoundBias);
+        }
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    b[i] = __fadd_rn(__fdiv_rn(y[i], scale), kRoundBias);
+    n[i] = __fsub_rn(b[i], kRoundBias);
   }
 }
 
@@ -251,7 +274,7 @@ __device__ __forceinline__ uint4 pack_codes16(const float (&y)[16], float amax, 
                                               float inv_scale) {
   uint32_t w[4] = {0u, 0u, 0u, 0u};
   if (amax != 0.0f) {
-    const bool fast = scale >= kMinNormal;
+    const bool fast = scale >= kFastMinScale;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float n[8], b[8];
@@ -272,7 +295,7 @@ __device__ __forceinline__ uint2 pack_codes8(const float (&y)[8], float amax, fl
                                              float inv_scale) {
   if (amax == 0.0f) return make_uint2(0u, 0u);
   float n[8], b[8];
-  quant_codes8(y, scale, inv_scale, scale >= kMinNormal, n, b);
+  quant_codes8(y, scale, inv_scale, scale >= kFastMinScale, n, b);
   uint32_t w[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
@@ -285,6 +308,7 @@ __device__ __forceinline__ uint2 pack_codes8(const float (&y)[8], float amax, fl
 
 // m[i] = n[i] * scale, the fp32 values of the int8 round trip of eight values
 // of a row (0 for an all-zero row), scale = fl32(amax / 127).
+template <bool OUTLINE = false>
 __device__ __forceinline__ void quant_roundtrip8(const float (&y)[8], float amax, float scale,
                                                  float inv_scale, float (&m)[8]) {
   if (amax == 0.0f) {
@@ -293,10 +317,14 @@ __device__ __forceinline__ void quant_roundtrip8(const float (&y)[8], float amax
     return;
   }
   float n[8], b[8];
-  quant_codes8(y, scale, inv_scale, scale >= kMinNormal, n, b);
-  const unsigned long long s2 = pack2(scale, scale);
+  quant_codes8<OUTLINE>(y, scale, inv_scale, scale >= kFastMinScale, n, b);
+  const float2 s2 = f2(scale, scale);
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) unpack2(mul2_rn(pack2(n[i], n[i + 1]), s2), m[i], m[i + 1]);
+  for (int i = 0; i < 8; i += 2) {
+    const float2 v = __fmul2_rn(f2(n[i], n[i + 1]), s2);
+    m[i] = v.x;
+    m[i + 1] = v.y;
+  }
 }
 
 // Whether pair (t, k) is active under x_active_mask (1-D per token, 2-D per pair).

@@ -217,9 +217,9 @@ __global__ void __launch_bounds__(kSmoothThreads) permute_quant_smooth_kernel(
 
 // Smooth-scaled int8 with each warp's token rows staged in shared memory: a
 // CTA takes a contiguous run of slots and its warps take them in turn (so
-// they share the current expert's smooth row through L1). Lane 0 of a warp
-// looks up the pair and expert of the slot kSmoothStages - 1 places ahead and
-// starts one bulk copy of its token row into the warp's next buffer
+// they share the current expert's smooth row through L1). The warp loads the
+// pairs and experts of 32 of its slots at once; lane 0 starts one bulk copy of
+// the token row of the slot kSmoothStages - 1 places ahead into the warp's next buffer
 // (cp.async.bulk on the buffer's mbarrier), so the gather is in flight while
 // the current slot is quantised. Lane l handles 16-byte vectors l, l + 32, ...
 // of the row: one pass for max|x * s| (warp reduction), one for the codes
@@ -263,22 +263,33 @@ __global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
   const int lo = blockIdx.x * per;
   const int hi = min(R, lo + per);
 
-  // Lane 0: slot s into buffer b.
-  auto stage = [&](int s, int b) {
-    const int pair = __ldg(assist + s);
-    int e = pair >= 0 ? __ldg(topk_idx + pair) : -1;
-    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) e = -1;
-    info[b] = SmoothSlot{e, s};
-    fence_proxy_async_smem();  // the buffer was last read by the warp's loads
-    mbar_arrive_expect_tx(bars + b, e >= 0 ? row_bytes : 0u);
-    if (e >= 0)
-      bulk_g2s(rows + static_cast<size_t>(b) * V, x + static_cast<size_t>(pair / K) * V, row_bytes,
-               bars + b);
+  // The warp's q-th slot is lo + warp + q * nwarps. Lane l holds the pair and
+  // expert of slot qb + l of the current batch of 32, loaded together, so the
+  // index round trips are paid once per 32 slots.
+  int qb = -32, my_pair = -1, my_e = -1;
+  // All lanes: slot q into buffer b (lane 0 records it and starts the copy).
+  auto stage = [&](int q, int b) {
+    if (q >= qb + 32) {
+      qb = q;
+      const int s = lo + warp + (qb + lane) * nwarps;
+      my_pair = s < hi ? __ldg(assist + s) : -1;
+      my_e = my_pair >= 0 ? __ldg(topk_idx + my_pair) : -1;
+      if (static_cast<unsigned>(my_e) >= static_cast<unsigned>(E)) my_e = -1;
+    }
+    const int pair = __shfl_sync(0xFFFFFFFFu, my_pair, q - qb);
+    const int e = __shfl_sync(0xFFFFFFFFu, my_e, q - qb);
+    if (lane == 0) {
+      info[b] = SmoothSlot{e, lo + warp + q * nwarps};
+      fence_proxy_async_smem();  // the buffer was last read by the warp's loads
+      mbar_arrive_expect_tx(bars + b, e >= 0 ? row_bytes : 0u);
+      if (e >= 0)
+        bulk_g2s(rows + static_cast<size_t>(b) * V, x + static_cast<size_t>(pair / K) * V,
+                 row_bytes, bars + b);
+    }
   };
 
-  if (lane == 0)
-    for (int p = 0; p < kSmoothStages - 1; ++p)
-      if (lo + warp + p * nwarps < hi) stage(lo + warp + p * nwarps, p);
+  for (int p = 0; p < kSmoothStages - 1; ++p)
+    if (lo + warp + p * nwarps < hi) stage(p, p);
   int it = 0;
   for (int s = lo + warp; s < hi; s += nwarps, ++it) {
     const int b = it % kSmoothStages;
@@ -294,8 +305,8 @@ __global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
     }
     // the buffer of the previous slot is free (its reads ended before the
     // __syncwarp below): refill it with the slot kSmoothStages - 1 ahead
-    const int ahead = s + (kSmoothStages - 1) * nwarps;
-    if (lane == 0 && ahead < hi) stage(ahead, (it + kSmoothStages - 1) % kSmoothStages);
+    if (s + (kSmoothStages - 1) * nwarps < hi)
+      stage(it + kSmoothStages - 1, (it + kSmoothStages - 1) % kSmoothStages);
     const SmoothSlot si = info[b];
     if (si.e >= 0) {
       const uint4* xr = rows + static_cast<size_t>(b) * V;
