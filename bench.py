@@ -516,12 +516,12 @@ def main():
     # billed to the step. Both run before the step's start event.
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
     flush = torch.empty(2 * l2 // 4, dtype=torch.int32, device=dev)
-    sweep = torch.zeros(2 * l2 // 4, dtype=torch.int32, device=dev)
-    sweep_out = torch.empty((), dtype=torch.int64, device=dev)
+    sweep = torch.zeros(2 * l2 // 4, dtype=torch.float32, device=dev)
+    sweep_out = torch.empty((), dtype=torch.float32, device=dev)
 
     def flush_l2():
         flush.zero_()
-        torch.sum(sweep, dim=0, dtype=torch.int64, out=sweep_out)
+        torch.sum(sweep, dim=0, out=sweep_out)  # one reduction kernel
 
     for _ in range(args.warmup):
         flush_l2()
