@@ -179,7 +179,7 @@ def measured_hbm_peak():
 
 KERNEL_SOURCES = {"layout": "layout.cu", "dispatch": "layout.cu", "permute": "permute.cu",
                   "combine_fwd": "combine.cu", "combine_bwd_special": "special_bwd.cu",
-                  "combine_bwd": "combine.cu", "dispatch_bwd": "combine.cu"}
+                  "combine_bwd": "combine_bwd.cu", "dispatch_bwd": "combine.cu"}
 
 
 def kernel_source_hash(kernel: str) -> str:

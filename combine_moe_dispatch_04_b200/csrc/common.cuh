@@ -335,4 +335,21 @@ __device__ __forceinline__ bool pair_active(const uint8_t* mask, int mask_ndim, 
   return __ldg(mask + static_cast<size_t>(t) * K + k) != 0;
 }
 
+// Resident blocks per SM of a kernel (occupancy API), cached per kernel and
+// block size (a multiple of 32, at most 1024); each kernel is always launched
+// with the same shared memory size.
+template <auto Kernel>
+int blocks_per_sm(int threads, size_t smem) {
+  static int cached[33] = {};
+  const int slot = threads >= 1024 ? 32 : threads / 32;
+  if (cached[slot] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    cached[slot] = n;
+  }
+  return cached[slot];
+}
+
 }  // namespace moe
