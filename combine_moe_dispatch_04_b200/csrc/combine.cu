@@ -465,14 +465,14 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
       if (!redo) {
         // Routed rows only: every row computed without a branch, its terms
         // selected in (unselected ones add -0, which leaves any sum as it is).
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < KMAX; ++j) {
           const float rfj = __shfl_sync(0xFFFFFFFFu, rf, j);
           const float rsj = __shfl_sync(0xFFFFFFFFu, rs, j);
           const float wj = __shfl_sync(0xFFFFFFFFu, lw, j);
           float y[8], n[8], b[8], prod[8];
           widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
-          quant_codes8<true>(y, rsj, rfj, true, n, b);  // exact, ties included
+          quant_codes8<false>(y, rsj, rfj, true, n, b);  // exact, ties included
           const bool use = (routed >> j) & 1u;
           redo |= (use && !((fastm >> j) & 1u)) ? 1u : 0u;  // a tiny scale: IEEE divisions
 #pragma unroll

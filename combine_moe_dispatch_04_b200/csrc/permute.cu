@@ -227,6 +227,18 @@ __global__ void __launch_bounds__(kSmoothThreads) permute_quant_smooth_kernel(
 // gives up counts itself in *timeouts and returns.
 constexpr int kSmoothStages = 3;
 
+// y[i] = fl(y[i] * s[i]) for eight values, in pairs. y only feeds other
+// products and a max, never a sum, so the packed multiply keeps every
+// product's own rounding.
+__device__ __forceinline__ void smooth_mul8(float (&y)[8], const float4& m0, const float4& m1) {
+  const float2 p0 = __fmul2_rn(f2(y[0], y[1]), f2(m0.x, m0.y));
+  const float2 p1 = __fmul2_rn(f2(y[2], y[3]), f2(m0.z, m0.w));
+  const float2 p2 = __fmul2_rn(f2(y[4], y[5]), f2(m1.x, m1.y));
+  const float2 p3 = __fmul2_rn(f2(y[6], y[7]), f2(m1.z, m1.w));
+  y[0] = p0.x; y[1] = p0.y; y[2] = p1.x; y[3] = p1.y;
+  y[4] = p2.x; y[5] = p2.y; y[6] = p3.x; y[7] = p3.y;
+}
+
 struct SmoothSlot {
   int e;     // expert of the slot, -1: nothing to do
   int slot;
@@ -317,10 +329,7 @@ __global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
         float y[8];
         widen8<T16>(xr[v], y);
         const float4 m0 = __ldg(sr + 2 * v), m1 = __ldg(sr + 2 * v + 1);
-        y[0] = __fmul_rn(y[0], m0.x); y[1] = __fmul_rn(y[1], m0.y);
-        y[2] = __fmul_rn(y[2], m0.z); y[3] = __fmul_rn(y[3], m0.w);
-        y[4] = __fmul_rn(y[4], m1.x); y[5] = __fmul_rn(y[5], m1.y);
-        y[6] = __fmul_rn(y[6], m1.z); y[7] = __fmul_rn(y[7], m1.w);
+        smooth_mul8(y, m0, m1);
         amax = fmaxf(amax, absmax8(y));
       }
 #pragma unroll
@@ -333,10 +342,7 @@ __global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
         float y[8];
         widen8<T16>(xr[v], y);
         const float4 m0 = __ldg(sr + 2 * v), m1 = __ldg(sr + 2 * v + 1);
-        y[0] = __fmul_rn(y[0], m0.x); y[1] = __fmul_rn(y[1], m0.y);
-        y[2] = __fmul_rn(y[2], m0.z); y[3] = __fmul_rn(y[3], m0.w);
-        y[4] = __fmul_rn(y[4], m1.x); y[5] = __fmul_rn(y[5], m1.y);
-        y[6] = __fmul_rn(y[6], m1.z); y[7] = __fmul_rn(y[7], m1.w);
+        smooth_mul8(y, m0, m1);
         orow[v] = pack_codes8(y, amax, scale, inv_scale);
       }
       if (lane == 0) scales[si.slot] = scale;
