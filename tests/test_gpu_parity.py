@@ -111,6 +111,7 @@ COMM_QUANT = [
     W["uniform"].scaled(bs=2100, h=520, name="uniform_q8"),
     W["mixtral"].scaled(bs=1200, h=264, name="mixtral_fp16_mask_q8"),
     W["dsv3"].scaled(bs=300, h=7168, name="dsv3_shared_q8"),
+    W["dsv3"].scaled(bs=300, h=1024, name="dsv3_shared_q8_staged"),  # shared add, staged
     _custom("k16_q8", bs=700, k=16, num_experts=40, h=136, zero_expert_num=2,
             const_expert_num=2, backward=False),
     _custom("zero_only_q8", bs=900, k=4, num_experts=16, zero_expert_num=3, h=256,
