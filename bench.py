@@ -415,6 +415,10 @@ def main():
             const_v=d["v"], grad_w=gw, workspace=sp_ws)
         torch.cuda.synchronize()
 
+    # the step's results the caller reads back (swapped per slot by the e2e loop)
+    o = {"out": out}
+    if wl.backward:
+        o.update(gw=gw, gx=gx)
     cq = args.combine_comm_quant
     # the profiled kernel differs with the combine's quantisation mode
     traffic_key = wl.name + ("+comm_quant2" if cq == 2 else "")
@@ -439,23 +443,23 @@ def main():
         ("combine_fwd", lambda st: moe.combine_fwd(
             sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
             shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
-            const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, out=out,
+            const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, out=o["out"],
             stream=st)),
     ]
     if wl.backward:
         calls += [
             ("combine_bwd", lambda st: moe.combine_bwd(
                 sh, d["grad_out"], y, d["topk_weights"], lay, x_active_mask=d["mask"],
-                grad_expand=gexp, grad_w=gw, stream=st)),
+                grad_expand=gexp, grad_w=o["gw"], stream=st)),
         ]
         if "combine_bwd_special" in bytes_per:
             calls += [("combine_bwd_special", lambda st: moe.combine_bwd_special(
                 sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
                 x_active_mask=d["mask"], const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
-                const_v=d["v"], grad_w=gw, workspace=sp_ws, out=sp_out, stream=st))]
+                const_v=d["v"], grad_w=o["gw"], workspace=sp_ws, out=sp_out, stream=st))]
         calls += [
             ("dispatch_bwd", lambda st: moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"],
-                                                      grad_x=gx, stream=st)),
+                                                      grad_x=o["gx"], stream=st)),
         ]
     # the kernel that moves the most bytes; the timed steps bracket it with events
     dominant = max((k for k in kernels if k not in ("layout", "dispatch")),
@@ -592,40 +596,71 @@ def main():
     torch.cuda.synchronize()
     per_kernel_ms = {k: [m[k][0].elapsed_time(m[k][1]) for m in diag] for k in kernels}
 
-    # e2e: pinned host inputs -> H2D -> the path through the C ABI -> D2H of the results
+    # e2e: pinned host inputs -> H2D -> the path through the C ABI -> D2H of the results,
+    # every step. Inputs and results are double-buffered on the device: step i's
+    # uploads (a copy stream) and step i-1's read-back (another) overlap step i-1's
+    # and step i's kernels, as a serving loop would run them.
     e2e = None
     if not args.no_e2e:
         in_keys = [k for k in ("topk_idx", "topk_weights", "x", "mask", "shared", "grad_out")
                    if d[k] is not None]
         h_in = {k: d[k].cpu().pin_memory() for k in in_keys}
-        outs = [out] + ([gx, gw] if wl.backward else [])
-        h_out = [o.cpu().pin_memory() for o in outs]
+        out_keys = list(o)
+        h_out = {k: o[k].cpu().pin_memory() for k in out_keys}
         bi = sum(t.numel() * t.element_size() for t in h_in.values())
-        bo = sum(t.numel() * t.element_size() for t in h_out)
+        bo = sum(t.numel() * t.element_size() for t in h_out.values())
         e2e_steps = max(3, args.steps // 4)
+        slots = [({k: d[k] for k in in_keys}, dict(o)),
+                 ({k: torch.empty_like(d[k]) for k in in_keys},
+                  {k: torch.empty_like(o[k]) for k in out_keys})]
+        up_s, down_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev = [{n: torch.cuda.Event() for n in ("in", "done", "read")} for _ in slots]
+        uses_ori = d["ori_x"] is not None
 
-        def e2e_step():
-            for k in in_keys:
-                d[k].copy_(h_in[k], non_blocking=True)
+        def e2e_step(i):
+            din, dout = slots[i % 2]
+            e = ev[i % 2]
+            with torch.cuda.stream(up_s):
+                if i >= 2:
+                    up_s.wait_event(e["done"])  # step i-2 no longer reads these inputs
+                for k in in_keys:
+                    din[k].copy_(h_in[k], non_blocking=True)
+                e["in"].record(up_s)
+            stream.wait_event(e["in"])
+            if i >= 2:
+                stream.wait_event(e["read"])  # step i-2's results have been read back
+            d.update(din)
+            if uses_ori:
+                d["ori_x"] = din["x"]  # the token rows the copy/const experts return
+            o.update(dout)
             step()
-            for o, ho in zip(outs, h_out):
-                ho.copy_(o, non_blocking=True)
+            e["done"].record(stream)
+            with torch.cuda.stream(down_s):
+                down_s.wait_event(e["done"])
+                for k in out_keys:
+                    h_out[k].copy_(dout[k], non_blocking=True)
+                e["read"].record(down_s)
 
-        for _ in range(3):
-            e2e_step()
+        for i in range(4):
+            e2e_step(i)
         torch.cuda.synchronize()
         ea = torch.cuda.Event(enable_timing=True)
         eb = torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         ea.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
+        up_s.wait_stream(stream)
+        down_s.wait_stream(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        stream.wait_stream(down_s)
         eb.record(stream)
         torch.cuda.synchronize()
         e_ms = reduce_max(ea.elapsed_time(eb), dev)
         e2e = {"value": whole_job_throughput(wl.bs, e2e_steps, world, e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps}
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps,
+               "note": "double-buffered: each step's uploads and read-back overlap the "
+                       "neighbouring steps' kernels on two copy streams"}
 
     if rank == 0:
         peak, peak_kind = measured_hbm_peak()

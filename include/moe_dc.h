@@ -278,7 +278,7 @@ moe_status moe_dispatch_bwd(const moe_shape* shape, const void* grad_expand_in,
 
 /*
  * moe_dispatch_layout_noalloc — moe_dispatch_layout for callers that cannot
- * allocate device memory. No counterpart in the paper: an addition of this
+ * allocate device memory. No counterpart on the [combine] page: an addition of this
  * library. It is for code that runs where every byte of device memory is
  * owned by someone else — a plugin or kernel library handed buffers by a host
  * framework that exposes no allocator, or a latency-critical serving loop that
