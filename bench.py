@@ -420,6 +420,13 @@ def main():
     if wl.backward:
         o.update(gw=gw, gx=gx)
     cq = args.combine_comm_quant
+    q8_ws = None
+    if cq == 2:  # the int8 combine's workspace, allocated once outside the timed steps
+        nb = moe.moe_combine_fwd_comm_quant_workspace_bytes(ctypes.byref(sh.c()))
+        q8_ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+    special_ids = wl.zero_expert_num + wl.copy_expert_num + wl.const_expert_num
+    q8_two_pass = (cq == 2 and special_ids == 0 and
+                   wl.h // 8 >= 32 * (4 if wl.k <= 2 else 2 if wl.k <= 4 else 1))
     # the profiled kernel differs with the combine's quantisation mode
     traffic_key = wl.name + ("+comm_quant2" if cq == 2 else "")
     if args.fused_dispatch:
@@ -443,8 +450,8 @@ def main():
         ("combine_fwd", lambda st: moe.combine_fwd(
             sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
             shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
-            const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, out=o["out"],
-            stream=st)),
+            const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, workspace=q8_ws,
+            out=o["out"], stream=st)),
     ]
     if wl.backward:
         calls += [
@@ -512,7 +519,8 @@ def main():
     special_bwd_launches = 0
     if "combine_bwd_special" in bytes_per:
         special_bwd_launches = 1 + (2 if wl.const_expert_num else 0)
-    launches_per_step = dispatch_launches + 1 + (2 if wl.backward else 0) + special_bwd_launches
+    launches_per_step = (dispatch_launches + (2 if q8_two_pass else 1) + (2 if wl.backward else 0)
+                         + special_bwd_launches)
 
     # L2 flush between steps: write a buffer twice the size of L2, then read
     # another one as large, so the step starts with none of its data in L2 and
@@ -684,6 +692,8 @@ def main():
                        "fused_dispatch": bool(args.fused_dispatch),
                        "smooth_quant": bool(wl.smooth),
                        "combine_comm_quant_mode": cq,
+                       "combine_int8_kernels": ("two-pass" if q8_two_pass else "single-pass")
+                                               if cq == 2 else None,
                        "launch": "CUDA graph of the step" if use_graph else "eager launches",
                        "l2": "flushed before every step (write of 2x L2, then a read of another 2x L2 so "
                              "no dirty flush lines are written back inside the step), outside "

@@ -28,7 +28,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_dispatch_layout_noalloc", "moe_layout_noalloc_max_workspace_bytes",
            "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
            "moe_combine_bwd_special_workspace_bytes", "moe_dispatch_permute_smooth",
-           "moe_async_wait_timeouts")
+           "moe_async_wait_timeouts", "moe_combine_fwd_comm_quant_ws",
+           "moe_combine_fwd_comm_quant_workspace_bytes")
 
 
 class MoeShape(ctypes.Structure):
@@ -64,6 +65,10 @@ def _load():
     L.moe_async_wait_timeouts.argtypes, L.moe_async_wait_timeouts.restype = [], ctypes.c_uint32
     L.moe_combine_fwd.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_combine_fwd_comm_quant.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P]
+    L.moe_combine_fwd_comm_quant_ws.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, I, P, P,
+                                                ctypes.c_size_t, P]
+    L.moe_combine_fwd_comm_quant_workspace_bytes.argtypes = [S]
+    L.moe_combine_fwd_comm_quant_workspace_bytes.restype = ctypes.c_size_t
     L.moe_dispatch.argtypes = [S, P, P, P, I, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_combine_bwd_special.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                           ctypes.c_size_t, P]
@@ -77,7 +82,7 @@ def _load():
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
               "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
               "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
-              "moe_dispatch_permute_smooth"):
+              "moe_dispatch_permute_smooth", "moe_combine_fwd_comm_quant_ws"):
         getattr(L, n).restype = I
     return L
 
@@ -98,6 +103,8 @@ moe_combine_bwd = _lib.moe_combine_bwd
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
 moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
 moe_combine_fwd_comm_quant = _lib.moe_combine_fwd_comm_quant
+moe_combine_fwd_comm_quant_ws = _lib.moe_combine_fwd_comm_quant_ws
+moe_combine_fwd_comm_quant_workspace_bytes = _lib.moe_combine_fwd_comm_quant_workspace_bytes
 moe_dispatch = _lib.moe_dispatch
 moe_combine_bwd_special = _lib.moe_combine_bwd_special
 moe_combine_bwd_special_workspace_bytes = _lib.moe_combine_bwd_special_workspace_bytes
@@ -275,7 +282,11 @@ def dispatch_permute_smooth(shape: Shape, x, topk_idx, layout: Layout, smooth_sc
 
 def combine_fwd(shape: Shape, expand_x, topk_idx, topk_weights, layout: Layout, *,
                 x_active_mask=None, shared_expert_x=None, ori_x=None, const_alpha_1=None,
-                const_alpha_2=None, const_v=None, comm_quant_mode=0, out=None, stream=None):
+                const_alpha_2=None, const_v=None, comm_quant_mode=0, workspace=None,
+                use_workspace=True, out=None, stream=None):
+    """Combine forward. With comm_quant_mode 2, a workspace (allocated here unless
+    given, or none with use_workspace=False) lets shapes without zero/copy/const
+    experts take the two-pass kernels; the result is the same either way."""
     import torch
 
     if out is None:
@@ -286,9 +297,18 @@ def combine_fwd(shape: Shape, expand_x, topk_idx, topk_weights, layout: Layout, 
             _ptr(const_v))
     if comm_quant_mode == 0:
         _check("moe_combine_fwd", moe_combine_fwd(*args, _ptr(out), _stream(stream)))
+        return out
+    nbytes = 0
+    if use_workspace:
+        nbytes = moe_combine_fwd_comm_quant_workspace_bytes(ctypes.byref(shape.c()))
+        if workspace is None and nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=expand_x.device)
     else:
-        _check("moe_combine_fwd_comm_quant", moe_combine_fwd_comm_quant(
-            *args, comm_quant_mode, _ptr(out), _stream(stream)))
+        workspace = None
+    _check("moe_combine_fwd_comm_quant_ws", moe_combine_fwd_comm_quant_ws(
+        *args, comm_quant_mode, _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream(stream)))
     return out
 
 

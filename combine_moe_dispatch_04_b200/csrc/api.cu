@@ -233,7 +233,26 @@ moe_status moe_combine_fwd_comm_quant(const moe_shape* s, const void* expand_x,
                                       const void* ori_x, const void* const_alpha_1,
                                       const void* const_alpha_2, const void* const_v,
                                       int comm_quant_mode, void* out, void* stream) {
-  (void)ep_send_counts;
+  return moe_combine_fwd_comm_quant_ws(s, expand_x, topk_idx, topk_weights, assist_info,
+                                       ep_send_counts, x_active_mask, shared_expert_x, ori_x,
+                                       const_alpha_1, const_alpha_2, const_v, comm_quant_mode,
+                                       out, nullptr, 0, stream);
+}
+
+size_t moe_combine_fwd_comm_quant_workspace_bytes(const moe_shape* s) {
+  if (s == nullptr || s->a_capacity <= 0) return 0;
+  return moe::combine_q8_workspace_bytes(s->a_capacity);
+}
+
+moe_status moe_combine_fwd_comm_quant_ws(const moe_shape* s, const void* expand_x,
+                                         const int32_t* topk_idx, const float* topk_weights,
+                                         const int32_t* assist_info,
+                                         const int32_t* ep_send_counts,
+                                         const uint8_t* x_active_mask,
+                                         const void* shared_expert_x, const void* ori_x,
+                                         const void* const_alpha_1, const void* const_alpha_2,
+                                         const void* const_v, int comm_quant_mode, void* out,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
   if (comm_quant_mode != 0 && comm_quant_mode != 2) return MOE_ERR_ARG;
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
@@ -251,8 +270,12 @@ moe_status moe_combine_fwd_comm_quant(const moe_shape* s, const void* expand_x,
     return MOE_ERR_ARG;
   if (!aligned16(expand_x) || !aligned16(out) || !aligned16(shared_expert_x) ||
       !aligned16(ori_x) || !aligned16(const_alpha_1) || !aligned16(const_alpha_2) ||
-      !aligned16(const_v))
+      !aligned16(const_v) || !aligned16(workspace))
     return MOE_ERR_ALIGN;
+  if (workspace != nullptr &&
+      workspace_bytes < moe::combine_q8_workspace_bytes(s->a_capacity > 0 ? s->a_capacity : 0))
+    return MOE_ERR_CAPACITY;
+  if (workspace != nullptr && s->bs > 0 && ep_send_counts == nullptr) return MOE_ERR_ARG;
   moe::CombineArgs a;
   a.expand_x = expand_x;
   a.topk_idx = topk_idx;
@@ -276,8 +299,9 @@ moe_status moe_combine_fwd_comm_quant(const moe_shape* s, const void* expand_x,
   a.Q = s->const_expert_num;
   a.dtype = s->dtype;
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return cuda_status(comm_quant_mode == 2 ? moe::launch_combine_fwd_q8(a, cs)
-                                          : moe::launch_combine_fwd(a, cs));
+  return cuda_status(comm_quant_mode == 2
+                         ? moe::launch_combine_fwd_q8(a, ep_send_counts, workspace, cs)
+                         : moe::launch_combine_fwd(a, cs));
 }
 
 moe_status moe_combine_bwd(const moe_shape* s, const void* grad_out, const void* expand_x,

@@ -224,6 +224,118 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
 }
 
 // ---------------------------------------------------------------------------
+// Combine forward with comm_quant_mode 2 in two passes over a caller workspace.
+//
+// Pass 1 (row_scale_kernel): one warp per slot row s < R, streaming the row
+// once: max|y| on packed 16-bit pairs, a warp reduction, and then
+// rscale[s] = (scale, reciprocal) with scale = fl(max / 127) (IEEE division);
+// the reciprocal is 0 for an all-zero row (its codes are 0) and -1 marks a
+// scale below 2^-100 (the codes then come from IEEE divisions).
+template <typename T16>
+__global__ void __launch_bounds__(256) row_scale_kernel(const uint4* __restrict__ Y,
+                                                         const int32_t* __restrict__ send,
+                                                         int E, int A, int V,
+                                                         float2* __restrict__ rscale) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int R = min(max(__ldg(send + E), 0), A);
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int s = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); s < R; s += nw) {
+    const uint4* row = Y + static_cast<size_t>(s) * V;
+    uint32_t m2 = 0;
+#pragma unroll 4
+    for (int v = lane; v < V; v += 32) m2 = absmax_v4<T16>(m2, ld_nc_v4(row + v));
+    float mx = absmax_final<T16>(m2);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+    if (lane == 0) {
+      const float scale = __fdiv_rn(mx, 127.0f);
+      const float inv = mx == 0.0f ? 0.0f : (scale >= kFastMinScale ? 1.0f / scale : -1.0f);
+      rscale[s] = make_float2(scale, inv);
+    }
+  }
+}
+
+// Pass 2 (combine_fwd_rt_kernel): the one-shot gather of combine_fwd_kernel
+// (routed pairs only, rows of at least 32 U vectors) with, per routed pair,
+// the int8 codes of its values (quant_codes8) and their dequantisation
+// fl(code * scale) before the same weighted fp32 sum. The lane that classified
+// a pair also holds its (scale, reciprocal); every lane fetches them by
+// shuffle when the pair's turn comes, so no per-pair array is kept.
+template <typename T16, int KMAX>
+__global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, false>() - 1))
+    combine_fwd_rt_kernel(CombineArgs a, const float2* __restrict__ rscale) {
+  constexpr int U = fwd_vectors_per_thread<KMAX>();
+  pdl_trigger();
+  pdl_wait();
+  const int V = a.H / kVecElems;
+  const int K = a.K;
+  const int n = a.bs * V;
+  const int lane = threadIdx.x & 31;
+  const int span = blockIdx.x * (kFwdThreads * U) + (threadIdx.x >> 5) * (32 * U);
+  if (span >= n) return;  // warp-uniform
+  const uint4* Y = static_cast<const uint4*>(a.expand_x);
+  // lanes 0..K-1 classify the span's first token's pairs, lanes 16..16+K-1 the next one's
+  const int t0 = span / V;
+  const int tm = t0 + (lane >> 4), km = lane & 15;
+  PairMeta pm{kSkip, 0, 1.0f};
+  if (km < K && tm < a.bs) pm = classify_pair<false, false, false>(a, tm, km);
+  const float2 ms = pm.kind == kRouted ? __ldg(rscale + pm.row) : make_float2(0.0f, 0.0f);
+  uint4 val[U][KMAX];
+  uint32_t routed[U];
+  int src[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int item = span + u * 32 + lane;
+    const int v = item % V;
+    src[u] = item / V == t0 ? 0 : 16;
+    routed[u] = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const int kind = __shfl_sync(0xFFFFFFFFu, pm.kind, src[u] + j);
+      const int row = __shfl_sync(0xFFFFFFFFu, pm.row, src[u] + j);
+      if (j < K && item < n && kind == kRouted) {
+        routed[u] |= 1u << j;
+        val[u][j] = ld_nc_v4(Y + static_cast<size_t>(row) * V + v);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int item = span + u * 32 + lane;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const float w = __shfl_sync(0xFFFFFFFFu, pm.w, src[u] + j);
+      const float sc = __shfl_sync(0xFFFFFFFFu, ms.x, src[u] + j);
+      const float iv = __shfl_sync(0xFFFFFFFFu, ms.y, src[u] + j);
+      if ((routed[u] >> j) & 1u) {
+        float y[8], q[8], b[8], m[8];
+        widen8<T16>(val[u][j], y);
+        quant_codes8<true>(y, sc, iv, iv >= 0.0f, q, b);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          const float2 p = __fmul2_rn(f2(q[i], q[i + 1]), f2(sc, sc));
+          m[i] = p.x;
+          m[i + 1] = p.y;
+        }
+        axpy8_rn(acc, w, m);
+      }
+    }
+    if (item >= n) continue;
+    if (a.shared != nullptr) {
+      float sh[8];
+      widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.shared) + item), sh);
+      add8_rn(acc, sh);
+    }
+    st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Combine forward with comm_quant_mode 2 ([combine] Parameters): every routed
 // row returns through the per-row int8 round trip (scale = max|y| / 127 in
 // fp32, q = clamp(rne(y / scale), -127, 127), value = q * scale) before the
@@ -617,6 +729,39 @@ cudaError_t launch_fwd_q8(const CombineArgs& a, cudaStream_t st) {
   return launch_fwd_q8_t<T16, false>(a, st);
 }
 
+template <typename T16, int KMAX>
+cudaError_t launch_fwd_rt_k(const CombineArgs& a, const float2* rscale, cudaStream_t st) {
+  constexpr int U = fwd_vectors_per_thread<KMAX>();
+  const long long n = static_cast<long long>(a.bs) * (a.H / kVecElems);
+  const int blocks = static_cast<int>((n + kFwdThreads * U - 1) / (kFwdThreads * U));
+  return launch_pdl(combine_fwd_rt_kernel<T16, KMAX>, dim3(blocks), dim3(kFwdThreads), 0, st, a,
+                    rscale);
+}
+
+// The two-pass path: whether it applies (routed pairs only, rows wide enough
+// for the shared pair metadata), and its two launches.
+bool rt_applies(const CombineArgs& a) {
+  const int V = a.H / kVecElems;
+  const int U = a.K <= 2 ? 4 : a.K <= 4 ? 2 : 1;
+  return a.Z + a.C + a.Q == 0 && a.weights != nullptr && V >= 32 * U;
+}
+
+template <typename T16>
+cudaError_t launch_fwd_rt(const CombineArgs& a, const int32_t* send, float2* rscale,
+                          cudaStream_t st) {
+  const int V = a.H / kVecElems;
+  const long long want = (static_cast<long long>(a.A) + 7) / 8;  // 8 warps per CTA
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  const int blocks = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+  cudaError_t err = launch_pdl(row_scale_kernel<T16>, dim3(blocks), dim3(256), 0, st,
+                               static_cast<const uint4*>(a.expand_x), send, a.E, a.A, V, rscale);
+  if (err != cudaSuccess) return err;
+  if (a.K <= 2) return launch_fwd_rt_k<T16, 2>(a, rscale, st);
+  if (a.K <= 4) return launch_fwd_rt_k<T16, 4>(a, rscale, st);
+  if (a.K <= 8) return launch_fwd_rt_k<T16, 8>(a, rscale, st);
+  return launch_fwd_rt_k<T16, 16>(a, rscale, st);
+}
+
 }  // namespace
 
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st) {
@@ -624,8 +769,16 @@ cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st) {
   return a.dtype == MOE_BF16 ? launch_fwd_t<Bf16>(a, st) : launch_fwd_t<Fp16>(a, st);
 }
 
-cudaError_t launch_combine_fwd_q8(const CombineArgs& a, cudaStream_t st) {
+size_t combine_q8_workspace_bytes(int A) { return static_cast<size_t>(A) * sizeof(float2); }
+
+cudaError_t launch_combine_fwd_q8(const CombineArgs& a, const int32_t* send, void* workspace,
+                                  cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
+  if (workspace != nullptr && send != nullptr && a.A > 0 && rt_applies(a)) {
+    float2* rscale = static_cast<float2*>(workspace);
+    return a.dtype == MOE_BF16 ? launch_fwd_rt<Bf16>(a, send, rscale, st)
+                               : launch_fwd_rt<Fp16>(a, send, rscale, st);
+  }
   return a.dtype == MOE_BF16 ? launch_fwd_q8<Bf16>(a, st) : launch_fwd_q8<Fp16>(a, st);
 }
 

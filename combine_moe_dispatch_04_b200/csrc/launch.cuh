@@ -63,7 +63,12 @@ struct CombineArgs {
 };
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st);
 // comm_quant_mode 2: every routed row through the per-row int8 round trip (H <= 16384).
-cudaError_t launch_combine_fwd_q8(const CombineArgs& a, cudaStream_t st);
+// With a workspace of combine_q8_workspace_bytes(A) bytes and the total R in send[E], shapes
+// with routed pairs only take two passes (per-row scales, then the gather); otherwise the
+// staged kernel runs and the workspace is not touched.
+size_t combine_q8_workspace_bytes(int A);
+cudaError_t launch_combine_fwd_q8(const CombineArgs& a, const int32_t* send, void* workspace,
+                                  cudaStream_t st);
 
 struct CombineBwdArgs {
   const void* grad_out;

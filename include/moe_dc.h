@@ -224,6 +224,30 @@ moe_status moe_combine_fwd_comm_quant(const moe_shape* shape, const void* expand
                                       int comm_quant_mode, void* out, void* stream);
 
 /*
+ * moe_combine_fwd_comm_quant_ws — moe_combine_fwd_comm_quant with an optional
+ * device workspace (same results, bit for bit). With a workspace of
+ * moe_combine_fwd_comm_quant_workspace_bytes() bytes (16-byte aligned) and
+ * mode 2, shapes without zero/copy/const experts run in two passes: each slot
+ * row's scale and reciprocal into the workspace (one streaming read of the
+ * rows, R = ep_send_counts[E] of them), then the weighted gather with the
+ * round trip. Other shapes, or workspace NULL, take the single-pass kernel.
+ *   workspace        NULL or device scratch; its contents on entry do not
+ *                    matter (MOE_ERR_CAPACITY if smaller than required,
+ *                    MOE_ERR_ALIGN if not 16-byte aligned)
+ *   ep_send_counts   from moe_dispatch_layout; required with a workspace
+ */
+size_t moe_combine_fwd_comm_quant_workspace_bytes(const moe_shape* shape);
+moe_status moe_combine_fwd_comm_quant_ws(const moe_shape* shape, const void* expand_x,
+                                         const int32_t* topk_idx, const float* topk_weights,
+                                         const int32_t* assist_info,
+                                         const int32_t* ep_send_counts,
+                                         const uint8_t* x_active_mask,
+                                         const void* shared_expert_x, const void* ori_x,
+                                         const void* const_alpha_1, const void* const_alpha_2,
+                                         const void* const_v, int comm_quant_mode, void* out,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * moe_combine_bwd — gradient of the combine Formula for routed pairs (the
  * fused EP MoE layer of the Triton-distributed ep_moe_fused PR has a backward):
  *   grad_expand[slot(t,k)] = round16(w[t,k] * grad_out[t])     (fp32 product)

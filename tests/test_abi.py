@@ -110,6 +110,13 @@ def test_other_entry_points_check_first():
     # combine comm_quant_mode outside {0, 2}
     args2 = [p, p, p, p, None, None, None, None, None, None, None]
     assert moe.moe_combine_fwd_comm_quant(s, *args2, 1, p, None) == moe.MOE_ERR_ARG
+    # the workspace variant: 16-byte aligned, large enough, and ep_send_counts with it
+    ws = moe.moe_combine_fwd_comm_quant_workspace_bytes(s)
+    assert ws == 8 * 4096 * 8  # A = BS * K
+    cq = moe.moe_combine_fwd_comm_quant_ws
+    assert cq(s, *args2, 2, p, ctypes.c_void_p(264), ws, None) == moe.MOE_ERR_ALIGN
+    assert cq(s, *args2, 2, p, p, ws - 1, None) == moe.MOE_ERR_CAPACITY
+    assert cq(s, *args2, 2, p, p, ws, None) == moe.MOE_ERR_ARG  # ep_send_counts is NULL
     assert moe.moe_combine_bwd(s, None, p, None, p, p, None, p, p, None) == moe.MOE_ERR_ARG
     assert moe.moe_dispatch_bwd(s, p, None, None, p, None) == moe.MOE_ERR_ARG
     # special-expert backward: ori_x required; const tensors with const experts

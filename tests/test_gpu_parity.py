@@ -120,10 +120,12 @@ COMM_QUANT = [
 ]
 
 
+@pytest.mark.parametrize("use_ws", [True, False], ids=["two_pass", "single_pass"])
 @pytest.mark.parametrize("wl", COMM_QUANT, ids=lambda w: w.name)
-def test_combine_comm_quant_mode2(wl):
+def test_combine_comm_quant_mode2(wl, use_ws):
     """Combine with comm_quant_mode 2 (per-row int8 round trip of the returning
-    rows) against the oracle on the same expert outputs."""
+    rows) against the oracle on the same expert outputs, with and without the
+    workspace (two-pass kernels where the shape allows, else the single pass)."""
     import gpu_chain
     import oracle
     import combine_moe_dispatch_04_b200 as moe
@@ -150,7 +152,7 @@ def test_combine_comm_quant_mode2(wl):
                           x_active_mask=dev(inp["mask"]), shared_expert_x=dev(inp["shared"], dt),
                           ori_x=dev(inp["ori_x"], dt), const_alpha_1=dev(inp["alpha1"], dt),
                           const_alpha_2=dev(inp["alpha2"], dt), const_v=dev(inp["v"], dt),
-                          comm_quant_mode=2)
+                          comm_quant_mode=2, use_workspace=use_ws)
     torch.cuda.synchronize()
     got = gpu_chain.host(out)
     d = gpu_chain.ulp_dist(got, want)
@@ -159,8 +161,9 @@ def test_combine_comm_quant_mode2(wl):
     assert moe.moe_async_wait_timeouts() == 0  # no staged copy was given up on
 
 
+@pytest.mark.parametrize("use_ws", [True, False], ids=["two_pass", "single_pass"])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
-def test_combine_q8_rounding_ties(dtype):
+def test_combine_q8_rounding_ties(dtype, use_ws):
     """Returning rows whose values sit exactly on, or one 16-bit step beside,
     half-integer multiples of their scale: the combine round trip must match the
     oracle's IEEE division and rounding bit for bit."""
@@ -188,7 +191,7 @@ def test_combine_q8_rounding_ties(dtype):
     dev = gpu_chain.dev
     lay = moe.dispatch_layout(sh, dev(inp["topk_idx"]))
     out = moe.combine_fwd(sh, dev(y, dtype), dev(inp["topk_idx"]), dev(inp["topk_weights"]), lay,
-                          comm_quant_mode=2)
+                          comm_quant_mode=2, use_workspace=use_ws)
     torch.cuda.synchronize()
     assert np.array_equal(gpu_chain.host(out), want)
 
