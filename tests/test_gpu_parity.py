@@ -116,6 +116,11 @@ COMM_QUANT = [
             const_expert_num=2, backward=False),
     _custom("zero_only_q8", bs=900, k=4, num_experts=16, zero_expert_num=3, h=256,
             backward=False),
+    # routed pairs only: every K bucket of the two-pass gather, and rows too narrow for it
+    _custom("k4_routed_q8", bs=700, k=4, num_experts=16, h=520, backward=False),
+    _custom("k16_routed_q8", bs=600, k=16, num_experts=40, h=264, dtype="fp16",
+            mask_ndim=2, mask_false_p=0.2, backward=False),
+    _custom("k8_narrow_q8", bs=500, k=8, num_experts=32, h=136, backward=False),
     W["special"],  # full size
 ]
 
