@@ -121,6 +121,9 @@ COMM_QUANT = [
     _custom("k16_routed_q8", bs=600, k=16, num_experts=40, h=264, dtype="fp16",
             mask_ndim=2, mask_false_p=0.2, backward=False),
     _custom("k8_narrow_q8", bs=500, k=8, num_experts=32, h=136, backward=False),
+    # special experts at H 3072: the single-pass kernel with two row buffers
+    _custom("k8_h3072_special_q8", bs=300, k=8, num_experts=16, zero_expert_num=1,
+            copy_expert_num=1, h=3072, backward=False),
     W["special"],  # full size
 ]
 
@@ -298,6 +301,7 @@ SMOOTH = [
     W["special"].scaled(bs=1500, h=528, mask_ndim=2, mask_false_p=0.2, name="special_mask"),
     W["dsv3"].scaled(bs=700, dtype="fp16", name="dsv3_fp16"),  # rows streamed twice
     _custom("smooth_h16384", bs=40, k=3, num_experts=5, h=16384, quant_mode=2),
+    _custom("smooth_h4096", bs=200, k=4, num_experts=8, h=4096, quant_mode=2),  # 4 warps
     _custom("smooth_h16_one_expert", bs=333, k=1, num_experts=1, h=16, quant_mode=2),
     _custom("smooth_empty", bs=0, quant_mode=2),
 ]
