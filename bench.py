@@ -10,9 +10,19 @@ untimed, and stay resident in HBM like every other input.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
 
-Prints one JSON line (rank 0). Multi-GPU runs are independent replicas (one process
-per GPU, launched with torch.distributed.run); only the barrier and the max-over-ranks
-timing use the process group.
+Prints one JSON line (rank 0): the headline workload (the largest single-GPU one,
+DeepSeek-V3-shaped, by default) with its roofline, end-to-end and CPU-baseline
+figures, plus a per-workload block timing all five workloads in the same process.
+
+Statistics follow the Megatron-LM MoE performance test's method: warm-up steps, then
+timed steps; the 3 slowest are dropped and the rest give the mean and standard
+deviation; a run is accepted when std/mean <= 2 %, and is repeated up to 5 times
+otherwise (the run with the smallest std/mean is kept and marked not accepted).
+
+Multi-GPU runs are independent replicas (one process per GPU, launched with
+torch.distributed.run). The process group is gloo on the host: only the barrier and
+the max over ranks of the timed duration cross ranks, and no collective touches
+device memory.
 """
 from __future__ import annotations
 
@@ -37,12 +47,17 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "dispatch+combine fwd+bwd tokens/s and achieved HBM GB/s (% of 8 TB/s), 1×B200"
-DEFAULT_WORKLOAD = "uniform_bs8192_h1536_k8_e64"
+# The largest configuration that fits one GPU: 2644 MB of algorithmic bytes per step.
+DEFAULT_WORKLOAD = "dsv3_bs4096_h7168_k8_e256"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 KERNELS = ("layout", "permute", "combine_fwd", "combine_bwd", "combine_bwd_special",
            "dispatch_bwd")
 DOM_EVERY = 4
+DROP_TOP = 3          # slowest steps dropped before the mean and std
+ACCEPT_CV = 0.02      # std / mean at or below which a run is accepted
+MAX_RUNS = 5          # runs of one workload before the best one is kept
+TARGET_FRAC_OF_8TBS = 0.70
 
 
 # ---------------------------------------------------------------------------
@@ -79,15 +94,17 @@ def byte_model(wl: workloads.Workload, r: int, ori_tokens: int) -> dict:
 
 
 # ---------------------------------------------------------------------------
-# Replicas: only the timing is reduced across ranks (max), never data.
+# Replicas: only the timing is reduced across ranks (max), never data. The group is
+# gloo, so the reduction runs on the host.
 
 def reduce_max(value: float, device=None) -> float:
     import torch
     import torch.distributed as dist
 
+    del device  # the reduction runs on a host tensor (gloo)
     if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device=device)
+    t = torch.tensor([value], dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -96,6 +113,18 @@ def whole_job_throughput(tokens_per_rank_step: int, steps: int, world: int,
                          max_total_ms: float) -> float:
     """Tokens of all replicas divided by the slowest replica's time."""
     return tokens_per_rank_step * steps * world / (max_total_ms * 1e-3)
+
+
+def trimmed_stats(step_ms: list, drop: int = DROP_TOP) -> dict:
+    """Mean and population std of the step times without the `drop` slowest (all of
+    them when there are too few steps to drop any)."""
+    kept = sorted(step_ms)[:-drop] if len(step_ms) > 2 * drop else list(step_ms)
+    mean = statistics.fmean(kept)
+    std = statistics.pstdev(kept) if len(kept) > 1 else 0.0
+    return {"mean": mean, "std": std, "cv": std / mean if mean > 0 else 0.0,
+            "kept": len(kept), "dropped": len(step_ms) - len(kept),
+            "plain_mean": statistics.fmean(step_ms), "median": statistics.median(step_ms),
+            "max": max(step_ms), "min": min(step_ms)}
 
 
 # ---------------------------------------------------------------------------
@@ -147,6 +176,7 @@ class ClockSampler:
             except ValueError:
                 continue
         os.unlink(self.path)
+        self.proc = None
         inside = [r for r in rows if t0 - 0.02 <= r[0] <= t1 + 0.02]
         window = "timed region"
         if not inside:  # timed region shorter than the sampling period
@@ -207,9 +237,12 @@ def profiled_traffic(kernel: str, workload: str):
     return ent.get("dram_bytes_per_launch")
 
 
+# ---------------------------------------------------------------------------
+# The CPU oracle as a timed baseline.
+
 def oracle_chain_timed(inputs: dict, sample_tokens: int) -> tuple[float, int]:
-    """Times the oracle's five calls on the first `sample_tokens` tokens of the
-    workload (expert stand-ins excluded). Returns (seconds, tokens)."""
+    """Times the oracle's calls on the first `sample_tokens` tokens of the workload
+    (expert stand-ins excluded). Returns (seconds, tokens)."""
     import oracle
 
     wl = inputs["workload"]
@@ -256,20 +289,39 @@ def oracle_chain_timed(inputs: dict, sample_tokens: int) -> tuple[float, int]:
     return secs, n
 
 
-def cpu_baseline(inputs: dict, budget_s: float = 10.0) -> dict:
-    wl = inputs["workload"]
-    sample = min(wl.bs, 2048)
+def _oracle_leg(inputs: dict, sample: int, budget_s: float) -> tuple[float, int, float, int]:
     total_s, total_tok, passes = 0.0, 0, 0
     while total_s < budget_s and passes < 50:
         s, n = oracle_chain_timed(inputs, sample)
         total_s += s
         total_tok += n
         passes += 1
-    return {"value": total_tok / total_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{passes} passes of the first {sample} tokens of {wl.name} through the "
-                      f"single-threaded C++ oracle (layout, permute, combine fwd"
-                      f"{', combine bwd, dispatch bwd' if wl.backward else ''}); "
-                      f"{total_s:.1f} s of CPU time"}
+    return total_tok / total_s, passes, total_s, total_tok
+
+
+def cpu_baseline(inputs: dict, budget_s: float = 10.0) -> dict:
+    """The oracle timed on this host: single-threaded (the pinned build, the
+    reported value) on a 2048-token sample, and its OpenMP build on all cores over
+    the whole batch."""
+    import oracle
+
+    wl = inputs["workload"]
+    sample = min(wl.bs, 2048)
+    value, passes, secs, _ = _oracle_leg(inputs, sample, budget_s)
+    steps_desc = (f"layout, permute, combine fwd"
+                  f"{', combine bwd, dispatch bwd' if wl.backward else ''}")
+    out = {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "sample": f"{passes} passes of the first {sample} tokens of {wl.name} through the "
+                     f"single-threaded C++ oracle ({steps_desc}); {secs:.1f} s of CPU time"}
+    nproc = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    with oracle.all_cores():
+        threads = oracle.num_threads()
+        v_all, p_all, s_all, _ = _oracle_leg(inputs, wl.bs, budget_s)
+    out["all_cores"] = {"value": v_all, "unit": "tokens/s", "cores": threads, "nproc": nproc,
+                        "kind": "oracle (OpenMP build, tokens split over threads)",
+                        "sample": f"{p_all} passes of all {wl.bs} tokens of {wl.name} "
+                                  f"({steps_desc}); {s_all:.1f} s wall"}
+    return out
 
 
 def run_reference(args, wl):
@@ -277,7 +329,9 @@ def run_reference(args, wl):
     if rank != 0:
         return 0
     inputs = workloads.generate(wl)
-    sample = min(wl.bs, 512)
+    # each step: a sample of tokens sized to about a quarter of a second of CPU work
+    probe_s, probe_n = oracle_chain_timed(inputs, 64)
+    sample = int(max(16, min(512, 0.25 / max(probe_s / probe_n, 1e-9))))
     for _ in range(args.warmup):
         oracle_chain_timed(inputs, sample)
     total_s, total_tok = 0.0, 0
@@ -288,7 +342,7 @@ def run_reference(args, wl):
     value = total_tok / total_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "ms_per_step": 1e3 * total_s / max(args.steps, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": wl.name, "bs": wl.bs, "h": wl.h, "k": wl.k,
                        "num_experts": wl.num_experts, "parallelism": "replicas"},
@@ -302,6 +356,311 @@ def run_reference(args, wl):
 
 
 # ---------------------------------------------------------------------------
+# One workload on the GPU: inputs resident in HBM, the path's calls, timing.
+
+class Bench:
+    """Builds one workload's resident inputs and the step's list of C-ABI calls."""
+
+    def __init__(self, wl, args, dev, rank):
+        import torch
+
+        import combine_moe_dispatch_04_b200 as moe
+
+        self.wl, self.args, self.dev = wl, args, dev
+        self.torch, self.moe = torch, moe
+        self.stream = torch.cuda.current_stream()
+        self.inputs = inputs = workloads.generate(wl, seed=wl.seed + 1000 * rank)
+        dt = wl.dtype
+        tdt = torch.bfloat16 if dt == "bf16" else torch.float16
+
+        def up(a):
+            if a is None:
+                return None
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:
+                return torch.from_numpy(a.view(np.int16)).to(dev).view(tdt)
+            return torch.from_numpy(a).to(dev)
+
+        def down16(t):
+            return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+        sh = moe.Shape(bs=wl.bs, k=wl.k, h=wl.h, num_experts=wl.num_experts,
+                       zero_expert_num=wl.zero_expert_num, copy_expert_num=wl.copy_expert_num,
+                       const_expert_num=wl.const_expert_num, a_capacity=wl.a_capacity,
+                       dtype=workloads.DTYPE_CODES[dt], mask_ndim=wl.mask_ndim)
+        d = {k: up(inputs[k]) for k in ("topk_idx", "topk_weights", "x", "mask", "shared",
+                                         "ori_x", "alpha1", "alpha2", "v", "grad_out",
+                                         "smooth")}
+        ws = moe.layout_workspace(sh, dev)
+        lay = moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws)
+        qm = wl.quant_mode
+        if wl.smooth:
+            expand, scales = moe.dispatch_permute_smooth(sh, d["x"], d["topk_idx"], lay,
+                                                         d["smooth"])
+        else:
+            expand, scales = moe.dispatch_permute(sh, d["x"], lay, qm)
+        torch.cuda.synchronize()
+        r = int(lay.ep_send_counts[-1].item())
+        # untimed expert stand-ins, computed once on the host from the GPU's dispatch output
+        if qm == 2:
+            y_host = workloads.expert_forward(inputs, expand.cpu().numpy(), scales.cpu().numpy())
+        else:
+            y_host = workloads.expert_forward(inputs, down16(expand))
+        y = up(y_host)
+        out = moe.combine_fwd(sh, y, d["topk_idx"], d["topk_weights"], lay,
+                              x_active_mask=d["mask"], shared_expert_x=d["shared"],
+                              ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
+                              const_alpha_2=d["alpha2"], const_v=d["v"])
+        gexp = gw = gin = gx = None
+        if wl.backward:
+            gexp, gw = moe.combine_bwd(sh, d["grad_out"], y, d["topk_weights"], lay,
+                                       x_active_mask=d["mask"])
+            torch.cuda.synchronize()
+            gin = up(workloads.expert_backward(inputs, down16(gexp)))
+            gx = moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"])
+        torch.cuda.synchronize()
+
+        ori_tokens = 0
+        if wl.copy_expert_num + wl.const_expert_num:
+            ids = inputs["topk_idx"]
+            lo = wl.num_experts + wl.zero_expert_num
+            ori_tokens = int(np.any(ids >= lo, axis=1).sum())
+        self.r = r
+        bytes_per = byte_model(wl, r, ori_tokens)
+        kernels = [k for k in KERNELS if k in bytes_per]
+        sp_ws = sp_out = None
+        if "combine_bwd_special" in bytes_per:
+            n_ws = moe.moe_combine_bwd_special_workspace_bytes(ctypes.byref(sh.c()))
+            sp_ws = torch.empty(max(n_ws, 16), dtype=torch.uint8, device=dev) if n_ws else None
+            _, *sp_out = moe.combine_bwd_special(
+                sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
+                x_active_mask=d["mask"], const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
+                const_v=d["v"], grad_w=gw, workspace=sp_ws)
+            torch.cuda.synchronize()
+
+        # the step's results the caller reads back (swapped per slot by the e2e loop)
+        o = {"out": out}
+        if wl.backward:
+            o.update(gw=gw, gx=gx)
+        cq = args.combine_comm_quant
+        q8_ws = None
+        if cq == 2:  # the int8 combine's workspace, allocated once outside the timed steps
+            nb = moe.moe_combine_fwd_comm_quant_workspace_bytes(ctypes.byref(sh.c()))
+            q8_ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        special_ids = wl.zero_expert_num + wl.copy_expert_num + wl.const_expert_num
+        self.q8_two_pass = (cq == 2 and special_ids == 0 and
+                            wl.h // 8 >= 32 * (4 if wl.k <= 2 else 2 if wl.k <= 4 else 1))
+        # the profiled kernel differs with the combine's quantisation mode
+        self.traffic_key = wl.name + ("+comm_quant2" if cq == 2 else "")
+        fused = args.fused_dispatch
+        if fused:
+            calls = [("dispatch", lambda st: moe.dispatch(
+                sh, d["topk_idx"], d["x"], x_active_mask=d["mask"], comm_quant_mode=qm,
+                workspace=ws, layout=lay, expand_x=expand, dynamic_scales=scales, stream=st))]
+            bytes_per["dispatch"] = bytes_per.pop("layout") + bytes_per.pop("permute")
+            kernels = ["dispatch"] + [k for k in kernels if k not in ("layout", "permute")]
+        else:
+            calls = [
+                ("layout", lambda st: moe.dispatch_layout(sh, d["topk_idx"], d["mask"],
+                                                       workspace=ws, out=lay, stream=st)),
+                ("permute", lambda st: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
+                                                         dynamic_scales=scales, stream=st)),
+            ]
+            if wl.smooth:
+                calls[1] = ("permute", lambda st: moe.dispatch_permute_smooth(
+                    sh, d["x"], d["topk_idx"], lay, d["smooth"], expand_x=expand,
+                    dynamic_scales=scales, stream=st))
+        calls += [
+            ("combine_fwd", lambda st: moe.combine_fwd(
+                sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
+                shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
+                const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, workspace=q8_ws,
+                out=o["out"], stream=st)),
+        ]
+        if wl.backward:
+            calls += [
+                ("combine_bwd", lambda st: moe.combine_bwd(
+                    sh, d["grad_out"], y, d["topk_weights"], lay, x_active_mask=d["mask"],
+                    grad_expand=gexp, grad_w=o["gw"], stream=st)),
+            ]
+            if "combine_bwd_special" in bytes_per:
+                calls += [("combine_bwd_special", lambda st: moe.combine_bwd_special(
+                    sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
+                    x_active_mask=d["mask"], const_alpha_1=d["alpha1"],
+                    const_alpha_2=d["alpha2"], const_v=d["v"], grad_w=o["gw"],
+                    workspace=sp_ws, out=sp_out, stream=st))]
+            calls += [
+                ("dispatch_bwd", lambda st: moe.dispatch_bwd(sh, gin, lay,
+                                                          x_active_mask=d["mask"],
+                                                          grad_x=o["gx"], stream=st)),
+            ]
+        self.d, self.o, self.calls = d, o, calls
+        self.bytes_per, self.kernels = bytes_per, kernels
+        # the kernel that moves the most bytes; the timed steps bracket it with events
+        self.dominant = max((k for k in kernels if k not in ("layout", "dispatch")),
+                            key=lambda k: bytes_per[k])
+        tiled = wl.bs > moe_layout_small_max_tokens()
+        if fused and not tiled and qm == 0:
+            dispatch_launches = 1
+        else:
+            dispatch_launches = (2 if tiled else 1) + 1
+        special_bwd_launches = 0
+        if "combine_bwd_special" in bytes_per:
+            special_bwd_launches = 1 + (2 if wl.const_expert_num else 0)
+        self.launches_per_step = (dispatch_launches + (2 if self.q8_two_pass else 1)
+                                  + (2 if wl.backward else 0) + special_bwd_launches)
+        self.use_graph = not args.no_graph
+        self.plain_graph = self.capture() if self.use_graph else None
+
+    # ---- launching
+
+    def run_calls(self, st, marks=None):
+        for name, fn in self.calls:
+            if marks is not None and name in marks:
+                marks[name][0].record(st)
+            fn(st)
+            if marks is not None and name in marks:
+                marks[name][1].record(st)
+
+    def new_marks(self, names, external=False):
+        torch = self.torch
+        ev = lambda: torch.cuda.Event(enable_timing=True, external=external)  # noqa: E731
+        m = {"start": ev(), "end": ev()}
+        for n_ in names:
+            m[n_] = (ev(), ev())
+        return m
+
+    def capture(self, marks=None):
+        """A CUDA graph of the step's launches (programmatic-launch edges kept), with
+        event-record nodes around the kernels named in `marks`."""
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run_calls(torch.cuda.current_stream(), marks)
+        return g
+
+    def step(self, marks=None, graph=None):
+        """One pass of the path. `marks` maps "start"/"end" to an event and kernel
+        names to (before, after) event pairs; kernels without events keep their
+        programmatic-launch overlap with their neighbours. With `graph`, the pass
+        is that captured graph (whose own events are already inside)."""
+        if marks is not None:
+            marks["start"].record(self.stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            self.run_calls(self.stream, marks)
+        if marks is not None:
+            marks["end"].record(self.stream)
+
+    # ---- timing
+
+    def timed_run(self, steps, warmup, flush_l2, world, sampler=None):
+        """W warm-up steps, then `steps` timed steps (an L2 flush before each, outside
+        the step's events). Every DOM_EVERY-th step also brackets the dominant kernel
+        with events (an event between two kernels costs both their launch overlap, so
+        the other steps carry only the step's own start/end events)."""
+        import torch.distributed as dist
+        torch = self.torch
+        dom = self.dominant
+        for _ in range(warmup):
+            flush_l2()
+            self.step(graph=self.plain_graph)
+        torch.cuda.synchronize()
+        sampled = [i % DOM_EVERY == DOM_EVERY - 1 for i in range(steps)]
+        marks, graphs = [], []
+        for i in range(steps):
+            m = self.new_marks([])
+            if sampled[i]:
+                inner = self.new_marks([dom], external=self.use_graph)
+                m[dom] = inner[dom]
+                graphs.append(self.capture({dom: inner[dom]}) if self.use_graph else None)
+            else:
+                graphs.append(self.plain_graph)
+            marks.append(m)
+        if self.use_graph:
+            for g in {id(g): g for g in graphs}.values():  # warm every graph once
+                flush_l2()
+                self.step(graph=g)
+            torch.cuda.synchronize()
+        if sampler is not None:
+            sampler.start()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.time()
+        for i in range(steps):
+            flush_l2()
+            if self.use_graph:
+                self.step({"start": marks[i]["start"], "end": marks[i]["end"]}, graph=graphs[i])
+            else:
+                self.step(marks[i] if sampled[i] else
+                          {"start": marks[i]["start"], "end": marks[i]["end"]})
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t1 = time.time()
+        clocks = sampler.stop(t0, t1) if sampler is not None else None
+        step_ms = [m["start"].elapsed_time(m["end"]) for m in marks]
+        dom_ms = [m[dom][0].elapsed_time(m[dom][1]) for m in marks if dom in m]
+        del graphs
+        return step_ms, dom_ms, clocks
+
+    def accepted_run(self, steps, warmup, flush_l2, world, rank, uuid):
+        """Runs until std/mean of the kept steps is at most ACCEPT_CV (max over ranks),
+        at most MAX_RUNS times; returns the run with the smallest std/mean."""
+        best = None
+        runs = 0
+        for _ in range(MAX_RUNS):
+            sampler = ClockSampler(uuid) if rank == 0 else None
+            step_ms, dom_ms, clocks = self.timed_run(steps, warmup, flush_l2, world, sampler)
+            runs += 1
+            st = trimmed_stats(step_ms)
+            cv = reduce_max(st["cv"])
+            mean = reduce_max(st["mean"])
+            if best is None or cv < best["cv"]:
+                best = {"cv": cv, "mean_ms": mean, "stats": st, "step_ms": step_ms,
+                        "dom_ms": dom_ms, "clocks": clocks}
+            if cv <= ACCEPT_CV:
+                break
+        best["runs"] = runs
+        best["accepted"] = best["cv"] <= ACCEPT_CV
+        return best
+
+    def kernel_diagnostic(self, flush_l2, n):
+        """Separate untimed steps with events around every kernel (each loses its
+        launch overlap): per-kernel means in microseconds."""
+        torch = self.torch
+        diag = [self.new_marks(self.kernels) for _ in range(n)]
+        for m in diag:
+            flush_l2()
+            self.step(m)
+        torch.cuda.synchronize()
+        return {k: 1e3 * statistics.fmean(m[k][0].elapsed_time(m[k][1]) for m in diag)
+                for k in self.kernels}
+
+    def summary(self, run, peak):
+        """Throughput and roofline figures of one accepted run."""
+        wl = self.wl
+        ms = run["mean_ms"]
+        bytes_step = sum(self.bytes_per.values())
+        gbs = bytes_step / (ms * 1e-3) / 1e9
+        dom = self.dominant
+        dom_us = 1e3 * statistics.fmean(run["dom_ms"]) if run["dom_ms"] else float("nan")
+        ach = self.bytes_per[dom] / (dom_us * 1e-6) / 1e9
+        return {
+            "ms_per_step": ms, "tokens_per_s": wl.bs / (ms * 1e-3),
+            "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+            "hbm_frac_of_measured": round(gbs / peak, 4),
+            "algorithmic_bytes_per_step": bytes_step,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(ach / peak, 4),
+                         "algorithmic_bytes": self.bytes_per[dom],
+                         "us_per_launch": round(dom_us, 3)},
+            "std_over_mean": round(run["cv"], 5), "accepted": run["accepted"],
+            "runs": run["runs"], "clocks": run["clocks"],
+        }
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -322,6 +681,9 @@ def main():
                     help="launch every step eagerly instead of replaying a CUDA graph of it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
+    ap.add_argument("--per-config-steps", type=int, default=100)
     args = ap.parse_args()
     wl = workloads.BY_NAME[args.workload]
     if args.with_backward and not wl.backward:
@@ -338,194 +700,19 @@ def main():
     import torch
     import torch.distributed as dist
 
-    import combine_moe_dispatch_04_b200 as moe
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        # replicas: a host-side group for the barrier and the timing max only
+        dist.init_process_group("gloo", timeout=_dt.timedelta(seconds=120))
     dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
 
-    inputs = workloads.generate(wl, seed=wl.seed + 1000 * rank)
-    dt = wl.dtype
-    tdt = torch.bfloat16 if dt == "bf16" else torch.float16
-
-    def up(a):
-        if a is None:
-            return None
-        a = np.ascontiguousarray(a)
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).to(dev).view(tdt)
-        return torch.from_numpy(a).to(dev)
-
-    def down16(t):
-        return t.cpu().view(torch.int16).numpy().view(np.uint16)
-
-    sh = moe.Shape(bs=wl.bs, k=wl.k, h=wl.h, num_experts=wl.num_experts,
-                   zero_expert_num=wl.zero_expert_num, copy_expert_num=wl.copy_expert_num,
-                   const_expert_num=wl.const_expert_num, a_capacity=wl.a_capacity,
-                   dtype=workloads.DTYPE_CODES[dt], mask_ndim=wl.mask_ndim)
-    d = {k: up(inputs[k]) for k in ("topk_idx", "topk_weights", "x", "mask", "shared", "ori_x",
-                                     "alpha1", "alpha2", "v", "grad_out", "smooth")}
-    ws = moe.layout_workspace(sh, dev)
-    lay = moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws)
-    qm = wl.quant_mode
-    if wl.smooth:
-        expand, scales = moe.dispatch_permute_smooth(sh, d["x"], d["topk_idx"], lay, d["smooth"])
-    else:
-        expand, scales = moe.dispatch_permute(sh, d["x"], lay, qm)
-    torch.cuda.synchronize()
-    r = int(lay.ep_send_counts[-1].item())
-    # untimed expert stand-ins, computed once on the host from the GPU's dispatch output
-    if qm == 2:
-        y_host = workloads.expert_forward(inputs, expand.cpu().numpy(), scales.cpu().numpy())
-    else:
-        y_host = workloads.expert_forward(inputs, down16(expand))
-    y = up(y_host)
-    out = moe.combine_fwd(sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
-                          shared_expert_x=d["shared"], ori_x=d["ori_x"],
-                          const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
-                          const_v=d["v"])
-    if wl.backward:
-        gexp, gw = moe.combine_bwd(sh, d["grad_out"], y, d["topk_weights"], lay,
-                                   x_active_mask=d["mask"])
-        torch.cuda.synchronize()
-        gin = up(workloads.expert_backward(inputs, down16(gexp)))
-        gx = moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"])
-    torch.cuda.synchronize()
-
-    ori_tokens = 0
-    if wl.copy_expert_num + wl.const_expert_num:
-        ids = inputs["topk_idx"]
-        lo = wl.num_experts + wl.zero_expert_num
-        ori_tokens = int(np.any(ids >= lo, axis=1).sum())
-    bytes_per = byte_model(wl, r, ori_tokens)
-    kernels = [k for k in KERNELS if k in bytes_per]
-    sp_ws = sp_out = None
-    if "combine_bwd_special" in bytes_per:
-        n_ws = moe.moe_combine_bwd_special_workspace_bytes(ctypes.byref(sh.c()))
-        sp_ws = torch.empty(max(n_ws, 16), dtype=torch.uint8, device=dev) if n_ws else None
-        _, *sp_out = moe.combine_bwd_special(
-            sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
-            x_active_mask=d["mask"], const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
-            const_v=d["v"], grad_w=gw, workspace=sp_ws)
-        torch.cuda.synchronize()
-
-    # the step's results the caller reads back (swapped per slot by the e2e loop)
-    o = {"out": out}
-    if wl.backward:
-        o.update(gw=gw, gx=gx)
-    cq = args.combine_comm_quant
-    q8_ws = None
-    if cq == 2:  # the int8 combine's workspace, allocated once outside the timed steps
-        nb = moe.moe_combine_fwd_comm_quant_workspace_bytes(ctypes.byref(sh.c()))
-        q8_ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
-    special_ids = wl.zero_expert_num + wl.copy_expert_num + wl.const_expert_num
-    q8_two_pass = (cq == 2 and special_ids == 0 and
-                   wl.h // 8 >= 32 * (4 if wl.k <= 2 else 2 if wl.k <= 4 else 1))
-    # the profiled kernel differs with the combine's quantisation mode
-    traffic_key = wl.name + ("+comm_quant2" if cq == 2 else "")
-    if args.fused_dispatch:
-        calls = [("dispatch", lambda st: moe.dispatch(
-            sh, d["topk_idx"], d["x"], x_active_mask=d["mask"], comm_quant_mode=qm,
-            workspace=ws, layout=lay, expand_x=expand, dynamic_scales=scales, stream=st))]
-        bytes_per["dispatch"] = bytes_per.pop("layout") + bytes_per.pop("permute")
-        kernels = ["dispatch"] + [k for k in kernels if k not in ("layout", "permute")]
-    else:
-        calls = [
-            ("layout", lambda st: moe.dispatch_layout(sh, d["topk_idx"], d["mask"], workspace=ws,
-                                                   out=lay, stream=st)),
-            ("permute", lambda st: moe.dispatch_permute(sh, d["x"], lay, qm, expand_x=expand,
-                                                     dynamic_scales=scales, stream=st)),
-        ]
-        if wl.smooth:
-            calls[1] = ("permute", lambda st: moe.dispatch_permute_smooth(
-                sh, d["x"], d["topk_idx"], lay, d["smooth"], expand_x=expand,
-                dynamic_scales=scales, stream=st))
-    calls += [
-        ("combine_fwd", lambda st: moe.combine_fwd(
-            sh, y, d["topk_idx"], d["topk_weights"], lay, x_active_mask=d["mask"],
-            shared_expert_x=d["shared"], ori_x=d["ori_x"], const_alpha_1=d["alpha1"],
-            const_alpha_2=d["alpha2"], const_v=d["v"], comm_quant_mode=cq, workspace=q8_ws,
-            out=o["out"], stream=st)),
-    ]
-    if wl.backward:
-        calls += [
-            ("combine_bwd", lambda st: moe.combine_bwd(
-                sh, d["grad_out"], y, d["topk_weights"], lay, x_active_mask=d["mask"],
-                grad_expand=gexp, grad_w=o["gw"], stream=st)),
-        ]
-        if "combine_bwd_special" in bytes_per:
-            calls += [("combine_bwd_special", lambda st: moe.combine_bwd_special(
-                sh, d["grad_out"], d["topk_idx"], d["topk_weights"], d["ori_x"],
-                x_active_mask=d["mask"], const_alpha_1=d["alpha1"], const_alpha_2=d["alpha2"],
-                const_v=d["v"], grad_w=o["gw"], workspace=sp_ws, out=sp_out, stream=st))]
-        calls += [
-            ("dispatch_bwd", lambda st: moe.dispatch_bwd(sh, gin, lay, x_active_mask=d["mask"],
-                                                      grad_x=o["gx"], stream=st)),
-        ]
-    # the kernel that moves the most bytes; the timed steps bracket it with events
-    dominant = max((k for k in kernels if k not in ("layout", "dispatch")),
-                   key=lambda k: bytes_per[k])
-
-    def run_calls(st, marks=None):
-        for name, fn in calls:
-            if marks is not None and name in marks:
-                marks[name][0].record(st)
-            fn(st)
-            if marks is not None and name in marks:
-                marks[name][1].record(st)
-
-    def new_marks(names, external=False):
-        ev = lambda: torch.cuda.Event(enable_timing=True, external=external)  # noqa: E731
-        m = {"start": ev(), "end": ev()}
-        for n_ in names:
-            m[n_] = (ev(), ev())
-        return m
-
-    # CUDA graphs of the step: one plain, and one per sampled step with timing
-    # events (graph event-record nodes) around the dominant kernel.
-    graphs = {}
-
-    def capture(marks=None):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            run_calls(torch.cuda.current_stream(), marks)
-        return g
-
-    def step(marks=None, graph=None):
-        """One pass of the path. `marks` maps "start"/"end" to an event and kernel
-        names to (before, after) event pairs; kernels without events keep their
-        programmatic-launch overlap with their neighbours. With `graph`, the
-        pass is that captured graph (whose own events are already inside)."""
-        if marks is not None:
-            marks["start"].record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            run_calls(stream, marks)
-        if marks is not None:
-            marks["end"].record(stream)
-
-    tiled = wl.bs > moe_layout_small_max_tokens()
-    if args.fused_dispatch and not tiled and qm == 0:
-        dispatch_launches = 1
-    else:
-        dispatch_launches = (2 if tiled else 1) + 1
-    special_bwd_launches = 0
-    if "combine_bwd_special" in bytes_per:
-        special_bwd_launches = 1 + (2 if wl.const_expert_num else 0)
-    launches_per_step = (dispatch_launches + (2 if q8_two_pass else 1) + (2 if wl.backward else 0)
-                         + special_bwd_launches)
-
-    # L2 flush between steps: write a buffer twice the size of L2, then read
-    # another one as large, so the step starts with none of its data in L2 and
-    # without the flush's dirty lines, whose write-back would otherwise be
-    # billed to the step. Both run before the step's start event.
+    # L2 flush between steps: write a buffer twice the size of L2, then read another
+    # one as large, so the step starts with none of its data in L2 and without the
+    # flush's dirty lines, whose write-back would otherwise be billed to the step.
+    # Both run before the step's start event.
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
     flush = torch.empty(2 * l2 // 4, dtype=torch.int32, device=dev)
     sweep = torch.zeros(2 * l2 // 4, dtype=torch.float32, device=dev)
@@ -535,74 +722,17 @@ def main():
         flush.zero_()
         torch.sum(sweep, dim=0, out=sweep_out)  # one reduction kernel
 
-    for _ in range(args.warmup):
-        flush_l2()
-        step()
-    torch.cuda.synchronize()
-
-    # Every DOM_EVERY-th timed step also brackets the dominant kernel with events
-    # (an event between two kernels costs both their launch overlap, so the
-    # other steps carry only the step's own start/end events).
-    sampled = [i % DOM_EVERY == DOM_EVERY - 1 for i in range(args.steps)]
-    use_graph = not args.no_graph
-    marks, step_graphs = [], []
-    if use_graph:
-        plain = capture()
-        for i in range(args.steps):
-            m = new_marks([])
-            if sampled[i]:
-                inner = new_marks([dominant], external=True)
-                m[dominant] = inner[dominant]
-                step_graphs.append(capture({dominant: inner[dominant]}))
-            else:
-                step_graphs.append(plain)
-            marks.append(m)
-        for _ in range(2):  # warm the graphs
-            flush_l2()
-            step(graph=plain)
-        torch.cuda.synchronize()
-    else:
-        marks = [new_marks([dominant] if sampled[i] else []) for i in range(args.steps)]
-        step_graphs = [None] * args.steps
-    uuid = None
     try:
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         uuid = None
-    sampler = ClockSampler(uuid if rank == 0 else None)
-    if rank == 0:
-        sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0 = time.time()
-    for i in range(args.steps):
-        flush_l2()
-        if step_graphs[i] is not None:
-            step({"start": marks[i]["start"], "end": marks[i]["end"]}, graph=step_graphs[i])
-        else:
-            step(marks[i])
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    t1 = time.time()
-    clocks = sampler.stop(t0, t1) if rank == 0 else None
+    peak, peak_kind = measured_hbm_peak()
 
-    step_ms = [m["start"].elapsed_time(m["end"]) for m in marks]
-    dom_ms = [m[dominant][0].elapsed_time(m[dominant][1]) for m in marks if dominant in m]
-    total_ms = reduce_max(float(sum(step_ms)), dev)
-    ms_per_step = total_ms / args.steps
-    value = whole_job_throughput(wl.bs, args.steps, world, total_ms)
-    bytes_step = sum(bytes_per.values())
-
-    # Per-kernel breakdown from separate diagnostic steps (not the timed ones):
-    # events around every kernel, which costs each kernel its launch overlap.
-    diag = [new_marks(kernels) for _ in range(min(args.steps, 20))]
-    for m in diag:
-        flush_l2()
-        step(m)
-    torch.cuda.synchronize()
-    per_kernel_ms = {k: [m[k][0].elapsed_time(m[k][1]) for m in diag] for k in kernels}
+    b = Bench(wl, args, dev, rank)
+    run = b.accepted_run(args.steps, args.warmup, flush_l2, world, rank, uuid)
+    ms_per_step = run["mean_ms"]
+    value = whole_job_throughput(wl.bs, 1, world, ms_per_step)
+    per_kernel_us = b.kernel_diagnostic(flush_l2, min(args.steps, 20))
 
     # e2e: pinned host inputs -> H2D -> the path through the C ABI -> D2H of the results,
     # every step. Inputs and results are double-buffered on the device: step i's
@@ -610,6 +740,7 @@ def main():
     # and step i's kernels, as a serving loop would run them.
     e2e = None
     if not args.no_e2e:
+        d, o, stream = b.d, b.o, b.stream
         in_keys = [k for k in ("topk_idx", "topk_weights", "x", "mask", "shared", "grad_out")
                    if d[k] is not None]
         h_in = {k: d[k].cpu().pin_memory() for k in in_keys}
@@ -641,7 +772,7 @@ def main():
             if uses_ori:
                 d["ori_x"] = din["x"]  # the token rows the copy/const experts return
             o.update(dout)
-            step()
+            b.step()
             e["done"].record(stream)
             with torch.cuda.stream(down_s):
                 down_s.wait_event(e["done"])
@@ -664,62 +795,102 @@ def main():
         stream.wait_stream(down_s)
         eb.record(stream)
         torch.cuda.synchronize()
-        e_ms = reduce_max(ea.elapsed_time(eb), dev)
+        e_ms = reduce_max(ea.elapsed_time(eb))
         e2e = {"value": whole_job_throughput(wl.bs, e2e_steps, world, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps,
                "note": "double-buffered: each step's uploads and read-back overlap the "
-                       "neighbouring steps' kernels on two copy streams"}
+                       "neighbouring steps' kernels on two copy streams; eager launches "
+                       "through the binding"}
+        # the timed graphs captured the original buffers: restore them
+        d.update(slots[0][0])
+        if uses_ori:
+            d["ori_x"] = slots[0][0]["x"]
+        o.update(slots[0][1])
+
+    head = b.summary(run, peak)
+    launches = b.launches_per_step
+    line_extra = {"dominant": b.dominant, "traffic_key": b.traffic_key, "r": b.r,
+                  "q8_two_pass": b.q8_two_pass, "kernels": b.kernels,
+                  "bytes_per": b.bytes_per, "use_graph": b.use_graph}
+    inputs_head = b.inputs
+    del b
+    torch.cuda.empty_cache()
+
+    # Every workload, same process and method (fewer steps), for the per-config block.
+    per_config = {}
+    if not args.no_per_config:
+        for w in workloads.WORKLOADS:
+            if w.name == wl.name and not (args.fused_dispatch or args.combine_comm_quant):
+                per_config[w.name] = {k: head[k] for k in (
+                    "ms_per_step", "tokens_per_s", "hbm_gbs", "hbm_frac_of_8tbs",
+                    "hbm_frac_of_measured", "roofline", "std_over_mean", "accepted", "runs",
+                    "clocks")}
+            else:
+                pc_args = argparse.Namespace(**vars(args))
+                pc_args.fused_dispatch = False
+                pc_args.combine_comm_quant = 0
+                bw = Bench(w, pc_args, dev, rank)
+                rw = bw.accepted_run(args.per_config_steps, args.warmup, flush_l2, world, rank,
+                                     uuid)
+                per_config[w.name] = bw.summary(rw, peak)
+                del bw
+                torch.cuda.empty_cache()
+            pc = per_config[w.name]
+            pc["meets_70pct_of_8tbs"] = (None if w.name.startswith("tiny")
+                                         else pc["hbm_frac_of_8tbs"] >= TARGET_FRAC_OF_8TBS)
 
     if rank == 0:
-        peak, peak_kind = measured_hbm_peak()
         kstats = {}
-        for k in kernels:
-            us = 1e3 * statistics.fmean(per_kernel_ms[k])
-            kstats[k] = {"us": round(us, 3), "bytes": bytes_per[k],
-                         "gbs": round(bytes_per[k] / (us * 1e-6) / 1e9, 1)}
-        dom = dominant
-        dom_us = 1e3 * statistics.fmean(dom_ms)
-        ach = round(bytes_per[dom] / (dom_us * 1e-6) / 1e9, 1)
-        gbs = bytes_step / (ms_per_step * 1e-3) / 1e9
+        for k in line_extra["kernels"]:
+            us = per_kernel_us[k]
+            kstats[k] = {"us": round(us, 3), "bytes": line_extra["bytes_per"][k],
+                         "gbs": round(line_extra["bytes_per"][k] / (us * 1e-6) / 1e9, 1)}
+        roof = dict(head["roofline"])
+        roof.update(peak_kind=peak_kind,
+                    traffic=profiled_traffic(line_extra["dominant"], line_extra["traffic_key"]),
+                    timed=f"CUDA events around this kernel in every {DOM_EVERY}th timed step "
+                          f"({len(run['dom_ms'])} launches)")
+        st = run["stats"]
+        cq = args.combine_comm_quant
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dt,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
             "data": "synthetic",
             "config": {"workload": wl.name, "bs": wl.bs, "h": wl.h, "k": wl.k,
-                       "num_experts": wl.num_experts, "routed_pairs": r,
+                       "num_experts": wl.num_experts, "routed_pairs": line_extra["r"],
                        "a_capacity": wl.a_capacity, "parallelism": "replicas",
                        "fused_dispatch": bool(args.fused_dispatch),
                        "smooth_quant": bool(wl.smooth),
                        "combine_comm_quant_mode": cq,
-                       "combine_int8_kernels": ("two-pass" if q8_two_pass else "single-pass")
-                                               if cq == 2 else None,
-                       "launch": "CUDA graph of the step" if use_graph else "eager launches",
-                       "l2": "flushed before every step (write of 2x L2, then a read of another 2x L2 so "
-                             "no dirty flush lines are written back inside the step), outside "
-                             "the step events"},
-            "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
-            "hbm_frac_of_measured": round(gbs / peak, 4),
-            "algorithmic_bytes_per_step": bytes_step,
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
-                         "traffic": profiled_traffic(dom, traffic_key),
-                         "algorithmic_bytes": bytes_per[dom], "us_per_launch": round(dom_us, 3),
-                         "timed": f"CUDA events around this kernel in every {DOM_EVERY}th timed "
-                                  f"step ({len(dom_ms)} launches)"},
+                       "combine_int8_kernels": ("two-pass" if line_extra["q8_two_pass"]
+                                                else "single-pass") if cq == 2 else None,
+                       "launch": ("CUDA graph of the step" if line_extra["use_graph"]
+                                  else "eager launches"),
+                       "l2": "flushed before every step (write of 2x L2, then a read of another "
+                             "2x L2 so no dirty flush lines are written back inside the step), "
+                             "outside the step events",
+                       "statistics": f"value and ms_per_step: mean of the timed steps without "
+                                     f"the {DROP_TOP} slowest, max over ranks; accepted when "
+                                     f"std/mean <= {ACCEPT_CV:.0%}, else rerun (at most "
+                                     f"{MAX_RUNS} runs, the steadiest kept)"},
+            "hbm_gbs": head["hbm_gbs"], "hbm_frac_of_8tbs": head["hbm_frac_of_8tbs"],
+            "hbm_frac_of_measured": head["hbm_frac_of_measured"],
+            "algorithmic_bytes_per_step": head["algorithmic_bytes_per_step"],
+            "roofline": roof,
             "kernels_diagnostic": {"note": "separate untimed steps with events around every "
                                            "kernel (no launch overlap)", **kstats},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches * args.steps,
             "e2e": e2e,
-            "clocks": clocks,
-            "step_ms_stats": {"mean": statistics.fmean(step_ms),
-                              "median": statistics.median(step_ms),
-                              "trimmed_mean_drop_top3": statistics.fmean(
-                                  sorted(step_ms)[:-3] if len(step_ms) > 6 else step_ms),
-                              "std": statistics.pstdev(step_ms)},
+            "clocks": run["clocks"],
+            "step_ms_stats": {"trimmed_mean_drop_top3": st["mean"], "std": st["std"],
+                              "std_over_mean": st["cv"], "plain_mean": st["plain_mean"],
+                              "median": st["median"], "min": st["min"], "max": st["max"],
+                              "runs": run["runs"], "accepted": run["accepted"]},
+            "per_config": per_config or None,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(inputs)
+            line["cpu_baseline"] = cpu_baseline(inputs_head)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

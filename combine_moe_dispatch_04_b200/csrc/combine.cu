@@ -9,6 +9,8 @@
 // (__fmul_rn / __fadd_rn: never contracted into an FMA), adds shared_expert_x
 // once, and narrows with round-to-nearest-even.
 
+#include <mutex>
+
 #include "async.cuh"
 #include "common.cuh"
 #include "launch.cuh"
@@ -19,9 +21,11 @@ namespace moe {
 __device__ unsigned g_wait_timeouts = 0;
 
 unsigned* wait_timeout_counter() {
+  static std::mutex mu;
   static unsigned* ptr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);  // host threads may make a device's first call together
   if (ptr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;

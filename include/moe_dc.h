@@ -227,10 +227,14 @@ moe_status moe_combine_fwd_comm_quant(const moe_shape* shape, const void* expand
  * moe_combine_fwd_comm_quant_ws — moe_combine_fwd_comm_quant with an optional
  * device workspace (same results, bit for bit). With a workspace of
  * moe_combine_fwd_comm_quant_workspace_bytes() bytes (16-byte aligned) and
- * mode 2, shapes without zero/copy/const experts run in two passes: each slot
- * row's scale and reciprocal into the workspace (one streaming read of the
- * rows, R = ep_send_counts[E] of them), then the weighted gather with the
- * round trip. Other shapes, or workspace NULL, take the single-pass kernel.
+ * mode 2, shapes without zero/copy/const experts whose rows are wide enough
+ * (H / 8 >= 32 * U, with U = 4, 2, 1 for K <= 2, K <= 4, K > 4) run in two
+ * passes: each slot row's scale and reciprocal into the workspace (one
+ * streaming read of the rows, R = ep_send_counts[E] of them), then the
+ * weighted gather with the round trip. Other shapes, or workspace NULL, take
+ * the one-pass int8 combine: a warp-specialised kernel that stages each
+ * token's rows in shared memory with bulk copies where its buffers fit, else a
+ * kernel that reads each token's rows twice through L1.
  *   workspace        NULL or device scratch; its contents on entry do not
  *                    matter (MOE_ERR_CAPACITY if smaller than required,
  *                    MOE_ERR_ALIGN if not 16-byte aligned)
@@ -319,8 +323,11 @@ moe_status moe_dispatch_bwd(const moe_shape* shape, const void* grad_expand_in,
  *
  * The call allocates nothing (no cudaMalloc, no cudaFree, no allocator of any
  * library). The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture. Every call shares the one array and
+ * (cudaGetSymbolAddress, with that device current) and caches it for the
+ * life of the process; make that first call before any stream capture. A
+ * device reset (cudaDeviceReset, or anything else that destroys the primary
+ * context) may move the array, so do not call this entry point in a process
+ * after resetting the device it runs on. Every call shares the one array and
  * leaves its contents behind; nothing in it needs clearing, because every
  * entry the layout reads is written earlier in the same call. Calls whose
  * work can overlap on the GPU (other streams, other threads) race on the

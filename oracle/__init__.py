@@ -7,6 +7,7 @@ All 16-bit tensors are numpy ``uint16`` bit patterns (bf16 or fp16, per ``dtype`
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -16,30 +17,57 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.cpp")
 LIB_PATH = os.path.join(_HERE, "liboracle.so")
+# The same source built with -fopenmp: the per-token loops run on all host cores
+# (results unchanged). Only the benchmark's all-cores CPU timing uses it; every
+# test of the oracle runs the plain single-threaded build above.
+LIB_OMP_PATH = os.path.join(_HERE, "liboracle_omp.so")
 DTYPE_CODES = {"bf16": 0, "fp16": 1}
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle with g++ (no FMA contraction, no fast-math)."""
-    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(_SRC):
+def build(force: bool = False, parallel: bool = False) -> str:
+    """Compile the oracle with g++ (no FMA contraction, no fast-math); with
+    parallel, the OpenMP build."""
+    path = LIB_OMP_PATH if parallel else LIB_PATH
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
         cmd = ["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math",
-               "-fPIC", "-shared", _SRC, "-o", LIB_PATH + ".tmp"]
+               "-fPIC", "-shared", *(["-fopenmp"] if parallel else []), _SRC,
+               "-o", path + ".tmp"]
         subprocess.check_call(cmd)
-        os.replace(LIB_PATH + ".tmp", LIB_PATH)
-    return LIB_PATH
+        os.replace(path + ".tmp", path)
+    return path
 
 
-_lib = None
+_libs: dict = {}
+_parallel = False
+
+
+@contextlib.contextmanager
+def all_cores():
+    """Within this block every oracle call runs the OpenMP build."""
+    global _parallel
+    prev, _parallel = _parallel, True
+    try:
+        yield
+    finally:
+        _parallel = prev
+
+
+def num_threads() -> int:
+    """Threads the active build runs its per-token loops on."""
+    return int(lib().oracle_num_threads())
 
 
 def lib():
-    global _lib
-    if _lib is None:
+    key = "omp" if _parallel else "plain"
+    if key not in _libs:
         # ORACLE_LIB lets the mutation tests load a deliberately broken copy.
-        path = os.environ.get("ORACLE_LIB") or build()
+        path = (build(parallel=True) if _parallel
+                else os.environ.get("ORACLE_LIB") or build())
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i = ctypes.c_int
+        L.oracle_num_threads.argtypes = []
+        L.oracle_num_threads.restype = i
         L.oracle_decode16.argtypes = [ctypes.c_uint16, i]
         L.oracle_decode16.restype = ctypes.c_float
         L.oracle_encode16.argtypes = [ctypes.c_float, i]
@@ -66,8 +94,8 @@ def lib():
         L.oracle_combine_bwd_special.restype = None
         L.oracle_dispatch_bwd.argtypes = [i, i, i, i, i, P, P, P, i, P]
         L.oracle_dispatch_bwd.restype = None
-        _lib = L
-    return _lib
+        _libs[key] = L
+    return _libs[key]
 
 
 def _p(a):

@@ -13,6 +13,11 @@
 //              with ep_size < 8": the fused EP MoE layer has a backward, which
 //              the combine backward below serves.
 //
+// Threads: built plain (the pinned build the tests check), every function is
+// single-threaded. Built with -fopenmp (the benchmark's all-cores CPU timing
+// only), the per-token loops that write disjoint outputs run their tokens on
+// all cores; each token's arithmetic, and so every result, is unchanged.
+//
 // Precision: the pages fix bf16/fp16 storage and fp32 topk_weights; the combine
 // accumulation is fp32, every product and every sum rounded on its own (this
 // file is compiled with -ffp-contract=off), in k order. grad_w is summed in
@@ -61,6 +66,10 @@
 #include <cstring>
 #include <algorithm>
 #include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 namespace {
 
@@ -163,6 +172,15 @@ void oracle_encode16_array(const float* f, uint16_t* b, long n, int dtype) {
   for (long i = 0; i < n; ++i) b[i] = store16(f[i], dtype);
 }
 
+// Threads the per-token loops use: 1 in the plain build.
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
 // Dispatch layout. [combine] Parameters (assist_info_for_combine,
 // ep_send_counts, x_active_mask), Constraints (A); readings R3, R5-R8, R10.
 // Returns the status bits found.
@@ -207,6 +225,7 @@ int oracle_dispatch_layout(int bs, int K, int num_experts, int n_ids, int a_capa
 void oracle_dispatch_permute(int bs, int K, int h, int a_capacity, const uint16_t* x,
                              const int32_t* assist_info, uint16_t* expand_x) {
   const size_t A = static_cast<size_t>(a_capacity);
+#pragma omp parallel for schedule(static)
   for (int t = 0; t < bs; ++t)
     for (int k = 0; k < K; ++k) {
       int32_t s = assist_info[A + static_cast<size_t>(t) * K + k];
@@ -223,8 +242,9 @@ void oracle_dispatch_permute_quant(int bs, int K, int h, int a_capacity, int dty
                                    int8_t* expand_q, float* dynamic_scales) {
   std::fesetround(FE_TONEAREST);
   const size_t A = static_cast<size_t>(a_capacity);
-  std::vector<int8_t> codes(h);
+#pragma omp parallel for schedule(static)
   for (int t = 0; t < bs; ++t) {
+    std::vector<int8_t> codes(h);
     const uint16_t* xr = x + static_cast<size_t>(t) * h;
     float amax = 0.0f;
     for (int j = 0; j < h; ++j) amax = std::max(amax, std::fabs(load16(xr, j, dtype)));
@@ -270,8 +290,9 @@ void oracle_dispatch_permute_quant_smooth(int bs, int K, int h, int a_capacity, 
                                           float* dynamic_scales) {
   std::fesetround(FE_TONEAREST);
   const size_t A = static_cast<size_t>(a_capacity);
-  std::vector<float> y(h);
+#pragma omp parallel for schedule(static)
   for (int t = 0; t < bs; ++t) {
+    std::vector<float> y(h);
     const uint16_t* xr = x + static_cast<size_t>(t) * h;
     for (int k = 0; k < K; ++k) {
       const int32_t s = assist_info[A + static_cast<size_t>(t) * K + k];
@@ -315,8 +336,9 @@ void oracle_combine_fwd(int bs, int K, int h, int num_experts, int zero_num, int
   const int n_ids = num_experts + zero_num + copy_num + const_num;
   const int zero_end = num_experts + zero_num;
   const int copy_end = zero_end + copy_num;
-  std::vector<float> amax(K);
+#pragma omp parallel for schedule(static)
   for (int t = 0; t < bs; ++t) {
+    std::vector<float> amax(K);
     const int32_t* row = topk_idx + static_cast<size_t>(t) * K;
     if (comm_quant_mode == 2)
       for (int k = 0; k < K; ++k) {
@@ -367,6 +389,7 @@ void oracle_combine_bwd(int bs, int K, int h, int a_capacity, int dtype,
                         const uint8_t* mask, int mask_ndim, uint16_t* grad_expand,
                         float* grad_w, double* abs_sum) {
   const size_t A = static_cast<size_t>(a_capacity);
+#pragma omp parallel for schedule(static)
   for (int t = 0; t < bs; ++t) {
     const uint16_t* g = grad_out + static_cast<size_t>(t) * h;
     for (int k = 0; k < K; ++k) {
@@ -485,6 +508,7 @@ void oracle_dispatch_bwd(int bs, int K, int h, int a_capacity, int dtype,
                          const uint16_t* grad_in, const int32_t* assist_info,
                          const uint8_t* mask, int mask_ndim, uint16_t* grad_x) {
   const size_t A = static_cast<size_t>(a_capacity);
+#pragma omp parallel for schedule(static)
   for (int t = 0; t < bs; ++t)
     for (int j = 0; j < h; ++j) {
       float acc = 0.0f;

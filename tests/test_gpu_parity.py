@@ -174,18 +174,26 @@ def test_combine_comm_quant_mode2(wl, use_ws):
 def test_combine_q8_rounding_ties(dtype, use_ws):
     """Returning rows whose values sit exactly on, or one 16-bit step beside,
     half-integer multiples of their scale: the combine round trip must match the
-    oracle's IEEE division and rounding bit for bit."""
+    oracle's IEEE division and rounding bit for bit. With the workspace the shape is
+    one the two-pass kernels take (routed pairs only, H / 8 >= 32 U); in bf16 some
+    rows have scales below 2^-100, which take the IEEE-division branch."""
     import gpu_chain
     import oracle
     import combine_moe_dispatch_04_b200 as moe
 
-    wl = _custom("q8_ties", bs=600, k=4, num_experts=8, h=256, backward=False, dtype=dtype)
+    k, h = (8, 256) if use_ws else (4, 256)
+    wl = _custom("q8_ties", bs=600, k=k, num_experts=16, h=h, backward=False, dtype=dtype)
+    u = 4 if k <= 2 else 2 if k <= 4 else 1
+    assert (h // 8 >= 32 * u) == use_ws  # the two-pass kernels' condition
     inp = workloads.generate(wl)
     _, send, assist, st = oracle.dispatch_layout(inp["topk_idx"], wl.num_experts, wl.n_ids,
                                                  wl.a_capacity)
     rng = np.random.default_rng(23)
     a_rows = wl.a_capacity
     c = 2.0 ** rng.integers(-6, 3, (a_rows, 1))
+    if dtype == "bf16":  # scales 2^-110 .. 2^-102: below the reciprocal's range
+        tiny = rng.random(a_rows) < 0.1
+        c[tiny, 0] = 2.0 ** rng.integers(-110, -101, int(tiny.sum()))
     ties = (rng.integers(-127, 127, (a_rows, wl.h)) + 0.5) * c
     ties[:, 0] = 127 * c[:, 0]  # the row max, so scale = c exactly
     y = workloads.encode16(ties, dtype)

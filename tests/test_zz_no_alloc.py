@@ -76,6 +76,15 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     limit = moe.moe_layout_noalloc_max_workspace_bytes()
     big = moe.Shape(bs=70000, k=16, h=1024, num_experts=1024)
     assert moe.moe_layout_workspace_bytes(ctypes.byref(big.c())) > limit
-    p = ctypes.c_void_p(256)
-    assert moe.moe_dispatch_layout_noalloc(ctypes.byref(big.c()), p, None, p, p, p, None,
-                                           None) == moe.MOE_ERR_CAPACITY
+    # real buffers of the shape's sizes: were the size check ever lost, the layout
+    # would run on valid memory and this assertion would fail, not the GPU
+    dev = torch.device("cuda", 0)
+    idx = torch.zeros((big.bs, big.k), dtype=torch.int32, device=dev)
+    out = _outputs(big, dev)
+    st = moe.moe_dispatch_layout_noalloc(
+        ctypes.byref(big.c()), idx.data_ptr(), None, out.expert_token_nums.data_ptr(),
+        out.ep_send_counts.data_ptr(), out.assist_info.data_ptr(), out.dev_status.data_ptr(),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == moe.MOE_ERR_CAPACITY
+    torch.cuda.synchronize()
+    assert int(out.ep_send_counts[0].item()) == -7  # nothing was written
