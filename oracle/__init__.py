@@ -89,6 +89,8 @@ def lib():
         L.oracle_combine_fwd.restype = None
         L.oracle_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, i, P, P, P]
         L.oracle_combine_bwd.restype = None
+        L.oracle_combine_bwd_comm_quant.argtypes = [i, i, i, i, i, P, P, P, P, P, i, P, P, P]
+        L.oracle_combine_bwd_comm_quant.restype = None
         L.oracle_combine_bwd_special.argtypes = [i, i, i, i, i, i, i, i, P, P, P, P, i, P, P, P,
                                                  P, P, P, P, P, P, P, P, P, P]
         L.oracle_combine_bwd_special.restype = None
@@ -199,10 +201,12 @@ def combine_fwd(expand_x, topk_idx, topk_weights, assist_info, *, num_experts, a
 
 
 def combine_bwd(grad_out, expand_x, topk_weights, assist_info, *, k, a_capacity, dtype,
-                mask=None):
+                mask=None, comm_quant_mode=0):
     """Returns (grad_expand (A, H), grad_w (BS, K) f32, abs_sum (BS, K) f64).
 
-    Rows of grad_expand without a slot are left zero.
+    Rows of grad_expand without a slot are left zero. With comm_quant_mode 2 the
+    backward of the int8 round-trip combine: grad_w against the round-trip values,
+    grad_expand straight through.
     """
     g = _c(grad_out, np.uint16)
     bs, h = g.shape
@@ -211,9 +215,9 @@ def combine_bwd(grad_out, expand_x, topk_weights, assist_info, *, k, a_capacity,
     ge = np.zeros((a_capacity, h), np.uint16)
     gw = np.zeros((bs, k), np.float32)
     mag = np.zeros((bs, k), np.float64)
-    lib().oracle_combine_bwd(bs, k, h, a_capacity, DTYPE_CODES[dtype], _p(g), _p(ex),
-                             _p(_c(topk_weights, np.float32)), _p(_c(assist_info, np.int32)),
-                             _p(m), 0 if m is None else m.ndim, _p(ge), _p(gw), _p(mag))
+    fn = lib().oracle_combine_bwd_comm_quant if comm_quant_mode == 2 else lib().oracle_combine_bwd
+    fn(bs, k, h, a_capacity, DTYPE_CODES[dtype], _p(g), _p(ex), _p(_c(topk_weights, np.float32)),
+       _p(_c(assist_info, np.int32)), _p(m), 0 if m is None else m.ndim, _p(ge), _p(gw), _p(mag))
     return ge, gw, mag
 
 

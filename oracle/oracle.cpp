@@ -59,6 +59,13 @@
 //      token is quantised as in R9 (per row, scale = max|y| / 127) and used as
 //      the fp32 value q * scale; special experts and shared_expert_x are local
 //      and are not quantised.
+//   R19 backward of combine with comm_quant_mode 2: the weighted sum uses the
+//      round-trip values D(y) = q * scale, so grad_w[t,k] = <grad_out[t],
+//      D(y_slot)> exactly; the round trip itself is piecewise constant and is
+//      passed straight through (its Jacobian taken as the identity), so
+//      grad_expand = round16(w * grad_out) as without quantisation. The same
+//      straight-through reading makes the dispatch-side int8 backward the plain
+//      dispatch backward.
 
 #include <cfenv>
 #include <cmath>
@@ -408,6 +415,47 @@ void oracle_combine_bwd(int bs, int K, int h, int a_capacity, int dtype,
         float gj = load16(g, j, dtype);
         ge[j] = store16(w * gj, dtype);
         double term = static_cast<double>(gj) * static_cast<double>(load16(xr, j, dtype));
+        dot += term;
+        mag += std::fabs(term);
+      }
+      grad_w[tk] = static_cast<float>(dot);
+      if (abs_sum) abs_sum[tk] = mag;
+    }
+  }
+}
+
+// Combine backward with comm_quant_mode 2 (reading R19; [combine] Parameters,
+// comm_quant_mode): as oracle_combine_bwd, but the dot product takes each
+// element of the returned row through the per-row int8 round trip (R15) the
+// forward applied; grad_expand passes the round trip straight through.
+void oracle_combine_bwd_comm_quant(int bs, int K, int h, int a_capacity, int dtype,
+                                   const uint16_t* grad_out, const uint16_t* expand_x,
+                                   const float* topk_weights, const int32_t* assist_info,
+                                   const uint8_t* mask, int mask_ndim, uint16_t* grad_expand,
+                                   float* grad_w, double* abs_sum) {
+  std::fesetround(FE_TONEAREST);
+  const size_t A = static_cast<size_t>(a_capacity);
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < bs; ++t) {
+    const uint16_t* g = grad_out + static_cast<size_t>(t) * h;
+    for (int k = 0; k < K; ++k) {
+      const size_t tk = static_cast<size_t>(t) * K + k;
+      const int32_t s = assist_info[A + tk];
+      if (s < 0 || !pair_active(mask, mask_ndim, t, k, K)) {
+        grad_w[tk] = 0.0f;
+        if (abs_sum) abs_sum[tk] = 0.0;
+        continue;
+      }
+      const float w = topk_weights[tk];
+      const uint16_t* yr = expand_x + static_cast<size_t>(s) * h;
+      uint16_t* ge = grad_expand + static_cast<size_t>(s) * h;
+      const float amax = row_amax(yr, h, dtype);
+      double dot = 0.0, mag = 0.0;
+      for (int j = 0; j < h; ++j) {
+        const float gj = load16(g, j, dtype);
+        ge[j] = store16(w * gj, dtype);
+        const float d = int8_roundtrip(load16(yr, j, dtype), amax);
+        const double term = static_cast<double>(gj) * static_cast<double>(d);
         dot += term;
         mag += std::fabs(term);
       }

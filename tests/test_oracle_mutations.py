@@ -12,7 +12,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.cpp")
 PIN_TESTS = ["tests/test_oracle_layout.py", "tests/test_oracle_quant.py",
-             "tests/test_oracle_combine.py", "tests/test_oracle_special_bwd.py"]
+             "tests/test_oracle_combine.py", "tests/test_oracle_special_bwd.py",
+             "tests/test_oracle_quant_bwd.py"]
 
 # (name, text in oracle.cpp, replacement)
 MUTATIONS = [
@@ -37,8 +38,8 @@ MUTATIONS = [
      "      for (int k = 0; k < K; ++k) {\n        if (pair_problem(row, k, n_ids)) continue;",
      "      for (int k = K - 1; k >= 0; --k) {\n        if (pair_problem(row, k, n_ids)) continue;"),
     ("grad_w_weighted",
-     "        dot += term;\n        mag += std::fabs(term);\n      }\n      grad_w[tk] = static_cast<float>(dot);\n      if (abs_sum) abs_sum[tk] = mag;\n    }\n  }\n}",
-     "        dot += w * term;\n        mag += std::fabs(term);\n      }\n      grad_w[tk] = static_cast<float>(dot);\n      if (abs_sum) abs_sum[tk] = mag;\n    }\n  }\n}"),
+     "static_cast<double>(load16(xr, j, dtype));\n        dot += term;",
+     "static_cast<double>(load16(xr, j, dtype));\n        dot += w * term;"),
     ("scan_off_by_one",
      "ep_send_counts[e + 1] = ep_send_counts[e] + expert_token_nums[e];",
      "ep_send_counts[e + 1] = ep_send_counts[e] + expert_token_nums[e] + (e == 0);"),
@@ -65,6 +66,11 @@ MUTATIONS = [
      "        amax = std::max(amax, std::fabs(load16(xr, j, dtype)));"),
     ("duplicate_ids_accepted",
      "    if (row[j] == id) return ST_DUP_ID;", "    if (false) return ST_DUP_ID;"),
+    ("quant_bwd_roundtrip_dropped",
+     "const float d = int8_roundtrip(load16(yr, j, dtype), amax);",
+     "const float d = load16(yr, j, dtype);"),
+    ("quant_bwd_scale_of_grad_row",
+     "const float amax = row_amax(yr, h, dtype);", "const float amax = row_amax(g, h, dtype);"),
 ]
 
 
