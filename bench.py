@@ -193,9 +193,13 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------
 
-def moe_layout_small_max_tokens() -> int:
-    """Largest BS the layout handles in one launch (one CTA); above it, two launches."""
-    return 1024
+def layout_launches(bs: int, num_experts: int) -> int:
+    """Launches of moe_dispatch_layout: one thread-block cluster for BS <= 16384 when
+    its lane masks fit in shared memory, else count, column scan and scatter."""
+    tpt = 1 if bs <= 8192 else 2
+    stride = num_experts | 1
+    smem = tpt * 32 * stride * 4 + (tpt * 32 * stride * 2 + 3) // 4 * 4 + num_experts * 8
+    return 1 if bs <= 16384 and smem <= 210 * 1024 else 3
 
 
 def measured_hbm_peak():
@@ -481,7 +485,7 @@ class Bench:
             calls += [
                 ("combine_bwd", lambda st: moe.combine_bwd(
                     sh, d["grad_out"], y, d["topk_weights"], lay, x_active_mask=d["mask"],
-                    grad_expand=gexp, grad_w=o["gw"], stream=st)),
+                    comm_quant_mode=cq, grad_expand=gexp, grad_w=o["gw"], stream=st)),
             ]
             if "combine_bwd_special" in bytes_per:
                 calls += [("combine_bwd_special", lambda st: moe.combine_bwd_special(
@@ -499,11 +503,10 @@ class Bench:
         # the kernel that moves the most bytes; the timed steps bracket it with events
         self.dominant = max((k for k in kernels if k not in ("layout", "dispatch")),
                             key=lambda k: bytes_per[k])
-        tiled = wl.bs > moe_layout_small_max_tokens()
-        if fused and not tiled and qm == 0:
+        if fused and wl.bs <= 1024 and qm == 0:
             dispatch_launches = 1
         else:
-            dispatch_launches = (2 if tiled else 1) + 1
+            dispatch_launches = layout_launches(wl.bs, wl.num_experts) + 1
         special_bwd_launches = 0
         if "combine_bwd_special" in bytes_per:
             special_bwd_launches = 1 + (2 if wl.const_expert_num else 0)

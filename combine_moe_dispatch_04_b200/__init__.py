@@ -29,7 +29,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
            "moe_combine_bwd_special_workspace_bytes", "moe_dispatch_permute_smooth",
            "moe_async_wait_timeouts", "moe_combine_fwd_comm_quant_ws",
-           "moe_combine_fwd_comm_quant_workspace_bytes")
+           "moe_combine_fwd_comm_quant_workspace_bytes", "moe_combine_bwd_comm_quant",
+           "moe_test_combine_fwd_wait_timeout", "moe_test_dispatch_permute_wait_timeout")
 
 
 class MoeShape(ctypes.Structure):
@@ -75,6 +76,11 @@ def _load():
     L.moe_combine_bwd_special_workspace_bytes.argtypes = [S]
     L.moe_combine_bwd_special_workspace_bytes.restype = ctypes.c_size_t
     L.moe_combine_bwd.argtypes = [S, P, P, P, P, P, P, P, P, P]
+    L.moe_combine_bwd_comm_quant.argtypes = [S, P, P, P, P, P, P, I, P, P, P]
+    U64 = ctypes.c_uint64
+    L.moe_test_combine_fwd_wait_timeout.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, U64, I,
+                                                    P]
+    L.moe_test_dispatch_permute_wait_timeout.argtypes = [S, P, P, P, U64, I, P]
     L.moe_dispatch_bwd.argtypes = [S, P, P, P, P, P]
     L.moe_dispatch_layout_noalloc.argtypes = [S, P, P, P, P, P, P, P]
     L.moe_layout_noalloc_max_workspace_bytes.argtypes = []
@@ -82,7 +88,9 @@ def _load():
     for n in ("moe_dispatch_layout", "moe_dispatch_permute", "moe_combine_fwd",
               "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
               "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
-              "moe_dispatch_permute_smooth", "moe_combine_fwd_comm_quant_ws"):
+              "moe_dispatch_permute_smooth", "moe_combine_fwd_comm_quant_ws",
+              "moe_combine_bwd_comm_quant", "moe_test_combine_fwd_wait_timeout",
+              "moe_test_dispatch_permute_wait_timeout"):
         getattr(L, n).restype = I
     return L
 
@@ -100,6 +108,9 @@ moe_dispatch_permute_smooth = _lib.moe_dispatch_permute_smooth
 moe_async_wait_timeouts = _lib.moe_async_wait_timeouts
 moe_combine_fwd = _lib.moe_combine_fwd
 moe_combine_bwd = _lib.moe_combine_bwd
+moe_combine_bwd_comm_quant = _lib.moe_combine_bwd_comm_quant
+moe_test_combine_fwd_wait_timeout = _lib.moe_test_combine_fwd_wait_timeout
+moe_test_dispatch_permute_wait_timeout = _lib.moe_test_dispatch_permute_wait_timeout
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
 moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
 moe_combine_fwd_comm_quant = _lib.moe_combine_fwd_comm_quant
@@ -313,8 +324,10 @@ def combine_fwd(shape: Shape, expand_x, topk_idx, topk_weights, layout: Layout, 
 
 
 def combine_bwd(shape: Shape, grad_out, expand_x, topk_weights, layout: Layout, *,
-                topk_idx=None, x_active_mask=None, grad_expand=None, grad_w=None, stream=None):
-    """Returns (grad_expand (A, H), grad_w (BS, K) fp32). Rows without a slot are not written."""
+                topk_idx=None, x_active_mask=None, comm_quant_mode=0, grad_expand=None,
+                grad_w=None, stream=None):
+    """Returns (grad_expand (A, H), grad_w (BS, K) fp32). Rows without a slot are not
+    written. comm_quant_mode 2: the backward of the int8 round-trip combine."""
     import torch
 
     if grad_expand is None:
@@ -322,10 +335,10 @@ def combine_bwd(shape: Shape, grad_out, expand_x, topk_weights, layout: Layout, 
                                   device=grad_out.device)
     if grad_w is None:
         grad_w = torch.empty(shape.bs, shape.k, dtype=torch.float32, device=grad_out.device)
-    _check("moe_combine_bwd", moe_combine_bwd(
+    _check("moe_combine_bwd_comm_quant", moe_combine_bwd_comm_quant(
         ctypes.byref(shape.c()), _ptr(grad_out), _ptr(expand_x), _ptr(topk_idx),
-        _ptr(topk_weights), _ptr(layout.assist_info), _ptr(x_active_mask), _ptr(grad_expand),
-        _ptr(grad_w), _stream(stream)))
+        _ptr(topk_weights), _ptr(layout.assist_info), _ptr(x_active_mask), comm_quant_mode,
+        _ptr(grad_expand), _ptr(grad_w), _stream(stream)))
     return grad_expand, grad_w
 
 

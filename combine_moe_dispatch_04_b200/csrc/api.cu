@@ -51,6 +51,54 @@ moe_status check_mask(const moe_shape* s, const uint8_t* mask) {
   return (s->bs > 0 && s->mask_ndim > 0 && mask == nullptr) ? MOE_ERR_ARG : MOE_OK;
 }
 
+// Checks of the combine forward's arguments, then its launch arguments.
+moe_status combine_args(const moe_shape* s, const void* expand_x, const int32_t* topk_idx,
+                        const float* topk_weights, const int32_t* assist_info,
+                        const uint8_t* x_active_mask, const void* shared_expert_x,
+                        const void* ori_x, const void* const_alpha_1, const void* const_alpha_2,
+                        const void* const_v, void* out, moe::CombineArgs* a) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if ((st = check_mask(s, x_active_mask)) != MOE_OK) return st;
+  const bool special = s->zero_expert_num + s->copy_expert_num + s->const_expert_num > 0;
+  if (s->bs > 0 && (expand_x == nullptr || topk_weights == nullptr || assist_info == nullptr ||
+                    out == nullptr || (special && topk_idx == nullptr)))
+    return MOE_ERR_ARG;
+  // [combine] Parameters: ori_x is required with copy or const experts, and
+  // the three const-expert tensors with const experts.
+  if (s->bs > 0 && (s->copy_expert_num > 0 || s->const_expert_num > 0) && ori_x == nullptr)
+    return MOE_ERR_ARG;
+  if (s->bs > 0 && s->const_expert_num > 0 &&
+      (const_alpha_1 == nullptr || const_alpha_2 == nullptr || const_v == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(expand_x) || !aligned16(out) || !aligned16(shared_expert_x) ||
+      !aligned16(ori_x) || !aligned16(const_alpha_1) || !aligned16(const_alpha_2) ||
+      !aligned16(const_v))
+    return MOE_ERR_ALIGN;
+  a->expand_x = expand_x;
+  a->topk_idx = topk_idx;
+  a->weights = topk_weights;
+  a->assist = assist_info;
+  a->mask = x_active_mask;
+  a->mask_ndim = s->mask_ndim;
+  a->shared = shared_expert_x;
+  a->ori_x = ori_x;
+  a->alpha1 = const_alpha_1;
+  a->alpha2 = const_alpha_2;
+  a->const_v = const_v;
+  a->out = out;
+  a->bs = s->bs;
+  a->K = s->k;
+  a->H = s->h;
+  a->A = s->a_capacity;
+  a->E = s->num_experts;
+  a->Z = s->zero_expert_num;
+  a->C = s->copy_expert_num;
+  a->Q = s->const_expert_num;
+  a->dtype = s->dtype;
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -254,61 +302,85 @@ moe_status moe_combine_fwd_comm_quant_ws(const moe_shape* s, const void* expand_
                                          const void* const_v, int comm_quant_mode, void* out,
                                          void* workspace, size_t workspace_bytes, void* stream) {
   if (comm_quant_mode != 0 && comm_quant_mode != 2) return MOE_ERR_ARG;
-  moe_status st = check_shape(s);
+  moe::CombineArgs a;
+  moe_status st = combine_args(s, expand_x, topk_idx, topk_weights, assist_info, x_active_mask,
+                               shared_expert_x, ori_x, const_alpha_1, const_alpha_2, const_v,
+                               out, &a);
   if (st != MOE_OK) return st;
-  if ((st = check_mask(s, x_active_mask)) != MOE_OK) return st;
-  const bool special = s->zero_expert_num + s->copy_expert_num + s->const_expert_num > 0;
-  if (s->bs > 0 && (expand_x == nullptr || topk_weights == nullptr || assist_info == nullptr ||
-                    out == nullptr || (special && topk_idx == nullptr)))
-    return MOE_ERR_ARG;
-  // [combine] Parameters: ori_x is required with copy or const experts, and
-  // the three const-expert tensors with const experts.
-  if (s->bs > 0 && (s->copy_expert_num > 0 || s->const_expert_num > 0) && ori_x == nullptr)
-    return MOE_ERR_ARG;
-  if (s->bs > 0 && s->const_expert_num > 0 &&
-      (const_alpha_1 == nullptr || const_alpha_2 == nullptr || const_v == nullptr))
-    return MOE_ERR_ARG;
-  if (!aligned16(expand_x) || !aligned16(out) || !aligned16(shared_expert_x) ||
-      !aligned16(ori_x) || !aligned16(const_alpha_1) || !aligned16(const_alpha_2) ||
-      !aligned16(const_v) || !aligned16(workspace))
-    return MOE_ERR_ALIGN;
+  if (!aligned16(workspace)) return MOE_ERR_ALIGN;
   if (workspace != nullptr &&
       workspace_bytes < moe::combine_q8_workspace_bytes(s->a_capacity > 0 ? s->a_capacity : 0))
     return MOE_ERR_CAPACITY;
   if (workspace != nullptr && s->bs > 0 && ep_send_counts == nullptr) return MOE_ERR_ARG;
-  moe::CombineArgs a;
-  a.expand_x = expand_x;
-  a.topk_idx = topk_idx;
-  a.weights = topk_weights;
-  a.assist = assist_info;
-  a.mask = x_active_mask;
-  a.mask_ndim = s->mask_ndim;
-  a.shared = shared_expert_x;
-  a.ori_x = ori_x;
-  a.alpha1 = const_alpha_1;
-  a.alpha2 = const_alpha_2;
-  a.const_v = const_v;
-  a.out = out;
-  a.bs = s->bs;
-  a.K = s->k;
-  a.H = s->h;
-  a.A = s->a_capacity;
-  a.E = s->num_experts;
-  a.Z = s->zero_expert_num;
-  a.C = s->copy_expert_num;
-  a.Q = s->const_expert_num;
-  a.dtype = s->dtype;
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
   return cuda_status(comm_quant_mode == 2
                          ? moe::launch_combine_fwd_q8(a, ep_send_counts, workspace, cs)
                          : moe::launch_combine_fwd(a, cs));
 }
 
+moe_status moe_test_combine_fwd_wait_timeout(const moe_shape* s, const void* expand_x,
+                                             const int32_t* topk_idx, const float* topk_weights,
+                                             const int32_t* assist_info,
+                                             const uint8_t* x_active_mask,
+                                             const void* shared_expert_x, const void* ori_x,
+                                             const void* const_alpha_1,
+                                             const void* const_alpha_2, const void* const_v,
+                                             void* out, uint64_t wait_limit_ns,
+                                             int withhold_unit, void* stream) {
+  moe::CombineArgs a;
+  moe_status st = combine_args(s, expand_x, topk_idx, topk_weights, assist_info, x_active_mask,
+                               shared_expert_x, ori_x, const_alpha_1, const_alpha_2, const_v,
+                               out, &a);
+  if (st != MOE_OK) return st;
+  if (withhold_unit < 0 || wait_limit_ns == 0 || wait_limit_ns > moe::kWaitLimitNs)
+    return MOE_ERR_ARG;
+  if (!moe::gather_staged_applies(a)) return MOE_ERR_UNSUPPORTED;
+  const moe::WaitCfg wc = {wait_limit_ns, withhold_unit};
+  return cuda_status(moe::launch_gather_staged(a, static_cast<cudaStream_t>(stream), wc));
+}
+
+moe_status moe_test_dispatch_permute_wait_timeout(const moe_shape* s, const void* x,
+                                                  const int32_t* assist_info, void* expand_x,
+                                                  uint64_t wait_limit_ns, int withhold_unit,
+                                                  void* stream) {
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (s->bs > 0 && (x == nullptr || assist_info == nullptr || expand_x == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(expand_x)) return MOE_ERR_ALIGN;
+  if (withhold_unit < 0 || wait_limit_ns == 0 || wait_limit_ns > moe::kWaitLimitNs)
+    return MOE_ERR_ARG;
+  if (s->bs == 0 || s->h / 8 < moe::kPermuteBulkMinVecs) return MOE_ERR_UNSUPPORTED;
+  moe::PermuteArgs a;
+  a.x = x;
+  a.assist = assist_info;
+  a.expand_x = expand_x;
+  a.scales = nullptr;
+  a.bs = s->bs;
+  a.K = s->k;
+  a.H = s->h;
+  a.A = s->a_capacity;
+  a.dtype = s->dtype;
+  a.quant_mode = 0;
+  const moe::WaitCfg wc = {wait_limit_ns, withhold_unit};
+  return cuda_status(moe::launch_permute_bulk(a, static_cast<cudaStream_t>(stream), wc));
+}
+
 moe_status moe_combine_bwd(const moe_shape* s, const void* grad_out, const void* expand_x,
                            const int32_t* topk_idx, const float* topk_weights,
                            const int32_t* assist_info, const uint8_t* x_active_mask,
                            void* grad_expand, float* grad_w, void* stream) {
+  return moe_combine_bwd_comm_quant(s, grad_out, expand_x, topk_idx, topk_weights, assist_info,
+                                    x_active_mask, 0, grad_expand, grad_w, stream);
+}
+
+moe_status moe_combine_bwd_comm_quant(const moe_shape* s, const void* grad_out,
+                                      const void* expand_x, const int32_t* topk_idx,
+                                      const float* topk_weights, const int32_t* assist_info,
+                                      const uint8_t* x_active_mask, int comm_quant_mode,
+                                      void* grad_expand, float* grad_w, void* stream) {
   (void)topk_idx;
+  if (comm_quant_mode != 0 && comm_quant_mode != 2) return MOE_ERR_ARG;
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
   if ((st = check_mask(s, x_active_mask)) != MOE_OK) return st;
@@ -331,6 +403,7 @@ moe_status moe_combine_bwd(const moe_shape* s, const void* grad_out, const void*
   a.H = s->h;
   a.A = s->a_capacity;
   a.dtype = s->dtype;
+  a.quant_mode = comm_quant_mode;
   return cuda_status(moe::launch_combine_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 

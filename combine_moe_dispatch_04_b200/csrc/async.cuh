@@ -1,5 +1,6 @@
-// Bulk asynchronous copies from global into shared memory, completed on an
-// mbarrier (PTX cp.async.bulk / mbarrier, sm_90 and later), and bounded waits.
+// Bulk asynchronous copies between global and shared memory (PTX
+// cp.async.bulk, sm_90 and later): global -> shared completed on an mbarrier,
+// shared -> global tracked by bulk async-groups; and bounded mbarrier waits.
 // Copies are plain (never multicast); both addresses 16-byte aligned and the
 // size a multiple of 16.
 #pragma once
@@ -84,17 +85,56 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Bulk copy of `bytes` from this CTA's shared memory to global memory, tracked
+// by this thread's bulk async-groups (plain, never multicast or reducing).
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_addr(src)), "r"(bytes)
+               : "memory");
+}
+
+// Closes this thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's bulk async-groups still read their
+// source (shared memory may then be reused)...
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// ... or are still in progress at all (their writes performed).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // A wait gives up after about this long (timed with the global nanosecond
 // timer, so the bound holds however long each suspended try lasts).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr uint32_t kWaitHintNs = 20000;
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity, kWaitHintNs)) return true;
   const uint64_t t0 = global_time_ns();
   while (!mbar_try_wait(bar, parity, kWaitHintNs))
-    if (global_time_ns() - t0 > kWaitLimitNs) return false;
+    if (global_time_ns() - t0 > limit_ns) return false;
   return true;
 }
+
+// Waits of a staged kernel: the limit of its pipeline waits, and a test hook
+// (off in every product call: withhold < 0) that makes the first CTA arm one
+// unit's "full" barrier for 16 bytes without starting any copy for it, so
+// that the waits on that unit run out while no copy is in flight for it. The
+// waits that let started copies land before a CTA leaves always use
+// kWaitLimitNs and skip the withheld unit.
+struct WaitCfg {
+  uint64_t limit_ns;
+  int withhold;
+};
+constexpr WaitCfg kProductWaits = {kWaitLimitNs, -1};
 
 }  // namespace moe

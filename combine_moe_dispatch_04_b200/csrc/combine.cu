@@ -770,6 +770,7 @@ cudaError_t launch_fwd_rt(const CombineArgs& a, const int32_t* send, float2* rsc
 
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
+  if (gather_staged_applies(a)) return launch_gather_staged(a, st);
   return a.dtype == MOE_BF16 ? launch_fwd_t<Bf16>(a, st) : launch_fwd_t<Fp16>(a, st);
 }
 

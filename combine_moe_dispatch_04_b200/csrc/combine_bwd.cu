@@ -1,6 +1,7 @@
-// Combine backward: the gradient of the combine Formula for routed pairs.
-// [combine] Function (Formula); the fused EP MoE layer of the Triton-distributed
-// ep_moe_fused PR has a backward.
+// Combine backward: the gradient of the combine Formula for routed pairs, and
+// of the combine with comm_quant_mode 2. [combine] Function (Formula),
+// Parameters (comm_quant_mode); the fused EP MoE layer of the
+// Triton-distributed ep_moe_fused PR has a backward.
 //
 // One warp per (token, k) pair on a persistent grid; the warp streams the
 // pair's expand_x row against grad_out[t] (the K warps of a token share
@@ -17,7 +18,12 @@ constexpr int kBwdThreads = 256;
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kBwdUnroll = 4;
 
-template <typename T16>
+// Q8: the backward of the combine with comm_quant_mode 2 (straight-through):
+// grad_w takes the dot of grad_out with the row's int8 round-trip values
+// fl(q * scale), scale = fl(max|y| / 127), the codes decided exactly as in
+// the forward; grad_expand is unchanged. The row is read twice through L1:
+// once for its max, once for the dot.
+template <typename T16, bool Q8>
 __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pair, int lane) {
   const int t = pair / a.K;
   const int k = pair - t * a.K;
@@ -31,6 +37,17 @@ __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pa
   const uint4* g = static_cast<const uint4*>(a.grad_out) + static_cast<size_t>(t) * V;
   const uint4* y = static_cast<const uint4*>(a.expand_x) + static_cast<size_t>(s) * V;
   uint4* ge = static_cast<uint4*>(a.grad_expand) + static_cast<size_t>(s) * V;
+  float mx = 0.0f, scale = 0.0f, inv = 0.0f;
+  if (Q8) {
+    uint32_t m2 = 0;
+#pragma unroll 4
+    for (int v = lane; v < V; v += 32) m2 = absmax_v4<T16>(m2, __ldg(y + v));
+    mx = absmax_final<T16>(m2);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    scale = __fdiv_rn(mx, 127.0f);
+    inv = 1.0f / scale;
+  }
   float d[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) d[i] = 0.0f;
@@ -41,7 +58,7 @@ __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pa
       const int v = v0 + u * 32;
       if (v < V) {
         gv[u] = __ldg(g + v);  // kept in L1: the other K-1 warps of the token re-read it
-        yv[u] = ld_nc_v4(y + v);
+        yv[u] = Q8 ? __ldg(y + v) : ld_nc_v4(y + v);
       }
     }
 #pragma unroll
@@ -50,7 +67,13 @@ __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pa
       if (v >= V) continue;
       float gf[8], yf[8], o[8];
       widen8<T16>(gv[u], gf);
-      widen8<T16>(yv[u], yf);
+      if (Q8) {
+        float yr[8];
+        widen8<T16>(yv[u], yr);
+        quant_roundtrip8<true>(yr, mx, scale, inv, yf);
+      } else {
+        widen8<T16>(yv[u], yf);
+      }
       const float2 ww = f2(w, w);
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
@@ -71,7 +94,7 @@ __device__ __forceinline__ void combine_bwd_pair(const CombineBwdArgs& a, int pa
   if (lane == 0) a.grad_w[pair] = dot;
 }
 
-template <typename T16>
+template <typename T16, bool Q8>
 __global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(CombineBwdArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -79,21 +102,26 @@ __global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(CombineBwdArgs
   const int n_pairs = a.bs * a.K;
   const int stride = gridDim.x * kBwdWarps;
   for (int pair = blockIdx.x * kBwdWarps + (threadIdx.x >> 5); pair < n_pairs; pair += stride)
-    combine_bwd_pair<T16>(a, pair, lane);
+    combine_bwd_pair<T16, Q8>(a, pair, lane);
+}
+
+template <typename T16, bool Q8>
+cudaError_t launch_bwd(const CombineBwdArgs& a, cudaStream_t st) {
+  constexpr auto kernel = combine_bwd_kernel<T16, Q8>;
+  const long long pairs = static_cast<long long>(a.bs) * a.K;
+  const long long want = (pairs + kBwdWarps - 1) / kBwdWarps;
+  const long long cap = static_cast<long long>(sm_count()) * blocks_per_sm<kernel>(kBwdThreads, 0);
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(kernel, dim3(blocks), dim3(kBwdThreads), 0, st, a);
 }
 
 }  // namespace
 
 cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
-  auto kernel = a.dtype == MOE_BF16 ? combine_bwd_kernel<Bf16> : combine_bwd_kernel<Fp16>;
-  const long long pairs = static_cast<long long>(a.bs) * a.K;
-  const long long want = (pairs + kBwdWarps - 1) / kBwdWarps;
-  const long long cap = static_cast<long long>(sm_count()) *
-                        (a.dtype == MOE_BF16 ? blocks_per_sm<combine_bwd_kernel<Bf16>>(kBwdThreads, 0)
-                                             : blocks_per_sm<combine_bwd_kernel<Fp16>>(kBwdThreads, 0));
-  const int blocks = static_cast<int>(want < cap ? want : cap);
-  return launch_pdl(kernel, dim3(blocks), dim3(kBwdThreads), 0, st, a);
+  if (a.quant_mode == 2)
+    return a.dtype == MOE_BF16 ? launch_bwd<Bf16, true>(a, st) : launch_bwd<Fp16, true>(a, st);
+  return a.dtype == MOE_BF16 ? launch_bwd<Bf16, false>(a, st) : launch_bwd<Fp16, false>(a, st);
 }
 
 }  // namespace moe

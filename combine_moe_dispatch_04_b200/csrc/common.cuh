@@ -290,12 +290,14 @@ __device__ __forceinline__ uint4 pack_codes16(const float (&y)[16], float amax, 
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Eight int8 codes (element i in byte i) of one 16-byte vector of a row.
+// Eight int8 codes (element i in byte i) of one 16-byte vector of a row (the
+// rare tie decisions as an out-of-line call with OUTLINE).
+template <bool OUTLINE = false>
 __device__ __forceinline__ uint2 pack_codes8(const float (&y)[8], float amax, float scale,
                                              float inv_scale) {
   if (amax == 0.0f) return make_uint2(0u, 0u);
   float n[8], b[8];
-  quant_codes8(y, scale, inv_scale, scale >= kFastMinScale, n, b);
+  quant_codes8<OUTLINE>(y, scale, inv_scale, scale >= kFastMinScale, n, b);
   uint32_t w[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {

@@ -5,6 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "async.cuh"
 #include "moe_dc.h"
 
 namespace moe {
@@ -36,6 +37,14 @@ struct PermuteArgs {
   int bs, K, H, A, dtype, quant_mode;
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
+// The bulk-copy permute (plain copy) with the given waits (test hook).
+cudaError_t launch_permute_bulk(const PermuteArgs& a, cudaStream_t st,
+                                const WaitCfg& wc = kProductWaits);
+// Rows of at least this many 16-byte vectors take the bulk-copy permute.
+#ifndef MOE_PERMUTE_BULK_MIN_VECS
+#define MOE_PERMUTE_BULK_MIN_VECS 32
+#endif
+constexpr int kPermuteBulkMinVecs = MOE_PERMUTE_BULK_MIN_VECS;
 // int8 permute of x[t] * smooth[e] per slot (H <= 16384, multiple of 16; smooth 16-byte
 // aligned); reads the total R from send[E].
 cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
@@ -62,6 +71,16 @@ struct CombineArgs {
   int bs, K, H, A, E, Z, C, Q, dtype;
 };
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st);
+// The same gather (combine forward, or dispatch backward with weights == null)
+// with each token's rows staged in shared memory by bulk copies (gather.cu);
+// launch_combine_fwd takes it for rows of at least kGatherStagedMinVecs vectors.
+#ifndef MOE_GATHER_STAGED_MIN_VECS
+#define MOE_GATHER_STAGED_MIN_VECS 32
+#endif
+constexpr int kGatherStagedMinVecs = MOE_GATHER_STAGED_MIN_VECS;
+bool gather_staged_applies(const CombineArgs& a);
+cudaError_t launch_gather_staged(const CombineArgs& a, cudaStream_t st,
+                                 const WaitCfg& wc = kProductWaits);
 // comm_quant_mode 2: every routed row through the per-row int8 round trip (H <= 16384).
 // With a workspace of combine_q8_workspace_bytes(A) bytes and the total R in send[E], shapes
 // with routed pairs only take two passes (per-row scales, then the gather); otherwise the
@@ -80,6 +99,7 @@ struct CombineBwdArgs {
   void* grad_expand;
   float* grad_w;
   int bs, K, H, A, dtype;
+  int quant_mode;  // 0, or 2: the backward of the int8 round-trip combine
 };
 cudaError_t launch_combine_bwd(const CombineBwdArgs& a, cudaStream_t st);
 

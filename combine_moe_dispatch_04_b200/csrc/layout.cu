@@ -10,12 +10,16 @@
 // those masks give counts and ranks with no ordering race, so the result is
 // deterministic.
 //
-//   BS <= 1024: one CTA of 32 warps does everything (one launch).
-//   otherwise : count (one CTA per 256-token tile) -> scatter (same tiles):
-//               every scatter CTA sums the per-(tile, expert) counts of the
-//               caller's workspace itself (its tile's prefix and the expert
-//               totals), scans the totals, and writes its tile's slots; CTA 0
-//               also writes the counts and the status word.
+//   BS <= 16384 (and the masks fit in shared memory): one launch of a
+//               thread-block cluster of up to 8 CTAs of 1024 threads. Each CTA
+//               counts its tokens, scans its per-warp counts per expert, and
+//               publishes its per-expert totals; after one cluster barrier
+//               every CTA reads the others' totals from distributed shared
+//               memory, scans the grand totals and writes its tokens' slots.
+//               No workspace.
+//   otherwise : count (one CTA per 256-token tile) -> column scan (the count
+//               matrix's exclusive prefix over tiles, in place, and the expert
+//               totals) -> scatter (same tiles): O(tiles * E) work in all.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -126,99 +130,218 @@ __device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const in
 }
 
 // ---------------------------------------------------------------------------
-// One-CTA layout for BS <= 1024: 32 warps, one token per thread.
-// Dynamic shared memory: words[32][E].
-template <int KM>
-__global__ void __launch_bounds__(1024) layout_small_kernel(LayoutArgs a) {
-  extern __shared__ uint32_t words[];
-  __shared__ int offs[1024];
-  __shared__ int warp_sums[32];
-  __shared__ uint32_t status;
-  pdl_trigger();
-  pdl_wait();
-  const int E = a.E;
-  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) words[i] = 0;
-  if (threadIdx.x == 0) status = 0;
-  __syncthreads();
+// Cluster layout. CTA r of the cluster (CS <= 8 CTAs of 1024 threads) takes the
+// tokens [r P, (r + 1) P), P = TPT * 1024, as TPT sub-blocks of 32 warps x 32
+// lanes. Dynamic shared memory: words[TPT][32][S] (lane masks per warp and
+// expert, S = E | 1 so a warp's column reads hit 32 different banks),
+// pre[TPT][32][S] uint16 (exclusive prefix of the mask popcounts over the
+// CTA's warps, per expert), tot[E] (this CTA's per-expert totals, read by the
+// other CTAs of the cluster) and base[E] (first slot of this CTA's pairs per
+// expert).
 
-  const int t = threadIdx.x;
-  int e[KM];
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Cluster-wide barrier halves (every thread of every CTA of the cluster).
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// A 32-bit word of the shared memory of CTA `rank` of this cluster, at the
+// position of `local` in this CTA's shared memory.
+__device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t rank) {
+  const uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+  uint32_t raddr, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(addr), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(raddr) : "memory");
+  return v;
+}
+
+__host__ __device__ constexpr int cluster_stride(int E) { return E | 1; }
+
+__host__ __device__ constexpr size_t cluster_smem_bytes(int E, int tpt) {
+  return static_cast<size_t>(tpt) * 32 * cluster_stride(E) * 4 +
+         (static_cast<size_t>(tpt) * 32 * cluster_stride(E) * 2 + 3) / 4 * 4 +
+         static_cast<size_t>(E) * 8;
+}
+
+// Counts this CTA's tokens [t0, t0 + TPT * 1024) (one per thread and sub-block)
+// into the lane masks, then per expert the exclusive prefix of the popcounts
+// over (sub-block, warp) into pre and the CTA's total into tot (warp w scans
+// the columns w, w + 32, ...; lane = warp of the column). words must be zero
+// on entry; e receives each token's routed experts (-1 elsewhere) and the
+// status bits are ORed into *status.
+template <int KM, int TPT>
+__device__ __forceinline__ void cta_count_scan(const LayoutArgs& a, int t0, int S,
+                                               uint32_t* words, uint16_t* pre, int* tot,
+                                               uint32_t* status, int (&e)[TPT][KM]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t st = 0;
-  if (t < a.bs) {
-    st = classify_row<KM>(a, t, e);
-    mark_words<KM>(words, E, e, a.K);
-  } else {
 #pragma unroll
-    for (int k = 0; k < KM; ++k) e[k] = -1;
+  for (int i = 0; i < TPT; ++i) {
+    const int t = t0 + i * 1024 + threadIdx.x;
+    if (t < a.bs) {
+      st |= classify_row<KM>(a, t, e[i]);
+      const uint32_t bit = 1u << lane;
+#pragma unroll
+      for (int k = 0; k < KM; ++k)
+        if (k < a.K && e[i][k] >= 0) atomicOr(&words[(i * 32 + warp) * S + e[i][k]], bit);
+    } else {
+#pragma unroll
+      for (int k = 0; k < KM; ++k) e[i][k] = -1;
+    }
   }
-  if (st) atomicOr(&status, st);
+  if (st) atomicOr(status, st);
   __syncthreads();
+  for (int ex = warp; ex < a.E; ex += 32) {
+    int carry = 0;
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+      const int c = __popc(words[(i * 32 + lane) * S + ex]);
+      int inc = c;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, d);
+        if (lane >= d) inc += n;
+      }
+      pre[(i * 32 + lane) * S + ex] = static_cast<uint16_t>(carry + inc - c);
+      carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+    }
+    if (lane == 0) tot[ex] = carry;
+  }
+}
 
-  int cnt = 0;
-  if (threadIdx.x < E)
-    for (int w = 0; w < 32; ++w) cnt += __popc(words[w * E + threadIdx.x]);
-  int total;
-  const int excl = block_exclusive_scan(cnt, warp_sums, &total);
+// Slot of each routed pair of token t (sub-block i of this CTA, its own lane).
+template <int KM>
+__device__ __forceinline__ void cta_slots(const LayoutArgs& a, int i, int S, const uint32_t* words,
+                                          const uint16_t* pre, const int* base,
+                                          const int (&e)[KM], int (&slot)[KM]) {
+  const int row = (i * 32 + (threadIdx.x >> 5)) * S;
+#pragma unroll
+  for (int k = 0; k < KM; ++k) {
+    const int ex = e[k];
+    slot[k] = (k < a.K && ex >= 0)
+                  ? base[ex] + pre[row + ex] + __popc(words[row + ex] & lanemask_lt())
+                  : -1;
+  }
+}
+
+template <int KM, int TPT>
+__global__ void __launch_bounds__(1024, 1) layout_cluster_kernel(LayoutArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t status, status_all;
+  const int E = a.E;
+  const int S = cluster_stride(E);
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem);
+  uint16_t* pre = reinterpret_cast<uint16_t*>(smem + static_cast<size_t>(TPT) * 32 * S * 4);
+  int* tot = reinterpret_cast<int*>(smem + static_cast<size_t>(TPT) * 32 * S * 4 +
+                                    (static_cast<size_t>(TPT) * 32 * S * 2 + 3) / 4 * 4);
+  int* base = tot + E;
+  const uint32_t rank = cluster_ctarank(), cs = cluster_nctarank();
+  pdl_trigger();
+  for (int i = threadIdx.x; i < TPT * 32 * S; i += blockDim.x) words[i] = 0;
+  if (threadIdx.x == 0) {
+    status = 0;
+    status_all = 0;
+  }
+  __syncthreads();
+  pdl_wait();
+
+  const int t0 = static_cast<int>(rank) * TPT * 1024;
+  int e[TPT][KM];
+  cta_count_scan<KM, TPT>(a, t0, S, words, pre, tot, &status, e);
+  __syncwarp();
+  cluster_arrive_release();  // tot and status are published to the cluster
+  cluster_wait_acquire();
+
+  // grand totals and the pairs of the CTAs before this one, per expert
+  int grand = 0, before = 0;
   if (threadIdx.x < E) {
-    offs[threadIdx.x] = excl;
-    a.expert_token_nums[threadIdx.x] = cnt;
-    a.ep_send_counts[threadIdx.x] = excl;
+    for (uint32_t c = 0; c < cs; ++c) {
+      const int v = static_cast<int>(ld_dsmem_u32(tot + threadIdx.x, c));
+      grand += v;
+      before += c < rank ? v : 0;
+    }
   }
-  if (threadIdx.x == 0) a.ep_send_counts[E] = total;
+  uint32_t cst = 0;
+  if (rank == 0 && threadIdx.x < cs) cst = ld_dsmem_u32(&status, threadIdx.x);
+  __syncwarp();
+  cluster_arrive_release();  // done reading the other CTAs' shared memory
+  if (cst) atomicOr(&status_all, cst);
+  int total;
+  const int excl = block_exclusive_scan(threadIdx.x < E ? grand : 0, warp_sums, &total);
+  if (threadIdx.x < E) {
+    base[threadIdx.x] = excl + before;
+    if (rank == 0) {
+      a.expert_token_nums[threadIdx.x] = grand;
+      a.ep_send_counts[threadIdx.x] = excl;
+    }
+  }
   __syncthreads();
-
-  if (t < a.bs) {
-    int slot[KM];
-#pragma unroll
-    for (int k = 0; k < KM; ++k)
-      slot[k] = (k < a.K && e[k] >= 0) ? offs[e[k]] + tile_rank(words, E, e[k]) : -1;
-    write_slots<KM>(a, t, e, slot);
+  if (rank == 0 && threadIdx.x == 0) {
+    a.ep_send_counts[E] = total;
+    if (a.dev_status) *a.dev_status = status_all;
   }
-  for (int s = total + threadIdx.x; s < a.A; s += blockDim.x) a.assist[s] = -1;
-  if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) {
+    const int t = t0 + i * 1024 + threadIdx.x;
+    if (t >= a.bs) continue;
+    int slot[KM];
+    cta_slots<KM>(a, i, S, words, pre, base, e[i], slot);
+    write_slots<KM>(a, t, e[i], slot);
+  }
+  for (int s = total + static_cast<int>(rank * blockDim.x + threadIdx.x); s < a.A;
+       s += static_cast<int>(cs * blockDim.x))
+    a.assist[s] = -1;
+  __syncwarp();
+  cluster_wait_acquire();  // no CTA leaves while another may still read its tot
 }
 
 // ---------------------------------------------------------------------------
 // Fused dispatch for BS <= 1024 (layout + permute in one launch). Every CTA
-// rebuilds the whole layout in shared memory exactly as layout_small_kernel
-// does (the ids are at most 64 KB and sit in L2), CTA 0 alone writes the
+// builds the whole layout in shared memory as one CTA of the cluster layout
+// would (the ids are at most 64 KB and sit in L2), CTA 0 alone writes the
 // layout's outputs, and CTA c copies the rows of tokens [c * per, (c+1) * per)
 // to their slots: one thread per 16-byte vector, read once, stored K times.
-// Dynamic shared memory: words[32][E].
+// Dynamic shared memory: words[32][S], pre[32][S] uint16, tot[E], base[E].
 template <int KM>
-__global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, const uint4* x,
-                                                              uint4* expand_x, int V, int per) {
-  extern __shared__ uint32_t words[];
-  __shared__ int offs[1024];
+__global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, const uint4* x,
+                                                                 uint4* expand_x, int V, int per) {
+  extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
   __shared__ int slot_sh[kLayoutSmallMaxTokens / 8][KM];  // slots of this CTA's tokens
-  pdl_trigger();
-  pdl_wait();
   const int E = a.E;
+  const int S = cluster_stride(E);
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem);
+  uint16_t* pre = reinterpret_cast<uint16_t*>(smem + static_cast<size_t>(32) * S * 4);
+  int* tot = reinterpret_cast<int*>(smem + static_cast<size_t>(32) * S * 4 +
+                                    (static_cast<size_t>(32) * S * 2 + 3) / 4 * 4);
+  int* base = tot + E;
   const bool writer = blockIdx.x == 0;
-  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) words[i] = 0;
+  pdl_trigger();
+  for (int i = threadIdx.x; i < 32 * S; i += blockDim.x) words[i] = 0;
   if (threadIdx.x == 0) status = 0;
   __syncthreads();
-  const int t = threadIdx.x;
-  int e[KM];
-  uint32_t st = 0;
-  if (t < a.bs) {
-    st = classify_row<KM>(a, t, e);
-    mark_words<KM>(words, E, e, a.K);
-  } else {
-#pragma unroll
-    for (int k = 0; k < KM; ++k) e[k] = -1;
-  }
-  if (st) atomicOr(&status, st);
+  pdl_wait();
+  int e[1][KM];
+  cta_count_scan<KM, 1>(a, 0, S, words, pre, tot, &status, e);
   __syncthreads();
-  int cnt = 0;
-  if (threadIdx.x < E)
-    for (int w = 0; w < 32; ++w) cnt += __popc(words[w * E + threadIdx.x]);
+  const int cnt = threadIdx.x < E ? tot[threadIdx.x] : 0;
   int total;
   const int excl = block_exclusive_scan(cnt, warp_sums, &total);
   if (threadIdx.x < E) {
-    offs[threadIdx.x] = excl;
+    base[threadIdx.x] = excl;
     if (writer) {
       a.expert_token_nums[threadIdx.x] = cnt;
       a.ep_send_counts[threadIdx.x] = excl;
@@ -226,13 +349,12 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, cons
   }
   if (writer && threadIdx.x == 0) a.ep_send_counts[E] = total;
   __syncthreads();
+  const int t = threadIdx.x;
   const int t0 = blockIdx.x * per;
   if (t < a.bs) {
     int slot[KM];
-#pragma unroll
-    for (int k = 0; k < KM; ++k)
-      slot[k] = (k < a.K && e[k] >= 0) ? offs[e[k]] + tile_rank(words, E, e[k]) : -1;
-    if (writer) write_slots<KM>(a, t, e, slot);
+    cta_slots<KM>(a, 0, S, words, pre, base, e[0], slot);
+    if (writer) write_slots<KM>(a, t, e[0], slot);
     if (t >= t0 && t < t0 + per) {
 #pragma unroll
       for (int k = 0; k < KM; ++k)
@@ -257,17 +379,20 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(LayoutArgs a, cons
 }
 
 // ---------------------------------------------------------------------------
-// Multi-CTA layout. Workspace: tile_counts[T][E] int32, then tile_status[T].
+// Multi-CTA layout. Workspace: tile_counts[T][E] int32 (turned into their
+// exclusive prefix over tiles by the column scan), totals[E], tile_status[T].
 
 struct TileWs {
   int32_t* counts;
+  int32_t* totals;
   uint32_t* status;
 };
 
 __device__ __forceinline__ TileWs tile_ws(const LayoutArgs& a, int T) {
   TileWs w;
   w.counts = static_cast<int32_t*>(a.workspace);
-  w.status = reinterpret_cast<uint32_t*>(w.counts + static_cast<size_t>(T) * a.E);
+  w.totals = w.counts + static_cast<size_t>(T) * a.E;
+  w.status = reinterpret_cast<uint32_t*>(w.totals + a.E);
   return w;
 }
 
@@ -276,7 +401,8 @@ constexpr int kTileWarps = kLayoutTileTokens / 32;
 // Phase 1: per-tile expert counts and status bits.
 template <int KM>
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutArgs a, int T) {
-  extern __shared__ uint32_t words[];  // [kTileWarps][E]
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem);  // [kTileWarps][E]
   __shared__ uint32_t status;
   pdl_trigger();
   pdl_wait();
@@ -302,12 +428,43 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_count_kernel(LayoutA
   if (threadIdx.x == 0) ws.status[blockIdx.x] = status;
 }
 
-// Phase 2 for one 256-token tile, run by a whole CTA: the tile's first slot
-// per expert from the count matrix (prefix over earlier tiles + exclusive
-// scan of the expert totals), then slot[] of this thread's token (t < BS).
-// The CTA with first_cta writes the counts, prefix sums and status word.
-// Shared memory (dynamic): words[kTileWarps][E], base[E], total[E], and two
-// [G][E] partial-sum arrays (G * E <= blockDim).
+// Phase 2: per expert, the exclusive prefix of the tile counts over tiles (in
+// place) and the expert total. A CTA takes 32 experts; its 32 warps split the
+// tiles into 32 segments (lane = expert, so each warp reads 32 consecutive
+// counts), sum their segment, take the prefix over segments from shared
+// memory, and rewrite their segment.
+__global__ void __launch_bounds__(1024) layout_colscan_kernel(LayoutArgs a, int T) {
+  __shared__ int part[32][33];
+  pdl_trigger();
+  pdl_wait();
+  const int el = threadIdx.x & 31, seg = threadIdx.x >> 5;
+  const int ex = blockIdx.x * 32 + el;
+  const int per = (T + 31) / 32;
+  const int i0 = min(T, seg * per), i1 = min(T, i0 + per);
+  const TileWs ws = tile_ws(a, T);
+  int sum = 0;
+  if (ex < a.E)
+    for (int i = i0; i < i1; ++i) sum += ws.counts[static_cast<size_t>(i) * a.E + ex];
+  part[seg][el] = sum;
+  __syncthreads();
+  int run = 0;
+  for (int g = 0; g < seg; ++g) run += part[g][el];
+  if (ex < a.E) {
+    if (seg == 31) ws.totals[ex] = run + sum;
+    for (int i = i0; i < i1; ++i) {
+      const size_t at = static_cast<size_t>(i) * a.E + ex;
+      const int c = ws.counts[at];
+      ws.counts[at] = run;
+      run += c;
+    }
+  }
+}
+
+// Phase 3 for one 256-token tile, run by a whole CTA: the tile's first slot
+// per expert (its prefix over earlier tiles + the exclusive scan of the expert
+// totals), then slot[] of this thread's token (t < BS). The CTA with first_cta
+// writes the counts, prefix sums and status word. Shared memory (dynamic):
+// words[kTileWarps][E], base[E], total[E].
 template <int KM>
 __device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile, bool first_cta,
                                            uint32_t* smem, int* warp_sums, uint32_t* status,
@@ -319,52 +476,15 @@ __device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile,
   for (int i = threadIdx.x; i < kTileWarps * E; i += blockDim.x) words[i] = 0;
   if (threadIdx.x == 0) *status = 0;
   // this thread's token: its ids are loaded now, so their latency overlaps
-  // the count-matrix loads below
+  // the workspace loads below
   const int t = tile * kLayoutTileTokens + threadIdx.x;
 #pragma unroll
   for (int k = 0; k < KM; ++k) e[k] = -1;
   if (t < a.bs) classify_row<KM>(a, t, e);
   const TileWs ws = tile_ws(a, T);
-  // Sum the count matrix over tiles: G groups of E threads split the tiles
-  // (G = 1 when E >= blockDim), then one thread per expert adds the groups.
-  const int G = E < static_cast<int>(blockDim.x) ? blockDim.x / E : 1;
-  int* part_before = total + E;         // [G][E]
-  int* part_all = part_before + G * E;  // [G][E]
-  if (G > 1) {
-    const int g = threadIdx.x / E, ex = threadIdx.x - g * E;
-    if (g < G) {
-      int before = 0, all = 0;
-#pragma unroll 4
-      for (int i = g; i < T; i += G) {
-        const int c = ws.counts[static_cast<size_t>(i) * E + ex];
-        before += i < tile ? c : 0;
-        all += c;
-      }
-      part_before[g * E + ex] = before;
-      part_all[g * E + ex] = all;
-    }
-    __syncthreads();
-    for (int ex2 = threadIdx.x; ex2 < E; ex2 += blockDim.x) {
-      int before = 0, all = 0;
-      for (int gg = 0; gg < G; ++gg) {
-        before += part_before[gg * E + ex2];
-        all += part_all[gg * E + ex2];
-      }
-      base[ex2] = before;
-      total[ex2] = all;
-    }
-  } else {
-    for (int ex = threadIdx.x; ex < E; ex += blockDim.x) {
-      int before = 0, all = 0;
-#pragma unroll 8
-      for (int i = 0; i < T; ++i) {
-        const int c = ws.counts[static_cast<size_t>(i) * E + ex];
-        before += i < tile ? c : 0;
-        all += c;
-      }
-      base[ex] = before;
-      total[ex] = all;
-    }
+  for (int ex = threadIdx.x; ex < E; ex += blockDim.x) {
+    base[ex] = ws.counts[static_cast<size_t>(tile) * E + ex];
+    total[ex] = ws.totals[ex];
   }
   if (first_cta) {
     uint32_t st = 0;
@@ -400,17 +520,18 @@ __device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile,
   *grand_out = grand;
 }
 
-// Phase 2 as its own launch: every tile's slots, and -1 for the unused
+// Phase 3 as its own launch: every tile's slots, and -1 for the unused
 // slots [R, A).
 template <int KM>
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
-  extern __shared__ uint32_t smem[];
+  extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
   pdl_trigger();
   pdl_wait();
   int e[KM], slot[KM], grand;
-  tile_slots<KM>(a, T, blockIdx.x, blockIdx.x == 0, smem, warp_sums, &status, e, slot, &grand);
+  tile_slots<KM>(a, T, blockIdx.x, blockIdx.x == 0, reinterpret_cast<uint32_t*>(smem), warp_sums,
+                 &status, e, slot, &grand);
   const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
   if (t < a.bs) write_slots<KM>(a, t, e, slot);
   for (int s = grand + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
@@ -429,35 +550,67 @@ cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* ex
   if (per > kLayoutSmallMaxTokens / 8) per = kLayoutSmallMaxTokens / 8;
   if (per < 1) per = 1;
   blocks = a.bs > 0 ? (a.bs + per - 1) / per : 1;
-  const size_t smem = 32u * a.E * sizeof(uint32_t);
-  if (smem > 32 * 1024) {  // with the static buffers: opt in before the total passes 48 KB
-    cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel<KM>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-  }
+  const size_t smem = cluster_smem_bytes(a.E, 1);
+  cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel<KM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
   return launch_pdl(dispatch_small_kernel<KM>, dim3(blocks), dim3(1024), smem, st, a,
                     static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
 }
 
+// Largest BS of the cluster layout (8 CTAs of 1024 threads, two tokens each),
+// and its shared memory limit.
+#ifndef MOE_LAYOUT_CLUSTER_MAX_TOKENS
+#define MOE_LAYOUT_CLUSTER_MAX_TOKENS (8 * 2 * 1024)
+#endif
+constexpr int kClusterMaxTokens = MOE_LAYOUT_CLUSTER_MAX_TOKENS;
+constexpr size_t kClusterSmemMax = 210 * 1024;
+
+int cluster_tpt(int bs) { return bs <= 8 * 1024 ? 1 : 2; }
+
+bool cluster_layout_applies(int bs, int E) {
+  return bs <= kClusterMaxTokens && cluster_smem_bytes(E, cluster_tpt(bs)) <= kClusterSmemMax;
+}
+
+template <int KM, int TPT>
+cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st) {
+  constexpr auto kernel = layout_cluster_kernel<KM, TPT>;
+  const size_t smem = cluster_smem_bytes(a.E, TPT);
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  int cs = (a.bs + TPT * 1024 - 1) / (TPT * 1024);
+  if (cs < 1) cs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs);
+  cfg.blockDim = dim3(1024);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 template <int KM>
 cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t st) {
-  if (a.bs <= kLayoutSmallMaxTokens) {
-    const size_t smem = 32u * a.E * sizeof(uint32_t);
-    if (smem > 32 * 1024) {
-      cudaError_t err = cudaFuncSetAttribute(layout_small_kernel<KM>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-      if (err != cudaSuccess) return err;
-    }
-    return launch_pdl(layout_small_kernel<KM>, dim3(1), dim3(1024), smem, st, a);
-  }
+  if (cluster_layout_applies(a.bs, a.E))
+    return cluster_tpt(a.bs) == 1 ? launch_layout_cluster<KM, 1>(a, st)
+                                  : launch_layout_cluster<KM, 2>(a, st);
   const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
   const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
-  const size_t smem_scatter =
-      smem_count + 2u * a.E * sizeof(int) + 2u * kLayoutTileTokens * sizeof(int);
+  const size_t smem_scatter = smem_count + 2u * a.E * sizeof(int);
   cudaError_t err = launch_pdl(layout_count_kernel<KM>, dim3(T), dim3(kLayoutTileTokens),
                                smem_count, st, a, T);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(layout_colscan_kernel, dim3((a.E + 31) / 32), dim3(1024), 0, st, a, T);
   if (err != cudaSuccess) return err;
   return launch_pdl(layout_scatter_kernel<KM>, dim3(T), dim3(kLayoutTileTokens), smem_scatter,
                     st, a, T);
@@ -474,9 +627,9 @@ cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expa
 }
 
 size_t layout_workspace_bytes(int bs, int E) {
-  if (bs <= kLayoutSmallMaxTokens) return 0;
+  if (cluster_layout_applies(bs, E)) return 0;
   const size_t T = (static_cast<size_t>(bs) + kLayoutTileTokens - 1) / kLayoutTileTokens;
-  return T * static_cast<size_t>(E) * 4 + T * 4;
+  return T * static_cast<size_t>(E) * 4 + static_cast<size_t>(E) * 4 + T * 4;
 }
 
 cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st) {

@@ -43,6 +43,95 @@ __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
   }
 }
 
+// The plain copy on the bulk-copy engine: each warp takes a contiguous range of
+// units (one column chunk of one token's row) and keeps kPbStages of them in
+// flight. Lane 0 brings a unit's chunk into the warp's stage buffer with one
+// bulk copy (global -> shared, on the buffer's mbarrier); once it has landed,
+// lane k < K copies the buffer to slot(t, k) with one bulk copy (shared ->
+// global, its own bulk async-group). A buffer is refilled only after every
+// lane's stores from it have finished reading it (wait_group.read). x is read
+// once, and the K-fold write fan-out costs K bulk operations per unit instead
+// of K 16-byte stores per thread. Every wait is bounded; a warp that gives up
+// counts itself in *timeouts, lets its started copies land and returns.
+constexpr int kPbWarps = 4;
+constexpr int kPbStages = 4;
+
+__host__ __device__ constexpr size_t pb_warp_bytes(int cvec) {
+  return 128 + static_cast<size_t>(kPbStages) * cvec * 16;
+}
+
+__global__ void __launch_bounds__(32 * kPbWarps) permute_bulk_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
+    int bs, int K, int V, int A, int nchunks, int cvec, WaitCfg wc, unsigned* timeouts) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char* wbase = smem + static_cast<size_t>(warp) * pb_warp_bytes(cvec);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase);
+  uint4* stages = reinterpret_cast<uint4*>(wbase + 128);
+  if (lane == 0) {
+    for (int b = 0; b < kPbStages; ++b) mbar_init(bars + b, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  pdl_trigger();
+  pdl_wait();
+  const long long units = static_cast<long long>(bs) * nchunks;
+  const long long nw = static_cast<long long>(gridDim.x) * kPbWarps;
+  const long long gw = static_cast<long long>(blockIdx.x) * kPbWarps + warp;
+  const long long per = (units + nw - 1) / nw;
+  const long long u0 = gw * per < units ? gw * per : units;
+  const long long u1 = u0 + per < units ? u0 + per : units;
+  const int32_t* slots = assist + static_cast<size_t>(A);
+
+  // test hook: the first warp's unit withhold waits for 16 bytes that never come
+  const long long held = (gw == 0 && wc.withhold >= 0) ? u0 + wc.withhold : -1;
+  auto issue = [&](long long u, int b) {  // lane 0: unit u into buffer b
+    if (u == held) {
+      mbar_arrive_expect_tx(bars + b, 16u);
+      return;
+    }
+    const int t = static_cast<int>(u / nchunks);
+    const int v0 = static_cast<int>(u - static_cast<long long>(t) * nchunks) * cvec;
+    const uint32_t bytes = static_cast<uint32_t>(min(cvec, V - v0)) * 16u;
+    mbar_arrive_expect_tx(bars + b, bytes);
+    bulk_g2s(stages + static_cast<size_t>(b) * cvec, x + static_cast<size_t>(t) * V + v0, bytes,
+             bars + b);
+  };
+  if (lane == 0)
+    for (int p = 0; p < kPbStages - 1; ++p)
+      if (u0 + p < u1) issue(u0 + p, p);
+  int next_slot = -1;
+  if (u0 < u1 && lane < K) next_slot = __ldg(slots + (u0 / nchunks) * K + lane);
+  int i = 0;
+  for (long long u = u0; u < u1; ++u, ++i) {
+    const int b = i % kPbStages;
+    const int slot = next_slot;
+    if (u + 1 < u1 && lane < K) next_slot = __ldg(slots + ((u + 1) / nchunks) * K + lane);
+    const bool ok = mbar_wait_bounded(bars + b, (i / kPbStages) & 1, wc.limit_ns);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) {
+        atomicAdd(timeouts, 1u);
+        for (int q = 0; q < kPbStages - 1; ++q)  // loads already started: let them land
+          if (u + q < u1 && u + q != held)
+            mbar_wait_bounded(bars + (i + q) % kPbStages, ((i + q) / kPbStages) & 1);
+      }
+      break;
+    }
+    fence_proxy_async_smem();
+    const int t = static_cast<int>(u / nchunks);
+    const int v0 = static_cast<int>(u - static_cast<long long>(t) * nchunks) * cvec;
+    const uint32_t bytes = static_cast<uint32_t>(min(cvec, V - v0)) * 16u;
+    if (lane < K && slot >= 0)
+      bulk_s2g(out + static_cast<size_t>(slot) * V + v0, stages + static_cast<size_t>(b) * cvec,
+               bytes);
+    bulk_commit_group();
+    bulk_wait_group_read<1>();  // the stores of earlier units have read their buffers
+    __syncwarp();
+    if (lane == 0 && u + kPbStages - 1 < u1) issue(u + kPbStages - 1, (i + kPbStages - 1) % kPbStages);
+  }
+  bulk_wait_group<0>();  // every store of this lane performed before the warp leaves
+}
+
 // CPT 16-element chunks per thread (1, 2 or 4), chosen by the launcher so a
 // row fits the CTA with as few registers as possible.
 template <typename T16, int CPT>
@@ -248,8 +337,22 @@ __host__ __device__ constexpr size_t smooth_warp_bytes(int H) {
   return (128 + static_cast<size_t>(kSmoothStages) * H * 2 + 127) / 128 * 128;
 }
 
-template <typename T16>
-__global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
+// SPL > 0 (H = 256 * SPL): the warp keeps the current expert's smooth row in
+// registers (lane l: vectors l, l + 32, ...), reloading it only when the
+// expert of its next slot differs, so the per-value smooth factors come from
+// registers instead of L1 (whose bandwidth bounded the SPL = 0 form, which
+// reads them from L1 in both passes).
+// Threads and resident blocks per SM of the staged smooth kernel: with the
+// smooth row of H = 2048 in registers a warp needs about 160 of them, so 12
+// warps make one block per SM; otherwise 8 warps and two blocks.
+template <int SPL>
+__host__ __device__ constexpr int smooth_threads() { return SPL >= 8 ? 384 : 256; }
+template <int SPL>
+__host__ __device__ constexpr int smooth_blocks_per_sm() { return SPL >= 8 ? 1 : 2; }
+
+template <typename T16, int SPL>
+__global__ void __launch_bounds__(smooth_threads<SPL>(), smooth_blocks_per_sm<SPL>())
+    permute_smooth_staged_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
     const float4* __restrict__ smooth, const int32_t* __restrict__ assist,
     const int32_t* __restrict__ send, uint2* __restrict__ out, float* __restrict__ scales, int K,
@@ -302,6 +405,8 @@ __global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
 
   for (int p = 0; p < kSmoothStages - 1; ++p)
     if (lo + warp + p * nwarps < hi) stage(p, p);
+  float4 sreg[SPL > 0 ? SPL : 1][2];  // the current expert's smooth factors (SPL > 0)
+  int cur_e = -1;
   int it = 0;
   for (int s = lo + warp; s < hi; s += nwarps, ++it) {
     const int b = it % kSmoothStages;
@@ -320,6 +425,44 @@ __global__ void __launch_bounds__(256, 2) permute_smooth_staged_kernel(
     if (s + (kSmoothStages - 1) * nwarps < hi)
       stage(it + kSmoothStages - 1, (it + kSmoothStages - 1) % kSmoothStages);
     const SmoothSlot si = info[b];
+    if constexpr (SPL > 0) {
+      if (si.e >= 0) {
+        if (si.e != cur_e) {  // warp-uniform: the slot's expert is in shared memory
+          const float4* sr = smooth + static_cast<size_t>(si.e) * (H / 4);
+#pragma unroll
+          for (int j = 0; j < SPL; ++j) {
+            const int v = lane + 32 * j;
+            sreg[j][0] = __ldg(sr + 2 * v);
+            sreg[j][1] = __ldg(sr + 2 * v + 1);
+          }
+          cur_e = si.e;
+        }
+        const uint4* xr = rows + static_cast<size_t>(b) * V;
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < SPL; ++j) {
+          float y[8];
+          widen8<T16>(xr[lane + 32 * j], y);
+          smooth_mul8(y, sreg[j][0], sreg[j][1]);
+          amax = fmaxf(amax, absmax8(y));
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+        const float scale = __fdiv_rn(amax, 127.0f);
+        const float inv_scale = 1.0f / scale;
+        uint2* orow = out + static_cast<size_t>(si.slot) * V;
+#pragma unroll
+        for (int j = 0; j < SPL; ++j) {
+          float y[8];
+          widen8<T16>(xr[lane + 32 * j], y);
+          smooth_mul8(y, sreg[j][0], sreg[j][1]);
+          orow[lane + 32 * j] = pack_codes8(y, amax, scale, inv_scale);
+        }
+        if (lane == 0) scales[si.slot] = scale;
+      }
+      __syncwarp();
+      continue;
+    }
     if (si.e >= 0) {
       const uint4* xr = rows + static_cast<size_t>(b) * V;
       const float4* sr = smooth + static_cast<size_t>(si.e) * (H / 4);
@@ -379,9 +522,19 @@ cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
   // Staged kernel when at least four warps' buffers fit in 110 KB (two CTAs per SM).
   const int staged_warps = static_cast<int>(110 * 1024 / smooth_warp_bytes(a.H));
   if (staged_warps >= 4) {
-    const int warps = staged_warps < 8 ? staged_warps : 8;
+    int warps = staged_warps < 8 ? staged_warps : 8;
+    auto sk = bf ? permute_smooth_staged_kernel<Bf16, 0> : permute_smooth_staged_kernel<Fp16, 0>;
+    if (a.H % 256 == 0 && a.H <= 2048) {  // the smooth row fits in a warp's registers
+      const int spl = a.H / 256;
+      if (spl == 1) sk = bf ? permute_smooth_staged_kernel<Bf16, 1> : permute_smooth_staged_kernel<Fp16, 1>;
+      if (spl == 2) sk = bf ? permute_smooth_staged_kernel<Bf16, 2> : permute_smooth_staged_kernel<Fp16, 2>;
+      if (spl == 4) sk = bf ? permute_smooth_staged_kernel<Bf16, 4> : permute_smooth_staged_kernel<Fp16, 4>;
+      if (spl == 8) {  // one block of 12 warps per SM (smooth_threads<8>)
+        sk = bf ? permute_smooth_staged_kernel<Bf16, 8> : permute_smooth_staged_kernel<Fp16, 8>;
+        warps = smooth_threads<8>() / 32;
+      }
+    }
     const size_t smem = static_cast<size_t>(warps) * smooth_warp_bytes(a.H);
-    auto sk = bf ? permute_smooth_staged_kernel<Bf16> : permute_smooth_staged_kernel<Fp16>;
     cudaError_t err = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
@@ -411,8 +564,49 @@ cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
                     static_cast<uint4*>(a.expand_x), a.scales, a.K, a.H, a.A, E);
 }
 
+// Column chunks per row for the bulk permute: with nw warps each taking
+// ceil(units / nw) units, pick the chunking (chunks of 1 to 4 KB) whose
+// busiest warp moves the fewest bytes (plus a per-unit overhead).
+void pb_chunking(int bs, int V, long long nw, int* nchunks, int* cvec) {
+  const int nmin = (V + 255) / 256;  // chunks of at most 4 KB
+  long long best = -1;
+  for (int n = nmin; n <= 4 * nmin && n <= V; ++n) {
+    const int cv = (V + n - 1) / n;
+    if (static_cast<long long>(n - 1) * cv >= V) continue;  // no empty last chunk
+    const long long units = static_cast<long long>(bs) * n;
+    const long long cost = ((units + nw - 1) / nw) * (static_cast<long long>(cv) * 16 + 256);
+    if (best < 0 || cost < best) {
+      best = cost;
+      *nchunks = n;
+      *cvec = cv;
+    }
+  }
+}
+
+cudaError_t launch_permute_bulk(const PermuteArgs& a, cudaStream_t st, const WaitCfg& wc) {
+  const int V = a.H / kVecElems;
+  unsigned* timeouts = wait_timeout_counter();
+  if (timeouts == nullptr) return cudaErrorInvalidSymbol;
+  const long long nw = static_cast<long long>(sm_count()) * 2 * kPbWarps;  // two CTAs per SM
+  int nchunks = 1, cvec = V;
+  pb_chunking(a.bs, V, nw, &nchunks, &cvec);
+  const size_t smem = kPbWarps * pb_warp_bytes(cvec);
+  cudaError_t err = cudaFuncSetAttribute(permute_bulk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const long long units = static_cast<long long>(a.bs) * nchunks;
+  const long long want = (units + kPbWarps - 1) / kPbWarps;
+  const long long cap = nw / kPbWarps;
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(permute_bulk_kernel, dim3(blocks), dim3(32 * kPbWarps), smem, st,
+                    static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
+                    a.bs, a.K, V, a.A, nchunks, cvec, wc, timeouts);
+}
+
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
+  if (a.quant_mode == 0 && a.H / kVecElems >= kPermuteBulkMinVecs) return launch_permute_bulk(a, st);
   if (a.quant_mode == 0) {
     const int V = a.H / kVecElems;
     const long long n = static_cast<long long>(a.bs) * V;

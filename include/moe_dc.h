@@ -267,6 +267,23 @@ moe_status moe_combine_bwd(const moe_shape* shape, const void* grad_out, const v
                            void* grad_expand, float* grad_w, void* stream);
 
 /*
+ * moe_combine_bwd_comm_quant — the backward of moe_combine_fwd_comm_quant
+ * ([combine] Parameters: comm_quant_mode). Mode 0 is moe_combine_bwd. Mode 2:
+ * the forward summed each routed row's int8 round-trip values D(y) = fp32
+ * q * scale (scale = max_h |y| / 127, IEEE division; q as in the forward), so
+ *   grad_w[t,k]            = sum_h grad_out[t,h] * D(expand_x[slot(t,k)])[h]
+ * and the round trip, piecewise constant, is passed straight through:
+ *   grad_expand[slot(t,k)] = round16(w[t,k] * grad_out[t])  (as in mode 0).
+ * Arguments, layouts and the pairs without a slot as in moe_combine_bwd;
+ * MOE_ERR_ARG for a mode other than 0 or 2.
+ */
+moe_status moe_combine_bwd_comm_quant(const moe_shape* shape, const void* grad_out,
+                                      const void* expand_x, const int32_t* topk_idx,
+                                      const float* topk_weights, const int32_t* assist_info,
+                                      const uint8_t* x_active_mask, int comm_quant_mode,
+                                      void* grad_expand, float* grad_w, void* stream);
+
+/*
  * moe_combine_bwd_special — gradient of the combine Formula through the copy
  * and const experts ([combine] Function, special expert use cases: copy
  * Moe(ori_x) = ori_x, const Moe(ori_x) = alpha_1 * ori_x + alpha_2 * v), the
@@ -341,6 +358,38 @@ moe_status moe_dispatch_layout_noalloc(const moe_shape* shape, const int32_t* to
 
 /* Bytes of the fixed scratch array moe_dispatch_layout_noalloc uses. */
 size_t moe_layout_noalloc_max_workspace_bytes(void);
+
+/*
+ * Test hooks for the bounded waits (no counterpart on the pages). The staged
+ * kernels wait on mbarriers for their own bulk copies; every such wait gives
+ * up after a time limit, counts the giving-up block in
+ * moe_async_wait_timeouts(), lets the copies it started land, and returns,
+ * leaving that block's part of the output unwritten. These two calls run the
+ * staged combine gather and the bulk-copy permute with a shorter limit and one
+ * unit of work whose barrier is armed for 16 bytes that no copy delivers (in
+ * the first block, or the first warp), so that the give-up path runs while no
+ * copy is in flight for that unit. Not for production use.
+ *   wait_limit_ns   limit of the pipeline waits, in (0, 1e9] ns
+ *   withhold_unit   index, among the units of the first block (combine: token
+ *                   column chunks; permute: the first warp's units), of the
+ *                   unit whose copies are withheld; >= 0
+ * Other arguments as moe_combine_fwd / moe_dispatch_permute (mode 0). Returns
+ * MOE_ERR_UNSUPPORTED for shapes those calls run on other kernels (rows
+ * narrower than 32 vectors of 16 bytes).
+ */
+moe_status moe_test_combine_fwd_wait_timeout(const moe_shape* shape, const void* expand_x,
+                                             const int32_t* topk_idx, const float* topk_weights,
+                                             const int32_t* assist_info,
+                                             const uint8_t* x_active_mask,
+                                             const void* shared_expert_x, const void* ori_x,
+                                             const void* const_alpha_1,
+                                             const void* const_alpha_2, const void* const_v,
+                                             void* out, uint64_t wait_limit_ns,
+                                             int withhold_unit, void* stream);
+moe_status moe_test_dispatch_permute_wait_timeout(const moe_shape* shape, const void* x,
+                                                  const int32_t* assist_info, void* expand_x,
+                                                  uint64_t wait_limit_ns, int withhold_unit,
+                                                  void* stream);
 
 #ifdef __cplusplus
 }

@@ -68,14 +68,19 @@ def test_k_larger_than_id_range():
                         idx=None) == moe.MOE_ERR_ARG  # K <= N accepted, null idx caught
 
 
+# Above 16384 tokens the layout runs in tiles and needs a workspace.
+TILED = moe.Shape(bs=20000, k=8, h=1536, num_experts=64)
+
+
 def test_null_pointers_and_workspace():
     assert _call_layout(GOOD, idx=None) == moe.MOE_ERR_ARG
     assert _call_layout(GOOD, assist=None) == moe.MOE_ERR_ARG
-    assert _call_layout(GOOD, ws=None) == moe.MOE_ERR_CAPACITY
-    need = moe.moe_layout_workspace_bytes(ctypes.byref(GOOD.c()))
-    assert need > 0
-    assert _call_layout(GOOD, ws_bytes=need - 1) == moe.MOE_ERR_CAPACITY
-    assert _call_layout(GOOD, ws=ctypes.c_void_p(8)) == moe.MOE_ERR_ALIGN
+    assert _call_layout(TILED, ws=None) == moe.MOE_ERR_CAPACITY
+    need = moe.moe_layout_workspace_bytes(ctypes.byref(TILED.c()))
+    t = (20000 + 255) // 256
+    assert need == 4 * (t * 64 + 64 + t)  # tile counts, expert totals, tile status words
+    assert _call_layout(TILED, ws_bytes=need - 1) == moe.MOE_ERR_CAPACITY
+    assert _call_layout(TILED, ws=ctypes.c_void_p(8)) == moe.MOE_ERR_ALIGN
     masked = moe.Shape(bs=64, k=8, h=1536, num_experts=64, mask_ndim=2)
     assert _call_layout(masked) == moe.MOE_ERR_ARG  # mask_ndim 2 without a mask
 
@@ -129,7 +134,12 @@ def test_other_entry_points_check_first():
 def test_sizes():
     s = moe.Shape(bs=128, k=8, h=1536, num_experts=64)
     assert moe.moe_assist_info_elems(ctypes.byref(s.c())) == 1024 + 128 * 8
-    assert moe.moe_layout_workspace_bytes(ctypes.byref(s.c())) == 0  # one-CTA layout
+    assert moe.moe_layout_workspace_bytes(ctypes.byref(s.c())) == 0  # cluster layout
+    # the cluster layout takes up to 16384 tokens while its masks fit in shared memory
+    for bs, e, need_ws in ((16384, 256, False), (16385, 64, True), (8192, 1024, False),
+                           (9000, 1024, True)):
+        sh = moe.Shape(bs=bs, k=8, h=1536, num_experts=e)
+        assert (moe.moe_layout_workspace_bytes(ctypes.byref(sh.c())) > 0) == need_ws
     assert moe.moe_status_string(moe.MOE_ERR_CUDA) == b"CUDA error"
 
 

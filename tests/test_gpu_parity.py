@@ -76,6 +76,14 @@ EDGE = [
     _custom("fp16_quant", bs=1030, h=2064, dtype="fp16", quant_mode=2, expert="dequant",
             backward=False),
     _custom("zipf_hot", bs=2048, k=2, num_experts=300, routing="zipf", zipf_s=3.0),
+    # layout paths: the cluster kernel at its largest E (one token per thread) and
+    # with two tokens per thread, then the tiled count / column-scan / scatter path
+    # just above the cluster's limit and at 65536 tokens with E = 1024
+    _custom("cluster_k16_e1024", bs=8192, k=16, num_experts=1024, h=64),
+    _custom("cluster_two_per_thread", bs=16384, k=16, num_experts=256, h=64, mask_ndim=1,
+            mask_false_p=0.2, backward=False),
+    _custom("tiled_just_above_cluster", bs=16385, k=4, num_experts=64, h=64, backward=False),
+    _custom("tiled_bs65536_e1024", bs=65536, k=8, num_experts=1024, h=64, backward=False),
 ]
 
 
@@ -390,3 +398,47 @@ def test_special_expert_backward(wl):
         close(host(ga1), ref["grad_alpha1"], ref["abs_alpha1"], "grad_alpha1")
         close(host(ga2), ref["grad_alpha2"], ref["abs_alpha2"], "grad_alpha2")
         close(host(gv), ref["grad_v"], ref["abs_v"], "grad_v")
+
+
+QBWD = [
+    W["special"].scaled(backward=True, name="special_full_q8_bwd"),
+    W["uniform"].scaled(name="uniform_full_q8_bwd"),
+    W["mixtral"].scaled(bs=1200, h=264, name="mixtral_fp16_mask_q8_bwd"),
+    _custom("k16_narrow_q8_bwd", bs=700, k=16, num_experts=40, h=136),
+]
+
+
+@pytest.mark.parametrize("wl", QBWD, ids=lambda w: w.name)
+def test_combine_bwd_comm_quant_mode2(wl):
+    """Backward of the int8 round-trip combine against the oracle: grad_expand bit
+    for bit (the round trip passed straight through), grad_w within 1e-5 of
+    max(|ref|, sum_h |grad_out * D(y)|), D the round-trip values; rows include
+    all-zero rows and, in bf16, rows whose scale is below 2^-100."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    inp = workloads.generate(wl)
+    dt = wl.dtype
+    _, send, assist, st = oracle.dispatch_layout(inp["topk_idx"], wl.num_experts, wl.n_ids,
+                                                 wl.a_capacity, inp["mask"])
+    r = int(send[-1])
+    rng = np.random.default_rng(9)
+    scale = rng.uniform(0.01, 10, (wl.a_capacity, 1))
+    if dt == "bf16":
+        scale[rng.random(wl.a_capacity) < 0.05] = 2.0 ** -110
+    y = workloads.encode16(rng.standard_normal((wl.a_capacity, wl.h)) * scale, dt)
+    y[:3] = 0
+    ge_ref, gw_ref, mag = oracle.combine_bwd(inp["grad_out"], y, inp["topk_weights"], assist,
+                                             k=wl.k, a_capacity=wl.a_capacity, dtype=dt,
+                                             mask=inp["mask"], comm_quant_mode=2)
+    sh = gpu_chain.shape_of(wl)
+    dev, host = gpu_chain.dev, gpu_chain.host
+    lay = moe.dispatch_layout(sh, dev(inp["topk_idx"]), dev(inp["mask"]))
+    ge, gw = moe.combine_bwd(sh, dev(inp["grad_out"], dt), dev(y, dt), dev(inp["topk_weights"]),
+                             lay, x_active_mask=dev(inp["mask"]), comm_quant_mode=2)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(ge)[:r], ge_ref[:r])
+    err = np.abs(host(gw).astype(np.float64) - gw_ref.astype(np.float64))
+    bound = gpu_chain.GRAD_W_RTOL * np.maximum(np.abs(gw_ref.astype(np.float64)), mag)
+    assert np.all(err <= bound), float((err / np.maximum(bound, 1e-30)).max())

@@ -48,6 +48,9 @@ def _host(lay):
     workloads.WORKLOADS[3],                                      # 16384 tokens, 2-D mask
     workloads.WORKLOADS[4].scaled(bs=3000, h=64),                # special experts
     workloads.WORKLOADS[0],                                      # 128 tokens, one-CTA layout
+    # tiled layouts, the ones that use the scratch array
+    workloads.WORKLOADS[1].scaled(bs=20000, h=64, name="tiled_20000"),
+    workloads.WORKLOADS[2].scaled(bs=40000, h=64, name="tiled_40000_e256"),
 ], ids=lambda w: w.name)
 def test_noalloc_matches_workspace_layout_twice(wl):
     dev = torch.device("cuda", 0)
