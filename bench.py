@@ -193,12 +193,13 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------
 
-def layout_launches(bs: int, num_experts: int) -> int:
+def layout_launches(bs: int, num_experts: int, k: int) -> int:
     """Launches of moe_dispatch_layout: one thread-block cluster for BS <= 16384 when
-    its lane masks fit in shared memory, else count, column scan and scatter."""
-    tpt = 1 if bs <= 8192 else 2
+    its lane masks and pair lists fit in shared memory, else count, column scan and
+    scatter."""
+    nt = 512 if bs <= 8192 and num_experts <= 512 else 1024
     stride = num_experts | 1
-    smem = tpt * 32 * stride * 4 + (tpt * 32 * stride * 2 + 3) // 4 * 4 + num_experts * 8
+    smem = (nt // 32) * stride * 8 + num_experts * 12 + nt * k * 4
     return 1 if bs <= 16384 and smem <= 210 * 1024 else 3
 
 
@@ -506,7 +507,7 @@ class Bench:
         if fused and wl.bs <= 1024 and qm == 0:
             dispatch_launches = 1
         else:
-            dispatch_launches = layout_launches(wl.bs, wl.num_experts) + 1
+            dispatch_launches = layout_launches(wl.bs, wl.num_experts, wl.k) + 1
         special_bwd_launches = 0
         if "combine_bwd_special" in bytes_per:
             special_bwd_launches = 1 + (2 if wl.const_expert_num else 0)

@@ -30,7 +30,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_assist_info_elems",
            "moe_combine_bwd_special_workspace_bytes", "moe_dispatch_permute_smooth",
            "moe_async_wait_timeouts", "moe_combine_fwd_comm_quant_ws",
            "moe_combine_fwd_comm_quant_workspace_bytes", "moe_combine_bwd_comm_quant",
-           "moe_test_combine_fwd_wait_timeout", "moe_test_dispatch_permute_wait_timeout")
+           "moe_test_combine_fwd_comm_quant_wait_timeout",
+           "moe_test_dispatch_permute_smooth_wait_timeout")
 
 
 class MoeShape(ctypes.Structure):
@@ -78,9 +79,10 @@ def _load():
     L.moe_combine_bwd.argtypes = [S, P, P, P, P, P, P, P, P, P]
     L.moe_combine_bwd_comm_quant.argtypes = [S, P, P, P, P, P, P, I, P, P, P]
     U64 = ctypes.c_uint64
-    L.moe_test_combine_fwd_wait_timeout.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, U64, I,
-                                                    P]
-    L.moe_test_dispatch_permute_wait_timeout.argtypes = [S, P, P, P, U64, I, P]
+    L.moe_test_combine_fwd_comm_quant_wait_timeout.argtypes = [S, P, P, P, P, P, P, P, P, P, P,
+                                                               P, U64, I, P]
+    L.moe_test_dispatch_permute_smooth_wait_timeout.argtypes = [S, P, P, P, P, P, P, P, U64, I,
+                                                                P]
     L.moe_dispatch_bwd.argtypes = [S, P, P, P, P, P]
     L.moe_dispatch_layout_noalloc.argtypes = [S, P, P, P, P, P, P, P]
     L.moe_layout_noalloc_max_workspace_bytes.argtypes = []
@@ -89,8 +91,8 @@ def _load():
               "moe_combine_bwd", "moe_dispatch_bwd", "moe_dispatch_layout_noalloc",
               "moe_combine_fwd_comm_quant", "moe_dispatch", "moe_combine_bwd_special",
               "moe_dispatch_permute_smooth", "moe_combine_fwd_comm_quant_ws",
-              "moe_combine_bwd_comm_quant", "moe_test_combine_fwd_wait_timeout",
-              "moe_test_dispatch_permute_wait_timeout"):
+              "moe_combine_bwd_comm_quant", "moe_test_combine_fwd_comm_quant_wait_timeout",
+              "moe_test_dispatch_permute_smooth_wait_timeout"):
         getattr(L, n).restype = I
     return L
 
@@ -109,8 +111,9 @@ moe_async_wait_timeouts = _lib.moe_async_wait_timeouts
 moe_combine_fwd = _lib.moe_combine_fwd
 moe_combine_bwd = _lib.moe_combine_bwd
 moe_combine_bwd_comm_quant = _lib.moe_combine_bwd_comm_quant
-moe_test_combine_fwd_wait_timeout = _lib.moe_test_combine_fwd_wait_timeout
-moe_test_dispatch_permute_wait_timeout = _lib.moe_test_dispatch_permute_wait_timeout
+moe_test_combine_fwd_comm_quant_wait_timeout = _lib.moe_test_combine_fwd_comm_quant_wait_timeout
+moe_test_dispatch_permute_smooth_wait_timeout = (
+    _lib.moe_test_dispatch_permute_smooth_wait_timeout)
 moe_dispatch_bwd = _lib.moe_dispatch_bwd
 moe_dispatch_layout_noalloc = _lib.moe_dispatch_layout_noalloc
 moe_combine_fwd_comm_quant = _lib.moe_combine_fwd_comm_quant

@@ -132,7 +132,7 @@ size_t moe_assist_info_elems(const moe_shape* s) {
 
 size_t moe_layout_workspace_bytes(const moe_shape* s) {
   if (s == nullptr || check_shape(s) != MOE_OK) return 0;
-  return moe::layout_workspace_bytes(s->bs, s->num_experts);
+  return moe::layout_workspace_bytes(s->bs, s->num_experts, s->k);
 }
 
 moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,
@@ -146,7 +146,7 @@ moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,
   if ((s->bs > 0 && topk_idx == nullptr) || expert_token_nums == nullptr ||
       ep_send_counts == nullptr || (moe_assist_info_elems(s) > 0 && assist_info == nullptr))
     return MOE_ERR_ARG;
-  const size_t need = moe::layout_workspace_bytes(s->bs, s->num_experts);
+  const size_t need = moe::layout_workspace_bytes(s->bs, s->num_experts, s->k);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return MOE_ERR_CAPACITY;
   if (need > 0 && !aligned16(workspace)) return MOE_ERR_ALIGN;
   moe::LayoutArgs a;
@@ -163,6 +163,7 @@ moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,
   a.assist = assist_info;
   a.dev_status = dev_status;
   a.workspace = workspace;
+  a.workspace_bytes = workspace == nullptr ? 0 : workspace_bytes;
   return cuda_status(moe::launch_layout(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -231,7 +232,8 @@ moe_status moe_dispatch(const moe_shape* s, const int32_t* topk_idx, const uint8
                         size_t workspace_bytes, void* stream) {
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
-  const bool fused = comm_quant_mode == 0 && s->bs <= moe::kLayoutSmallMaxTokens;
+  const bool fused = comm_quant_mode == 0 && s->bs <= moe::kLayoutSmallMaxTokens &&
+                     moe::dispatch_small_fits(s->num_experts, s->k);
   if (!fused) {
     st = moe_dispatch_layout(s, topk_idx, x_active_mask, expert_token_nums, ep_send_counts,
                              assist_info, dev_status, workspace, workspace_bytes, stream);
@@ -259,6 +261,7 @@ moe_status moe_dispatch(const moe_shape* s, const int32_t* topk_idx, const uint8
   a.assist = assist_info;
   a.dev_status = dev_status;
   a.workspace = nullptr;
+  a.workspace_bytes = 0;
   return cuda_status(
       moe::launch_dispatch_small(a, x, expand_x, s->h, static_cast<cudaStream_t>(stream)));
 }
@@ -318,15 +321,11 @@ moe_status moe_combine_fwd_comm_quant_ws(const moe_shape* s, const void* expand_
                          : moe::launch_combine_fwd(a, cs));
 }
 
-moe_status moe_test_combine_fwd_wait_timeout(const moe_shape* s, const void* expand_x,
-                                             const int32_t* topk_idx, const float* topk_weights,
-                                             const int32_t* assist_info,
-                                             const uint8_t* x_active_mask,
-                                             const void* shared_expert_x, const void* ori_x,
-                                             const void* const_alpha_1,
-                                             const void* const_alpha_2, const void* const_v,
-                                             void* out, uint64_t wait_limit_ns,
-                                             int withhold_unit, void* stream) {
+moe_status moe_test_combine_fwd_comm_quant_wait_timeout(
+    const moe_shape* s, const void* expand_x, const int32_t* topk_idx, const float* topk_weights,
+    const int32_t* assist_info, const uint8_t* x_active_mask, const void* shared_expert_x,
+    const void* ori_x, const void* const_alpha_1, const void* const_alpha_2, const void* const_v,
+    void* out, uint64_t wait_limit_ns, int withhold_unit, void* stream) {
   moe::CombineArgs a;
   moe_status st = combine_args(s, expand_x, topk_idx, topk_weights, assist_info, x_active_mask,
                                shared_expert_x, ori_x, const_alpha_1, const_alpha_2, const_v,
@@ -334,36 +333,47 @@ moe_status moe_test_combine_fwd_wait_timeout(const moe_shape* s, const void* exp
   if (st != MOE_OK) return st;
   if (withhold_unit < 0 || wait_limit_ns == 0 || wait_limit_ns > moe::kWaitLimitNs)
     return MOE_ERR_ARG;
-  if (!moe::gather_staged_applies(a)) return MOE_ERR_UNSUPPORTED;
+  if (s->bs == 0 || s->h > 16384) return MOE_ERR_UNSUPPORTED;
+  bool launched = false;
   const moe::WaitCfg wc = {wait_limit_ns, withhold_unit};
-  return cuda_status(moe::launch_gather_staged(a, static_cast<cudaStream_t>(stream), wc));
+  const cudaError_t err = moe::launch_combine_fwd_q8s_test(a, wc, static_cast<cudaStream_t>(stream),
+                                                           &launched);
+  if (!launched) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(err);
 }
 
-moe_status moe_test_dispatch_permute_wait_timeout(const moe_shape* s, const void* x,
-                                                  const int32_t* assist_info, void* expand_x,
-                                                  uint64_t wait_limit_ns, int withhold_unit,
-                                                  void* stream) {
+moe_status moe_test_dispatch_permute_smooth_wait_timeout(
+    const moe_shape* s, const void* x, const int32_t* topk_idx, const int32_t* assist_info,
+    const int32_t* ep_send_counts, const float* smooth_scales, void* expand_x,
+    float* dynamic_scales, uint64_t wait_limit_ns, int withhold_unit, void* stream) {
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
-  if (s->bs > 0 && (x == nullptr || assist_info == nullptr || expand_x == nullptr))
+  if (s->bs > 0 && (x == nullptr || topk_idx == nullptr || assist_info == nullptr ||
+                    ep_send_counts == nullptr || smooth_scales == nullptr ||
+                    expand_x == nullptr || dynamic_scales == nullptr))
     return MOE_ERR_ARG;
-  if (!aligned16(x) || !aligned16(expand_x)) return MOE_ERR_ALIGN;
+  if (!aligned16(x) || !aligned16(expand_x) || !aligned16(smooth_scales)) return MOE_ERR_ALIGN;
+  if (s->h % 16 != 0) return MOE_ERR_ALIGN;
   if (withhold_unit < 0 || wait_limit_ns == 0 || wait_limit_ns > moe::kWaitLimitNs)
     return MOE_ERR_ARG;
-  if (s->bs == 0 || s->h / 8 < moe::kPermuteBulkMinVecs) return MOE_ERR_UNSUPPORTED;
+  if (s->bs == 0 || s->h > 16384) return MOE_ERR_UNSUPPORTED;
   moe::PermuteArgs a;
   a.x = x;
   a.assist = assist_info;
   a.expand_x = expand_x;
-  a.scales = nullptr;
+  a.scales = dynamic_scales;
   a.bs = s->bs;
   a.K = s->k;
   a.H = s->h;
   a.A = s->a_capacity;
   a.dtype = s->dtype;
-  a.quant_mode = 0;
+  a.quant_mode = 2;
   const moe::WaitCfg wc = {wait_limit_ns, withhold_unit};
-  return cuda_status(moe::launch_permute_bulk(a, static_cast<cudaStream_t>(stream), wc));
+  const cudaError_t err = moe::launch_permute_smooth(a, topk_idx, smooth_scales, ep_send_counts,
+                                                     s->num_experts,
+                                                     static_cast<cudaStream_t>(stream), wc, true);
+  if (err == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(err);
 }
 
 moe_status moe_combine_bwd(const moe_shape* s, const void* grad_out, const void* expand_x,

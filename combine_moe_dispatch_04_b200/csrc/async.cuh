@@ -1,6 +1,5 @@
-// Bulk asynchronous copies between global and shared memory (PTX
-// cp.async.bulk, sm_90 and later): global -> shared completed on an mbarrier,
-// shared -> global tracked by bulk async-groups; and bounded mbarrier waits.
+// Bulk asynchronous copies from global into shared memory, completed on an
+// mbarrier (PTX cp.async.bulk / mbarrier, sm_90 and later), and bounded waits.
 // Copies are plain (never multicast); both addresses 16-byte aligned and the
 // size a multiple of 16.
 #pragma once
@@ -83,32 +82,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           "r"(smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
-}
-
-// Bulk copy of `bytes` from this CTA's shared memory to global memory, tracked
-// by this thread's bulk async-groups (plain, never multicast or reducing).
-__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_addr(src)), "r"(bytes)
-               : "memory");
-}
-
-// Closes this thread's current bulk async-group.
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Waits until at most N of this thread's bulk async-groups still read their
-// source (shared memory may then be reused)...
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// ... or are still in progress at all (their writes performed).
-template <int N>
-__device__ __forceinline__ void bulk_wait_group() {
-  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // A wait gives up after about this long (timed with the global nanosecond

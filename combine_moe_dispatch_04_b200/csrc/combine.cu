@@ -81,16 +81,21 @@ struct PairMeta {
 
 // Classifies pair (t, k) (k < K, t < BS). With CHECK_REPEATS the ids of the
 // same token's earlier k are read again (L1) for the repeat check; without it
-// the caller does that check itself.
-template <bool SPECIAL, bool UNIT, bool CHECK_REPEATS = true>
+// the caller does that check itself. With SRC_ROWS (combine_fwd_kernel) a copy
+// or const pair's row is its token t, whose ori_x row it loads together with
+// the routed rows, and a const pair keeps its const row j above the kind's
+// low three bits (kind = kConst | j << 3).
+template <bool SPECIAL, bool UNIT, bool CHECK_REPEATS = true, bool SRC_ROWS = false>
 __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, int k) {
   PairMeta m{kSkip, 0, 1.0f};
   const size_t tk = static_cast<size_t>(t) * a.K + k;
+  // every load first (none depends on another), so the pair costs one round trip
   if (!UNIT) m.w = __ldg(a.weights + tk);
+  const int s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
+  const int32_t* ids = a.topk_idx + static_cast<size_t>(t) * a.K;
+  const int id = SPECIAL ? __ldg(ids + k) : 0;
   if (!pair_active(a.mask, a.mask_ndim, t, k, a.K)) return m;
   if (SPECIAL) {
-    const int32_t* ids = a.topk_idx + static_cast<size_t>(t) * a.K;
-    const int id = __ldg(ids + k);
     if (id < 0 || id >= a.E + a.Z + a.C + a.Q) return m;
     if (CHECK_REPEATS)
       for (int j = 0; j < k; ++j)
@@ -98,10 +103,11 @@ __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, i
     if (id >= a.E) {
       m.kind = id < a.E + a.Z ? kZero : id < a.E + a.Z + a.C ? kCopy : kConst;
       m.row = id - (a.E + a.Z + a.C);
+      if (SRC_ROWS && m.kind == kConst) m.kind = kConst | (m.row << 3);
+      if (SRC_ROWS && m.kind != kZero) m.row = t;
       return m;
     }
   }
-  const int s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
   if (s >= 0) {
     m.kind = kRouted;
     m.row = s;
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
     const int tm = t0 + (lane >> 4), km = lane & 15;
     const bool mine = km < K && tm < a.bs;
     PairMeta m{kSkip, 0, 1.0f};
-    if (mine) m = classify_pair<SPECIAL, UNIT, false>(a, tm, km);
+    if (mine) m = classify_pair<SPECIAL, UNIT, false, true>(a, tm, km);
     if (SPECIAL) {
       // a repeat of an id held by an earlier lane of the same token takes no part
       const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
@@ -178,41 +184,58 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
         kind[u][j] = kSkip;
         wt[u][j] = 1.0f;
         if (j >= K || item >= n) continue;
-        const PairMeta m = classify_pair<SPECIAL, UNIT>(a, item / V, j);
+        const PairMeta m = classify_pair<SPECIAL, UNIT, true, true>(a, item / V, j);
         kind[u][j] = m.kind;
         row[u][j] = m.row;
         wt[u][j] = m.w;
       }
     }
   }
+  // every row a pair reads (a routed row, or the ori_x row of a copy / const
+  // pair) is loaded in one batch, before any is used
+  const uint4* ORI = static_cast<const uint4*>(a.ori_x);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int item = span + u * 32 + lane;
     const int v = item % V;
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-      if (kind[u][j] == kRouted) val[u][j] = ld_nc_v4(Y + static_cast<size_t>(row[u][j]) * V + v);
+    for (int j = 0; j < KMAX; ++j) {
+      const int kd = SPECIAL ? (kind[u][j] & 7) : kind[u][j];
+      if (kd == kRouted)
+        val[u][j] = ld_nc_v4(Y + static_cast<size_t>(row[u][j]) * V + v);
+      else if (SPECIAL && (kd == kCopy || kd == kConst))
+        val[u][j] = ld_nc_v4(ORI + static_cast<size_t>(row[u][j]) * V + v);
+    }
   }
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int item = span + u * 32 + lane;
     if (item >= n) continue;
     const int v = item % V;
-    float ori[8];
-    if (SPECIAL) {
-      bool need = false;
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) need |= kind[u][j] == kCopy || kind[u][j] == kConst;
-      if (need) widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
-    }
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      if (kind[u][j] == kSkip) continue;
+      const int kd = SPECIAL ? (kind[u][j] & 7) : kind[u][j];
+      if (kd == kSkip) continue;
       float m[8];
-      pair_values<T16, SPECIAL>(a, kind[u][j], row[u][j], V, v, val[u][j], ori, m);
+      if (!SPECIAL || kd == kRouted || kd == kCopy) {
+        widen8<T16>(val[u][j], m);
+      } else if (kd == kZero) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+      } else {  // alpha_1 * ori_x + alpha_2 * v, each product and the sum rounded
+        const size_t r = static_cast<size_t>(kind[u][j] >> 3) * V + v;
+        float o[8], a1[8], a2[8], cv[8];
+        widen8<T16>(val[u][j], o);
+        widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + r), a1);
+        widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + r), a2);
+        widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + r), cv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          m[i] = __fadd_rn(__fmul_rn(a1[i], o[i]), __fmul_rn(a2[i], cv[i]));
+      }
       if (UNIT)
         add8_rn(acc, m);
       else
@@ -454,6 +477,7 @@ struct Q8sLayout {  // byte offsets into the dynamic shared memory
 
 template <typename T16, int KMAX, bool SPECIAL, int NBUF>
 __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(CombineArgs a,
+                                                                         WaitCfg wc,
                                                                          unsigned* timeouts) {
   using L = Q8sLayout<KMAX, NBUF>;
   static_assert(NBUF >= 2 && NBUF <= 4, "buffers");
@@ -497,14 +521,16 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
       }
       const unsigned routed = __ballot_sync(0xFFFFFFFFu, pm.kind == kRouted);
       if (q >= NBUF) {  // wait until the consumers have released this buffer
-        const bool ok = mbar_wait_bounded(empty + b, ((q / NBUF) - 1) & 1);
-        if (__any_sync(0xFFFFFFFFu, !ok)) {
-          if (lane == 0) atomicAdd(timeouts, 1u);
-          return;
-        }
+        // (it gives up only after the consumers did: they count the block)
+        const bool ok = mbar_wait_bounded(empty + b, ((q / NBUF) - 1) & 1, wc.limit_ns);
+        if (__any_sync(0xFFFFFFFFu, !ok)) return;
       }
       if (lane < KMAX) meta[b * KMAX + lane] = pm;
       fence_proxy_async_smem();  // the buffer was last read by the consumers' loads
+      if (q == wc.withhold && blockIdx.x == 0) {  // test hook: 16 bytes that never come
+        if (lane == 0) mbar_arrive_expect_tx(full + b, 16u);
+        continue;
+      }
       if (lane == 0) mbar_arrive_expect_tx(full + b, __popc(routed) * static_cast<uint32_t>(V) * 16u);
       __syncwarp();
       if ((routed >> lane) & 1u)
@@ -518,7 +544,7 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
   for (int t = blockIdx.x; t < a.bs; t += stride, ++it) {
     const int b = it % NBUF;
     const int rb = it & 1;
-    const bool ok = mbar_wait_bounded(full + b, (it / NBUF) & 1);
+    const bool ok = mbar_wait_bounded(full + b, (it / NBUF) & 1, wc.limit_ns);
     const PairMeta* pmeta = meta + b * KMAX;
     const uint4* brows = rows + static_cast<size_t>(b) * KMAX * V;
     // this warp's max |y| of every row, the K reductions interleaved
@@ -547,7 +573,8 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
       if (threadIdx.x == 0) {
         atomicAdd(timeouts, 1u);
         for (int q = 0; q < NBUF; ++q)  // copies already started: let them land
-          if (t + q * stride < a.bs) mbar_wait_bounded(full + (it + q) % NBUF, ((it + q) / NBUF) & 1);
+          if (t + q * stride < a.bs && !(it + q == wc.withhold && blockIdx.x == 0))
+            mbar_wait_bounded(full + (it + q) % NBUF, ((it + q) / NBUF) & 1);
       }
       return;
     }
@@ -675,7 +702,7 @@ cudaError_t launch_fwd_t(const CombineArgs& a, cudaStream_t st) {
 constexpr size_t kQ8sSmemBudget = 110 * 1024;
 
 template <typename T16, bool SPECIAL, int KMAX, int NBUF>
-cudaError_t launch_fwd_q8s(const CombineArgs& a, cudaStream_t st) {
+cudaError_t launch_fwd_q8s(const CombineArgs& a, const WaitCfg& wc, cudaStream_t st) {
   constexpr auto kernel = combine_fwd_q8s_kernel<T16, KMAX, SPECIAL, NBUF>;
   const int V = a.H / kVecElems;
   const size_t smem = Q8sLayout<KMAX, NBUF>::bytes(V);
@@ -689,22 +716,33 @@ cudaError_t launch_fwd_q8s(const CombineArgs& a, cudaStream_t st) {
   if (err != cudaSuccess) return err;
   const int cap = sm_count() * (per_sm > 0 ? per_sm : 1);
   const int blocks = a.bs < cap ? a.bs : cap;
-  return launch_pdl(kernel, dim3(blocks), dim3(kQ8sThreads), smem, st, a, timeouts);
+  return launch_pdl(kernel, dim3(blocks), dim3(kQ8sThreads), smem, st, a, wc, timeouts);
 }
 
 // Staged kernel with three buffers when they fit the budget, else two; false
 // when even two do not fit (the caller then takes the two-pass kernel).
 template <typename T16, bool SPECIAL, int KMAX>
-bool try_launch_fwd_q8s(const CombineArgs& a, cudaStream_t st, cudaError_t* err) {
+bool try_launch_fwd_q8s(const CombineArgs& a, const WaitCfg& wc, cudaStream_t st,
+                        cudaError_t* err) {
   const int V = a.H / kVecElems;
   if (Q8sLayout<KMAX, 3>::bytes(V) <= kQ8sSmemBudget) {
-    *err = launch_fwd_q8s<T16, SPECIAL, KMAX, 3>(a, st);
+    *err = launch_fwd_q8s<T16, SPECIAL, KMAX, 3>(a, wc, st);
     return true;
   }
   if (Q8sLayout<KMAX, 2>::bytes(V) <= kQ8sSmemBudget) {
-    *err = launch_fwd_q8s<T16, SPECIAL, KMAX, 2>(a, st);
+    *err = launch_fwd_q8s<T16, SPECIAL, KMAX, 2>(a, wc, st);
     return true;
   }
+  return false;
+}
+
+// The staged single-pass kernel when the shape allows it (false otherwise).
+template <typename T16, bool SPECIAL>
+bool try_launch_q8s_k(const CombineArgs& a, const WaitCfg& wc, cudaStream_t st,
+                      cudaError_t* err) {
+  if (a.K <= 2) return try_launch_fwd_q8s<T16, SPECIAL, 2>(a, wc, st, err);
+  if (a.K <= 4) return try_launch_fwd_q8s<T16, SPECIAL, 4>(a, wc, st, err);
+  if (a.K <= 8) return try_launch_fwd_q8s<T16, SPECIAL, 8>(a, wc, st, err);
   return false;
 }
 
@@ -712,9 +750,7 @@ template <typename T16, bool SPECIAL>
 cudaError_t launch_fwd_q8_t(const CombineArgs& a, cudaStream_t st) {
   const int V = a.H / kVecElems;
   cudaError_t err = cudaSuccess;
-  if (a.K <= 2 && try_launch_fwd_q8s<T16, SPECIAL, 2>(a, st, &err)) return err;
-  if (a.K > 2 && a.K <= 4 && try_launch_fwd_q8s<T16, SPECIAL, 4>(a, st, &err)) return err;
-  if (a.K > 4 && a.K <= 8 && try_launch_fwd_q8s<T16, SPECIAL, 8>(a, st, &err)) return err;
+  if (try_launch_q8s_k<T16, SPECIAL>(a, kProductWaits, st, &err)) return err;
   const int threads = V < 256 ? (V + 31) / 32 * 32 : 256;
   const int cap = sm_count() * (2048 / threads);
   const int blocks = a.bs < cap ? a.bs : cap;
@@ -770,11 +806,23 @@ cudaError_t launch_fwd_rt(const CombineArgs& a, const int32_t* send, float2* rsc
 
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
-  if (gather_staged_applies(a)) return launch_gather_staged(a, st);
   return a.dtype == MOE_BF16 ? launch_fwd_t<Bf16>(a, st) : launch_fwd_t<Fp16>(a, st);
 }
 
 size_t combine_q8_workspace_bytes(int A) { return static_cast<size_t>(A) * sizeof(float2); }
+
+cudaError_t launch_combine_fwd_q8s_test(const CombineArgs& a, const WaitCfg& wc, cudaStream_t st,
+                                        bool* launched) {
+  cudaError_t err = cudaSuccess;
+  const bool special = a.Z + a.C + a.Q > 0;
+  if (a.dtype == MOE_BF16)
+    *launched = special ? try_launch_q8s_k<Bf16, true>(a, wc, st, &err)
+                        : try_launch_q8s_k<Bf16, false>(a, wc, st, &err);
+  else
+    *launched = special ? try_launch_q8s_k<Fp16, true>(a, wc, st, &err)
+                        : try_launch_q8s_k<Fp16, false>(a, wc, st, &err);
+  return err;
+}
 
 cudaError_t launch_combine_fwd_q8(const CombineArgs& a, const int32_t* send, void* workspace,
                                   cudaStream_t st) {

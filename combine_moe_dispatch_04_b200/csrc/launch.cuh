@@ -20,13 +20,14 @@ struct LayoutArgs {
   int32_t* assist;
   uint32_t* dev_status;  // may be null
   void* workspace;
+  size_t workspace_bytes;
 };
 
 // Tokens per CTA in the multi-CTA layout, and the largest BS of the one-CTA layout.
 constexpr int kLayoutTileTokens = 256;
 constexpr int kLayoutSmallMaxTokens = 1024;
 
-size_t layout_workspace_bytes(int bs, int E);
+size_t layout_workspace_bytes(int bs, int E, int K);
 cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st);
 
 struct PermuteArgs {
@@ -37,21 +38,16 @@ struct PermuteArgs {
   int bs, K, H, A, dtype, quant_mode;
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
-// The bulk-copy permute (plain copy) with the given waits (test hook).
-cudaError_t launch_permute_bulk(const PermuteArgs& a, cudaStream_t st,
-                                const WaitCfg& wc = kProductWaits);
-// Rows of at least this many 16-byte vectors take the bulk-copy permute.
-#ifndef MOE_PERMUTE_BULK_MIN_VECS
-#define MOE_PERMUTE_BULK_MIN_VECS 32
-#endif
-constexpr int kPermuteBulkMinVecs = MOE_PERMUTE_BULK_MIN_VECS;
 // int8 permute of x[t] * smooth[e] per slot (H <= 16384, multiple of 16; smooth 16-byte
 // aligned); reads the total R from send[E].
 cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
                                   const float* smooth, const int32_t* send, int E,
-                                  cudaStream_t st);
+                                  cudaStream_t st, const WaitCfg& wc = kProductWaits,
+                                  bool staged_only = false);
 
-// Layout and the plain (no quantisation) permute in one launch, BS <= kLayoutSmallMaxTokens.
+// Layout and the plain (no quantisation) permute in one launch, BS <= kLayoutSmallMaxTokens
+// and shared memory for E experts' masks (dispatch_small_fits).
+bool dispatch_small_fits(int E, int K);
 cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
                                   cudaStream_t st);
 
@@ -71,21 +67,15 @@ struct CombineArgs {
   int bs, K, H, A, E, Z, C, Q, dtype;
 };
 cudaError_t launch_combine_fwd(const CombineArgs& a, cudaStream_t st);
-// The same gather (combine forward, or dispatch backward with weights == null)
-// with each token's rows staged in shared memory by bulk copies (gather.cu);
-// launch_combine_fwd takes it for rows of at least kGatherStagedMinVecs vectors.
-#ifndef MOE_GATHER_STAGED_MIN_VECS
-#define MOE_GATHER_STAGED_MIN_VECS 32
-#endif
-constexpr int kGatherStagedMinVecs = MOE_GATHER_STAGED_MIN_VECS;
-bool gather_staged_applies(const CombineArgs& a);
-cudaError_t launch_gather_staged(const CombineArgs& a, cudaStream_t st,
-                                 const WaitCfg& wc = kProductWaits);
 // comm_quant_mode 2: every routed row through the per-row int8 round trip (H <= 16384).
 // With a workspace of combine_q8_workspace_bytes(A) bytes and the total R in send[E], shapes
 // with routed pairs only take two passes (per-row scales, then the gather); otherwise the
 // staged kernel runs and the workspace is not touched.
 size_t combine_q8_workspace_bytes(int A);
+// The staged single-pass int8 combine with the given waits (test hook); *launched is
+// false when the shape takes another kernel.
+cudaError_t launch_combine_fwd_q8s_test(const CombineArgs& a, const WaitCfg& wc, cudaStream_t st,
+                                        bool* launched);
 cudaError_t launch_combine_fwd_q8(const CombineArgs& a, const int32_t* send, void* workspace,
                                   cudaStream_t st);
 

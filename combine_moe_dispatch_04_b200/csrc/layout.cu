@@ -168,33 +168,66 @@ __device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t ran
 
 __host__ __device__ constexpr int cluster_stride(int E) { return E | 1; }
 
-__host__ __device__ constexpr size_t cluster_smem_bytes(int E, int tpt) {
-  return static_cast<size_t>(tpt) * 32 * cluster_stride(E) * 4 +
-         (static_cast<size_t>(tpt) * 32 * cluster_stride(E) * 2 + 3) / 4 * 4 +
-         static_cast<size_t>(E) * 8;
+// Per (sub-block, warp, expert): the lane mask of the warp's tokens routed to
+// the expert (x) and the number of the CTA's earlier tokens routed there (y).
+// One 8-byte entry, so a pair's rank is one shared-memory load.
+struct alignas(8) MaskPre {
+  uint32_t mask;
+  uint32_t pre;
+};
+// Per expert: the first slot of this CTA's pairs (x) and their start in the
+// CTA's expert-ordered pair list (y).
+struct alignas(8) BaseOfs {
+  int first;
+  int lofs;
+};
+
+// mp[tpt][nt / 32][S], bo[E], tot[E] (cluster kernel and fused dispatch, nt
+// threads); the cluster kernel also keeps its pairs in expert order,
+// ltk[tpt * nt * K].
+__host__ __device__ constexpr size_t cluster_smem_bytes(int E, int tpt, int nt = 1024) {
+  return static_cast<size_t>(tpt) * (nt / 32) * cluster_stride(E) * sizeof(MaskPre) +
+         static_cast<size_t>(E) * (4 + sizeof(BaseOfs));
+}
+__host__ __device__ constexpr size_t cluster_kernel_smem_bytes(int E, int tpt, int K, int nt) {
+  return cluster_smem_bytes(E, tpt, nt) + static_cast<size_t>(tpt) * nt * K * 4;
 }
 
-// Counts this CTA's tokens [t0, t0 + TPT * 1024) (one per thread and sub-block)
+// The slot -> pair half of assist_info for a block's routed pairs, written run
+// by run: the block's pairs of expert e take the consecutive slots
+// [first[e], first[e] + count[e]), and ltk[lofs[e] + r] holds t * K + k of the
+// one of rank r, so every warp (experts w, w + 32, ...) writes contiguous ints.
+__device__ __forceinline__ void write_runs(const LayoutArgs& a, const int* first, const int* count,
+                                           const int* lofs, const int* ltk, int stride) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  for (int ex = warp; ex < a.E; ex += nwarps) {
+    const int n = count[ex], f = first[ex * stride], l = lofs[ex * stride];
+    for (int j = lane; j < n; j += 32) a.assist[f + j] = ltk[l + j];
+  }
+}
+
+// Counts this CTA's tokens [t0, t0 + TPT * NT) (one per thread and sub-block)
 // into the lane masks, then per expert the exclusive prefix of the popcounts
-// over (sub-block, warp) into pre and the CTA's total into tot (warp w scans
-// the columns w, w + 32, ...; lane = warp of the column). words must be zero
-// on entry; e receives each token's routed experts (-1 elsewhere) and the
+// over (sub-block, warp) into mp[].pre and the CTA's total into tot (warp w
+// scans the columns w, w + NW, ...; lane = warp of the column). mp must be
+// zero on entry; e receives each token's routed experts (-1 elsewhere) and the
 // status bits are ORed into *status.
-template <int KM, int TPT>
-__device__ __forceinline__ void cta_count_scan(const LayoutArgs& a, int t0, int S,
-                                               uint32_t* words, uint16_t* pre, int* tot,
-                                               uint32_t* status, int (&e)[TPT][KM]) {
+template <int KM, int TPT, int NT>
+__device__ __forceinline__ void cta_count_scan(const LayoutArgs& a, int t0, int S, MaskPre* mp,
+                                               int* tot, uint32_t* status, int (&e)[TPT][KM]) {
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t st = 0;
 #pragma unroll
   for (int i = 0; i < TPT; ++i) {
-    const int t = t0 + i * 1024 + threadIdx.x;
+    const int t = t0 + i * NT + threadIdx.x;
     if (t < a.bs) {
       st |= classify_row<KM>(a, t, e[i]);
       const uint32_t bit = 1u << lane;
 #pragma unroll
       for (int k = 0; k < KM; ++k)
-        if (k < a.K && e[i][k] >= 0) atomicOr(&words[(i * 32 + warp) * S + e[i][k]], bit);
+        if (k < a.K && e[i][k] >= 0) atomicOr(&mp[(i * NW + warp) * S + e[i][k]].mask, bit);
     } else {
 #pragma unroll
       for (int k = 0; k < KM; ++k) e[i][k] = -1;
@@ -202,54 +235,46 @@ __device__ __forceinline__ void cta_count_scan(const LayoutArgs& a, int t0, int 
   }
   if (st) atomicOr(status, st);
   __syncthreads();
-  for (int ex = warp; ex < a.E; ex += 32) {
+  for (int ex = warp; ex < a.E; ex += NW) {
     int carry = 0;
 #pragma unroll
     for (int i = 0; i < TPT; ++i) {
-      const int c = __popc(words[(i * 32 + lane) * S + ex]);
+      const int c = lane < NW ? __popc(mp[(i * NW + lane) * S + ex].mask) : 0;
       int inc = c;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int n = __shfl_up_sync(0xFFFFFFFFu, inc, d);
         if (lane >= d) inc += n;
       }
-      pre[(i * 32 + lane) * S + ex] = static_cast<uint16_t>(carry + inc - c);
+      if (lane < NW) mp[(i * NW + lane) * S + ex].pre = static_cast<uint32_t>(carry + inc - c);
       carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
     }
     if (lane == 0) tot[ex] = carry;
   }
 }
 
-// Slot of each routed pair of token t (sub-block i of this CTA, its own lane).
-template <int KM>
-__device__ __forceinline__ void cta_slots(const LayoutArgs& a, int i, int S, const uint32_t* words,
-                                          const uint16_t* pre, const int* base,
-                                          const int (&e)[KM], int (&slot)[KM]) {
-  const int row = (i * 32 + (threadIdx.x >> 5)) * S;
-#pragma unroll
-  for (int k = 0; k < KM; ++k) {
-    const int ex = e[k];
-    slot[k] = (k < a.K && ex >= 0)
-                  ? base[ex] + pre[row + ex] + __popc(words[row + ex] & lanemask_lt())
-                  : -1;
-  }
+// Rank among the CTA's pairs of expert ex of this thread's token (sub-block i).
+template <int NT>
+__device__ __forceinline__ int cta_rank(const MaskPre* mp, int i, int S, int ex) {
+  const MaskPre m = mp[(i * (NT / 32) + (threadIdx.x >> 5)) * S + ex];
+  return static_cast<int>(m.pre) + __popc(m.mask & lanemask_lt());
 }
 
-template <int KM, int TPT>
-__global__ void __launch_bounds__(1024, 1) layout_cluster_kernel(LayoutArgs a) {
+template <int KM, int TPT, int NT>
+__global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status, status_all;
   const int E = a.E;
   const int S = cluster_stride(E);
-  uint32_t* words = reinterpret_cast<uint32_t*>(smem);
-  uint16_t* pre = reinterpret_cast<uint16_t*>(smem + static_cast<size_t>(TPT) * 32 * S * 4);
-  int* tot = reinterpret_cast<int*>(smem + static_cast<size_t>(TPT) * 32 * S * 4 +
-                                    (static_cast<size_t>(TPT) * 32 * S * 2 + 3) / 4 * 4);
-  int* base = tot + E;
+  MaskPre* mp = reinterpret_cast<MaskPre*>(smem);
+  BaseOfs* bo = reinterpret_cast<BaseOfs*>(smem + static_cast<size_t>(TPT) * (NT / 32) * S *
+                                                      sizeof(MaskPre));
+  int* tot = reinterpret_cast<int*>(bo + E);
+  int* ltk = tot + E;
   const uint32_t rank = cluster_ctarank(), cs = cluster_nctarank();
   pdl_trigger();
-  for (int i = threadIdx.x; i < TPT * 32 * S; i += blockDim.x) words[i] = 0;
+  for (int i = threadIdx.x; i < TPT * (NT / 32) * S; i += NT) mp[i] = MaskPre{0u, 0u};
   if (threadIdx.x == 0) {
     status = 0;
     status_all = 0;
@@ -257,9 +282,9 @@ __global__ void __launch_bounds__(1024, 1) layout_cluster_kernel(LayoutArgs a) {
   __syncthreads();
   pdl_wait();
 
-  const int t0 = static_cast<int>(rank) * TPT * 1024;
+  const int t0 = static_cast<int>(rank) * TPT * NT;
   int e[TPT][KM];
-  cta_count_scan<KM, TPT>(a, t0, S, words, pre, tot, &status, e);
+  cta_count_scan<KM, TPT, NT>(a, t0, S, mp, tot, &status, e);
   __syncwarp();
   cluster_arrive_release();  // tot and status are published to the cluster
   cluster_wait_acquire();
@@ -278,10 +303,13 @@ __global__ void __launch_bounds__(1024, 1) layout_cluster_kernel(LayoutArgs a) {
   __syncwarp();
   cluster_arrive_release();  // done reading the other CTAs' shared memory
   if (cst) atomicOr(&status_all, cst);
-  int total;
+  int total, cta_total;
   const int excl = block_exclusive_scan(threadIdx.x < E ? grand : 0, warp_sums, &total);
+  __syncthreads();  // every thread has read warp_sums before the second scan rewrites it
+  const int lexcl = block_exclusive_scan(threadIdx.x < E ? tot[threadIdx.x] : 0, warp_sums,
+                                         &cta_total);
   if (threadIdx.x < E) {
-    base[threadIdx.x] = excl + before;
+    bo[threadIdx.x] = BaseOfs{excl + before, lexcl};
     if (rank == 0) {
       a.expert_token_nums[threadIdx.x] = grand;
       a.ep_send_counts[threadIdx.x] = excl;
@@ -292,14 +320,30 @@ __global__ void __launch_bounds__(1024, 1) layout_cluster_kernel(LayoutArgs a) {
     a.ep_send_counts[E] = total;
     if (a.dev_status) *a.dev_status = status_all;
   }
+  // pair -> slot per token (contiguous per thread); each pair's t * K + k into
+  // the block's expert-ordered list for the slot -> pair half
+  const size_t A = static_cast<size_t>(a.A);
 #pragma unroll
   for (int i = 0; i < TPT; ++i) {
-    const int t = t0 + i * 1024 + threadIdx.x;
+    const int t = t0 + i * NT + threadIdx.x;
     if (t >= a.bs) continue;
-    int slot[KM];
-    cta_slots<KM>(a, i, S, words, pre, base, e[i], slot);
-    write_slots<KM>(a, t, e[i], slot);
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      if (k >= a.K) continue;
+      const int ex = e[i][k];
+      const int tk = t * a.K + k;
+      int slot = -1;
+      if (ex >= 0) {
+        const int r = cta_rank<NT>(mp, i, S, ex);
+        const BaseOfs b = bo[ex];
+        slot = b.first + r;
+        ltk[b.lofs + r] = tk;
+      }
+      a.assist[A + tk] = slot;
+    }
   }
+  __syncthreads();
+  write_runs(a, &bo[0].first, tot, &bo[0].lofs, ltk, 2);
   for (int s = total + static_cast<int>(rank * blockDim.x + threadIdx.x); s < a.A;
        s += static_cast<int>(cs * blockDim.x))
     a.assist[s] = -1;
@@ -313,7 +357,7 @@ __global__ void __launch_bounds__(1024, 1) layout_cluster_kernel(LayoutArgs a) {
 // would (the ids are at most 64 KB and sit in L2), CTA 0 alone writes the
 // layout's outputs, and CTA c copies the rows of tokens [c * per, (c+1) * per)
 // to their slots: one thread per 16-byte vector, read once, stored K times.
-// Dynamic shared memory: words[32][S], pre[32][S] uint16, tot[E], base[E].
+// Dynamic shared memory: mp[32][S], bo[E], tot[E].
 template <int KM>
 __global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, const uint4* x,
                                                                  uint4* expand_x, int V, int per) {
@@ -323,25 +367,23 @@ __global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, c
   __shared__ int slot_sh[kLayoutSmallMaxTokens / 8][KM];  // slots of this CTA's tokens
   const int E = a.E;
   const int S = cluster_stride(E);
-  uint32_t* words = reinterpret_cast<uint32_t*>(smem);
-  uint16_t* pre = reinterpret_cast<uint16_t*>(smem + static_cast<size_t>(32) * S * 4);
-  int* tot = reinterpret_cast<int*>(smem + static_cast<size_t>(32) * S * 4 +
-                                    (static_cast<size_t>(32) * S * 2 + 3) / 4 * 4);
-  int* base = tot + E;
+  MaskPre* mp = reinterpret_cast<MaskPre*>(smem);
+  BaseOfs* bo = reinterpret_cast<BaseOfs*>(smem + static_cast<size_t>(32) * S * sizeof(MaskPre));
+  int* tot = reinterpret_cast<int*>(bo + E);
   const bool writer = blockIdx.x == 0;
   pdl_trigger();
-  for (int i = threadIdx.x; i < 32 * S; i += blockDim.x) words[i] = 0;
+  for (int i = threadIdx.x; i < 32 * S; i += blockDim.x) mp[i] = MaskPre{0u, 0u};
   if (threadIdx.x == 0) status = 0;
   __syncthreads();
   pdl_wait();
   int e[1][KM];
-  cta_count_scan<KM, 1>(a, 0, S, words, pre, tot, &status, e);
+  cta_count_scan<KM, 1, 1024>(a, 0, S, mp, tot, &status, e);
   __syncthreads();
   const int cnt = threadIdx.x < E ? tot[threadIdx.x] : 0;
   int total;
   const int excl = block_exclusive_scan(cnt, warp_sums, &total);
   if (threadIdx.x < E) {
-    base[threadIdx.x] = excl;
+    bo[threadIdx.x] = BaseOfs{excl, 0};
     if (writer) {
       a.expert_token_nums[threadIdx.x] = cnt;
       a.ep_send_counts[threadIdx.x] = excl;
@@ -353,7 +395,10 @@ __global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, c
   const int t0 = blockIdx.x * per;
   if (t < a.bs) {
     int slot[KM];
-    cta_slots<KM>(a, 0, S, words, pre, base, e[0], slot);
+#pragma unroll
+    for (int k = 0; k < KM; ++k)
+      slot[k] = (k < a.K && e[0][k] >= 0) ? bo[e[0][k]].first + cta_rank<1024>(mp, 0, S, e[0][k])
+                                          : -1;
     if (writer) write_slots<KM>(a, t, e[0], slot);
     if (t >= t0 && t < t0 + per) {
 #pragma unroll
@@ -520,8 +565,10 @@ __device__ __forceinline__ void tile_slots(const LayoutArgs& a, int T, int tile,
   *grand_out = grand;
 }
 
-// Phase 3 as its own launch: every tile's slots, and -1 for the unused
-// slots [R, A).
+// Phase 3 as its own launch: every tile's slots (the slot -> pair half written
+// run by run, see write_runs), and -1 for the unused slots [R, A). Dynamic
+// shared memory: tile_slots' words[kTileWarps][E], base[E], total[E], then
+// cnt[E], lofs[E] and ltk[kLayoutTileTokens * K].
 template <int KM>
 __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(LayoutArgs a, int T) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -529,11 +576,45 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
   __shared__ uint32_t status;
   pdl_trigger();
   pdl_wait();
+  const int E = a.E;
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem);
+  int* base = reinterpret_cast<int*>(words + kTileWarps * E);
+  int* cnt = base + 2 * E;
+  int* lofs = cnt + E;
+  int* ltk = lofs + E;
   int e[KM], slot[KM], grand;
-  tile_slots<KM>(a, T, blockIdx.x, blockIdx.x == 0, reinterpret_cast<uint32_t*>(smem), warp_sums,
-                 &status, e, slot, &grand);
+  tile_slots<KM>(a, T, blockIdx.x, blockIdx.x == 0, words, warp_sums, &status, e, slot, &grand);
+  // the tile's own count per expert and their exclusive scan (each thread a run of experts)
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
+  int run = 0;
+  for (int ex = e0; ex < e1; ++ex) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kTileWarps; ++w) c += __popc(words[w * E + ex]);
+    cnt[ex] = c;
+    run += c;
+  }
+  int tile_total;
+  int off = block_exclusive_scan(run, warp_sums, &tile_total);
+  for (int ex = e0; ex < e1; ++ex) {
+    lofs[ex] = off;
+    off += cnt[ex];
+  }
+  __syncthreads();
   const int t = blockIdx.x * kLayoutTileTokens + threadIdx.x;
-  if (t < a.bs) write_slots<KM>(a, t, e, slot);
+  if (t < a.bs) {
+    const size_t A = static_cast<size_t>(a.A);
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      if (k >= a.K) continue;
+      const int tk = t * a.K + k;
+      if (e[k] >= 0) ltk[lofs[e[k]] + slot[k] - base[e[k]]] = tk;
+      a.assist[A + tk] = e[k] >= 0 ? slot[k] : -1;
+    }
+  }
+  __syncthreads();
+  write_runs(a, base, cnt, lofs, ltk, 1);
   for (int s = grand + blockIdx.x * blockDim.x + threadIdx.x; s < a.A;
        s += gridDim.x * blockDim.x)
     a.assist[s] = -1;
@@ -559,32 +640,48 @@ cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* ex
                     static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
 }
 
-// Largest BS of the cluster layout (8 CTAs of 1024 threads, two tokens each),
-// and its shared memory limit.
+// The cluster layout: CS <= 16 CTAs of NT threads, one token per thread: 512
+// threads per CTA up to 8192 tokens (and E <= 512), so that up to 16 SMs share
+// the work, else 1024.
 #ifndef MOE_LAYOUT_CLUSTER_MAX_TOKENS
-#define MOE_LAYOUT_CLUSTER_MAX_TOKENS (8 * 2 * 1024)
+#define MOE_LAYOUT_CLUSTER_MAX_TOKENS (16 * 1024)
 #endif
 constexpr int kClusterMaxTokens = MOE_LAYOUT_CLUSTER_MAX_TOKENS;
 constexpr size_t kClusterSmemMax = 210 * 1024;
 
-int cluster_tpt(int bs) { return bs <= 8 * 1024 ? 1 : 2; }
+// The kernel gives each expert one thread (its grand total, scan entry and first
+// slot), so E <= threads: 512 threads only for E <= 512.
+int cluster_threads(int bs, int E) { return (bs <= 16 * 512 && E <= 512) ? 512 : 1024; }
 
-bool cluster_layout_applies(int bs, int E) {
-  return bs <= kClusterMaxTokens && cluster_smem_bytes(E, cluster_tpt(bs)) <= kClusterSmemMax;
+// Workspace of the tiled path: tile counts, expert totals, tile status words.
+size_t tiled_workspace_bytes(int bs, int E) {
+  const size_t T = (static_cast<size_t>(bs) + kLayoutTileTokens - 1) / kLayoutTileTokens;
+  return T * static_cast<size_t>(E) * 4 + static_cast<size_t>(E) * 4 + T * 4;
+}
+int cluster_tpt(int bs) { return 1; }
+
+bool cluster_layout_applies(int bs, int E, int K) {
+  const int nt = cluster_threads(bs, E);
+  return bs <= kClusterMaxTokens && E <= nt &&
+         cluster_kernel_smem_bytes(E, cluster_tpt(bs), K, nt) <= kClusterSmemMax;
 }
 
-template <int KM, int TPT>
-cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st) {
-  constexpr auto kernel = layout_cluster_kernel<KM, TPT>;
-  const size_t smem = cluster_smem_bytes(a.E, TPT);
+template <int KM, int TPT, int NT>
+cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st, bool* fits) {
+  constexpr auto kernel = layout_cluster_kernel<KM, TPT, NT>;
+  const size_t smem = cluster_kernel_smem_bytes(a.E, TPT, a.K, NT);
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  int cs = (a.bs + TPT * 1024 - 1) / (TPT * 1024);
+  int cs = (a.bs + TPT * NT - 1) / (TPT * NT);
   if (cs < 1) cs = 1;
+  if (cs > 8) {  // clusters of more than 8 CTAs are opted into per kernel
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs);
-  cfg.blockDim = dim3(1024);
+  cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -596,27 +693,58 @@ cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  // a cluster this device cannot hold at all: the tiled path instead (host-side
+  // query, before any launch)
+  int clusters = 0;
+  cfg.numAttrs = 1;
+  err = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
+  cfg.numAttrs = 2;
+  if (err != cudaSuccess || clusters < 1) {
+    cudaGetLastError();
+    *fits = false;
+    return cudaSuccess;
+  }
+  *fits = true;
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 template <int KM>
 cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t st) {
-  if (cluster_layout_applies(a.bs, a.E))
-    return cluster_tpt(a.bs) == 1 ? launch_layout_cluster<KM, 1>(a, st)
-                                  : launch_layout_cluster<KM, 2>(a, st);
+  if (cluster_layout_applies(a.bs, a.E, a.K)) {
+    bool fits = false;
+    const cudaError_t err = cluster_threads(a.bs, a.E) == 512
+                                ? launch_layout_cluster<KM, 1, 512>(a, st, &fits)
+                                : launch_layout_cluster<KM, 1, 1024>(a, st, &fits);
+    if (err != cudaSuccess || fits) return err;
+    // a device that cannot hold the cluster: the tiled path, if given its workspace
+    if (a.workspace == nullptr || a.workspace_bytes < tiled_workspace_bytes(a.bs, a.E))
+      return cudaErrorInvalidClusterSize;
+  }
   const int T = (a.bs + kLayoutTileTokens - 1) / kLayoutTileTokens;
   const size_t smem_count = static_cast<size_t>(kTileWarps) * a.E * sizeof(uint32_t);
-  const size_t smem_scatter = smem_count + 2u * a.E * sizeof(int);
+  const size_t smem_scatter = smem_count + 4u * a.E * sizeof(int) +
+                              static_cast<size_t>(kLayoutTileTokens) * a.K * sizeof(int);
   cudaError_t err = launch_pdl(layout_count_kernel<KM>, dim3(T), dim3(kLayoutTileTokens),
                                smem_count, st, a, T);
   if (err != cudaSuccess) return err;
   err = launch_pdl(layout_colscan_kernel, dim3((a.E + 31) / 32), dim3(1024), 0, st, a, T);
   if (err != cudaSuccess) return err;
+  if (smem_scatter > 48 * 1024) {  // E = 1024 with K = 16: up to 64 KB
+    err = cudaFuncSetAttribute(layout_scatter_kernel<KM>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_scatter));
+    if (err != cudaSuccess) return err;
+  }
   return launch_pdl(layout_scatter_kernel<KM>, dim3(T), dim3(kLayoutTileTokens), smem_scatter,
                     st, a, T);
 }
 
 }  // namespace
+
+bool dispatch_small_fits(int E, int K) {
+  const size_t stat = static_cast<size_t>(kLayoutSmallMaxTokens / 8) * K * 4 + 1024;
+  return cluster_smem_bytes(E, 1) + stat <= kClusterSmemMax;
+}
 
 cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expand_x, int H,
                                   cudaStream_t st) {
@@ -626,10 +754,8 @@ cudaError_t launch_dispatch_small(const LayoutArgs& a, const void* x, void* expa
   return launch_dispatch_small_k<16>(a, x, expand_x, H, st);
 }
 
-size_t layout_workspace_bytes(int bs, int E) {
-  if (cluster_layout_applies(bs, E)) return 0;
-  const size_t T = (static_cast<size_t>(bs) + kLayoutTileTokens - 1) / kLayoutTileTokens;
-  return T * static_cast<size_t>(E) * 4 + static_cast<size_t>(E) * 4 + T * 4;
+size_t layout_workspace_bytes(int bs, int E, int K) {
+  return cluster_layout_applies(bs, E, K) ? 0 : tiled_workspace_bytes(bs, E);
 }
 
 cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t st) {

@@ -43,95 +43,6 @@ __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
   }
 }
 
-// The plain copy on the bulk-copy engine: each warp takes a contiguous range of
-// units (one column chunk of one token's row) and keeps kPbStages of them in
-// flight. Lane 0 brings a unit's chunk into the warp's stage buffer with one
-// bulk copy (global -> shared, on the buffer's mbarrier); once it has landed,
-// lane k < K copies the buffer to slot(t, k) with one bulk copy (shared ->
-// global, its own bulk async-group). A buffer is refilled only after every
-// lane's stores from it have finished reading it (wait_group.read). x is read
-// once, and the K-fold write fan-out costs K bulk operations per unit instead
-// of K 16-byte stores per thread. Every wait is bounded; a warp that gives up
-// counts itself in *timeouts, lets its started copies land and returns.
-constexpr int kPbWarps = 4;
-constexpr int kPbStages = 4;
-
-__host__ __device__ constexpr size_t pb_warp_bytes(int cvec) {
-  return 128 + static_cast<size_t>(kPbStages) * cvec * 16;
-}
-
-__global__ void __launch_bounds__(32 * kPbWarps) permute_bulk_kernel(
-    const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
-    int bs, int K, int V, int A, int nchunks, int cvec, WaitCfg wc, unsigned* timeouts) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned char* wbase = smem + static_cast<size_t>(warp) * pb_warp_bytes(cvec);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase);
-  uint4* stages = reinterpret_cast<uint4*>(wbase + 128);
-  if (lane == 0) {
-    for (int b = 0; b < kPbStages; ++b) mbar_init(bars + b, 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
-  pdl_trigger();
-  pdl_wait();
-  const long long units = static_cast<long long>(bs) * nchunks;
-  const long long nw = static_cast<long long>(gridDim.x) * kPbWarps;
-  const long long gw = static_cast<long long>(blockIdx.x) * kPbWarps + warp;
-  const long long per = (units + nw - 1) / nw;
-  const long long u0 = gw * per < units ? gw * per : units;
-  const long long u1 = u0 + per < units ? u0 + per : units;
-  const int32_t* slots = assist + static_cast<size_t>(A);
-
-  // test hook: the first warp's unit withhold waits for 16 bytes that never come
-  const long long held = (gw == 0 && wc.withhold >= 0) ? u0 + wc.withhold : -1;
-  auto issue = [&](long long u, int b) {  // lane 0: unit u into buffer b
-    if (u == held) {
-      mbar_arrive_expect_tx(bars + b, 16u);
-      return;
-    }
-    const int t = static_cast<int>(u / nchunks);
-    const int v0 = static_cast<int>(u - static_cast<long long>(t) * nchunks) * cvec;
-    const uint32_t bytes = static_cast<uint32_t>(min(cvec, V - v0)) * 16u;
-    mbar_arrive_expect_tx(bars + b, bytes);
-    bulk_g2s(stages + static_cast<size_t>(b) * cvec, x + static_cast<size_t>(t) * V + v0, bytes,
-             bars + b);
-  };
-  if (lane == 0)
-    for (int p = 0; p < kPbStages - 1; ++p)
-      if (u0 + p < u1) issue(u0 + p, p);
-  int next_slot = -1;
-  if (u0 < u1 && lane < K) next_slot = __ldg(slots + (u0 / nchunks) * K + lane);
-  int i = 0;
-  for (long long u = u0; u < u1; ++u, ++i) {
-    const int b = i % kPbStages;
-    const int slot = next_slot;
-    if (u + 1 < u1 && lane < K) next_slot = __ldg(slots + ((u + 1) / nchunks) * K + lane);
-    const bool ok = mbar_wait_bounded(bars + b, (i / kPbStages) & 1, wc.limit_ns);
-    if (!__all_sync(0xFFFFFFFFu, ok)) {
-      if (lane == 0) {
-        atomicAdd(timeouts, 1u);
-        for (int q = 0; q < kPbStages - 1; ++q)  // loads already started: let them land
-          if (u + q < u1 && u + q != held)
-            mbar_wait_bounded(bars + (i + q) % kPbStages, ((i + q) / kPbStages) & 1);
-      }
-      break;
-    }
-    fence_proxy_async_smem();
-    const int t = static_cast<int>(u / nchunks);
-    const int v0 = static_cast<int>(u - static_cast<long long>(t) * nchunks) * cvec;
-    const uint32_t bytes = static_cast<uint32_t>(min(cvec, V - v0)) * 16u;
-    if (lane < K && slot >= 0)
-      bulk_s2g(out + static_cast<size_t>(slot) * V + v0, stages + static_cast<size_t>(b) * cvec,
-               bytes);
-    bulk_commit_group();
-    bulk_wait_group_read<1>();  // the stores of earlier units have read their buffers
-    __syncwarp();
-    if (lane == 0 && u + kPbStages - 1 < u1) issue(u + kPbStages - 1, (i + kPbStages - 1) % kPbStages);
-  }
-  bulk_wait_group<0>();  // every store of this lane performed before the warp leaves
-}
-
 // CPT 16-element chunks per thread (1, 2 or 4), chosen by the launcher so a
 // row fits the CTA with as few registers as possible.
 template <typename T16, int CPT>
@@ -356,7 +267,7 @@ __global__ void __launch_bounds__(smooth_threads<SPL>(), smooth_blocks_per_sm<SP
     const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
     const float4* __restrict__ smooth, const int32_t* __restrict__ assist,
     const int32_t* __restrict__ send, uint2* __restrict__ out, float* __restrict__ scales, int K,
-    int H, int A, int E, unsigned* timeouts) {
+    int H, int A, int E, WaitCfg wc, unsigned* timeouts) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -382,6 +293,8 @@ __global__ void __launch_bounds__(smooth_threads<SPL>(), smooth_blocks_per_sm<SP
   // expert of slot qb + l of the current batch of 32, loaded together, so the
   // index round trips are paid once per 32 slots.
   int qb = -32, my_pair = -1, my_e = -1;
+  // test hook: the first warp's slot number wc.withhold waits for bytes that never come
+  const int held = (blockIdx.x == 0 && warp == 0) ? wc.withhold : -1;
   // All lanes: slot q into buffer b (lane 0 records it and starts the copy).
   auto stage = [&](int q, int b) {
     if (q >= qb + 32) {
@@ -396,6 +309,10 @@ __global__ void __launch_bounds__(smooth_threads<SPL>(), smooth_blocks_per_sm<SP
     if (lane == 0) {
       info[b] = SmoothSlot{e, lo + warp + q * nwarps};
       fence_proxy_async_smem();  // the buffer was last read by the warp's loads
+      if (q == held) {  // test hook: 16 bytes that never come
+        mbar_arrive_expect_tx(bars + b, 16u);
+        return;
+      }
       mbar_arrive_expect_tx(bars + b, e >= 0 ? row_bytes : 0u);
       if (e >= 0)
         bulk_g2s(rows + static_cast<size_t>(b) * V, x + static_cast<size_t>(pair / K) * V,
@@ -410,12 +327,12 @@ __global__ void __launch_bounds__(smooth_threads<SPL>(), smooth_blocks_per_sm<SP
   int it = 0;
   for (int s = lo + warp; s < hi; s += nwarps, ++it) {
     const int b = it % kSmoothStages;
-    const bool ok = mbar_wait_bounded(bars + b, (it / kSmoothStages) & 1);
+    const bool ok = mbar_wait_bounded(bars + b, (it / kSmoothStages) & 1, wc.limit_ns);
     if (__any_sync(0xFFFFFFFFu, !ok)) {
       if (lane == 0) {
         atomicAdd(timeouts, 1u);
         for (int q = 1; q < kSmoothStages; ++q)  // copies already started: let them land
-          if (s + q * nwarps < hi)
+          if (s + q * nwarps < hi && it + q != held)
             mbar_wait_bounded(bars + (it + q) % kSmoothStages, ((it + q) / kSmoothStages) & 1);
       }
       return;
@@ -508,7 +425,7 @@ void quant_shape(int H, int* threads, int* cpt) {
 
 cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
                                   const float* smooth, const int32_t* send, int E,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, const WaitCfg& wc, bool staged_only) {
   if (a.bs == 0 || a.A == 0) return cudaSuccess;
   const int C = a.H / 16;
   const bool bf = a.dtype == MOE_BF16;
@@ -549,8 +466,10 @@ cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
     return launch_pdl(sk, dim3(blocks), dim3(32 * warps), smem, st,
                       static_cast<const uint4*>(a.x), topk_idx,
                       reinterpret_cast<const float4*>(smooth), a.assist, send,
-                      static_cast<uint2*>(a.expand_x), a.scales, a.K, a.H, a.A, E, timeouts);
+                      static_cast<uint2*>(a.expand_x), a.scales, a.K, a.H, a.A, E, wc,
+                      timeouts);
   }
+  if (staged_only) return cudaErrorNotSupported;
   int per_sm = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSmoothThreads, 0);
   if (err != cudaSuccess) return err;
@@ -564,49 +483,8 @@ cudaError_t launch_permute_smooth(const PermuteArgs& a, const int32_t* topk_idx,
                     static_cast<uint4*>(a.expand_x), a.scales, a.K, a.H, a.A, E);
 }
 
-// Column chunks per row for the bulk permute: with nw warps each taking
-// ceil(units / nw) units, pick the chunking (chunks of 1 to 4 KB) whose
-// busiest warp moves the fewest bytes (plus a per-unit overhead).
-void pb_chunking(int bs, int V, long long nw, int* nchunks, int* cvec) {
-  const int nmin = (V + 255) / 256;  // chunks of at most 4 KB
-  long long best = -1;
-  for (int n = nmin; n <= 4 * nmin && n <= V; ++n) {
-    const int cv = (V + n - 1) / n;
-    if (static_cast<long long>(n - 1) * cv >= V) continue;  // no empty last chunk
-    const long long units = static_cast<long long>(bs) * n;
-    const long long cost = ((units + nw - 1) / nw) * (static_cast<long long>(cv) * 16 + 256);
-    if (best < 0 || cost < best) {
-      best = cost;
-      *nchunks = n;
-      *cvec = cv;
-    }
-  }
-}
-
-cudaError_t launch_permute_bulk(const PermuteArgs& a, cudaStream_t st, const WaitCfg& wc) {
-  const int V = a.H / kVecElems;
-  unsigned* timeouts = wait_timeout_counter();
-  if (timeouts == nullptr) return cudaErrorInvalidSymbol;
-  const long long nw = static_cast<long long>(sm_count()) * 2 * kPbWarps;  // two CTAs per SM
-  int nchunks = 1, cvec = V;
-  pb_chunking(a.bs, V, nw, &nchunks, &cvec);
-  const size_t smem = kPbWarps * pb_warp_bytes(cvec);
-  cudaError_t err = cudaFuncSetAttribute(permute_bulk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  const long long units = static_cast<long long>(a.bs) * nchunks;
-  const long long want = (units + kPbWarps - 1) / kPbWarps;
-  const long long cap = nw / kPbWarps;
-  const int blocks = static_cast<int>(want < cap ? want : cap);
-  return launch_pdl(permute_bulk_kernel, dim3(blocks), dim3(32 * kPbWarps), smem, st,
-                    static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
-                    a.bs, a.K, V, a.A, nchunks, cvec, wc, timeouts);
-}
-
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   if (a.bs == 0) return cudaSuccess;
-  if (a.quant_mode == 0 && a.H / kVecElems >= kPermuteBulkMinVecs) return launch_permute_bulk(a, st);
   if (a.quant_mode == 0) {
     const int V = a.H / kVecElems;
     const long long n = static_cast<long long>(a.bs) * V;

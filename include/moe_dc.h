@@ -111,6 +111,13 @@ size_t moe_layout_workspace_bytes(const moe_shape* shape);
  *   workspace          device scratch of moe_layout_workspace_bytes() bytes
  *                      (NULL allowed when that is 0); its contents on entry do
  *                      not matter
+ * Up to 16384 tokens (while the per-warp expert masks fit in shared memory)
+ * the layout is one launch of a thread-block cluster of up to 16 blocks and
+ * needs no workspace; a device that cannot hold such a cluster returns
+ * MOE_ERR_CUDA (cudaErrorInvalidClusterSize) unless a workspace for the
+ * tiled path is given (tile counts, expert totals and a status word per tile
+ * of 256 tokens: 4 * (T * E + E + T) bytes, T = ceil(BS / 256)). Larger shapes
+ * take the tiled path: three launches (count, column scan, scatter).
  */
 moe_status moe_dispatch_layout(const moe_shape* shape, const int32_t* topk_idx,
                                const uint8_t* x_active_mask, int32_t* expert_token_nums,
@@ -167,10 +174,12 @@ moe_status moe_dispatch_permute_smooth(const moe_shape* shape, const void* x,
  * moe_dispatch — moe_dispatch_layout followed by moe_dispatch_permute, in one
  * call (the dispatch of the [combine] Example: low_latency_dispatch returns
  * the expanded rows, the counts and assist_info together). For BS <= 1024
- * without quantisation both run in one launch (every CTA rebuilds the small
- * layout in shared memory and copies its share of rows); otherwise the
- * launches of the two separate calls. Arguments and results as in those
- * calls; the workspace may be NULL when BS <= 1024.
+ * without quantisation (and E <= 640, whose lane masks fit in shared memory)
+ * both run in one launch (every CTA
+ * rebuilds the small layout in shared memory and copies its share of rows);
+ * otherwise the launches of the two separate calls. Arguments and results as
+ * in those calls; the workspace may be NULL when moe_layout_workspace_bytes()
+ * is 0.
  */
 moe_status moe_dispatch(const moe_shape* shape, const int32_t* topk_idx,
                         const uint8_t* x_active_mask, const void* x, int comm_quant_mode,
@@ -361,35 +370,32 @@ size_t moe_layout_noalloc_max_workspace_bytes(void);
 
 /*
  * Test hooks for the bounded waits (no counterpart on the pages). The staged
- * kernels wait on mbarriers for their own bulk copies; every such wait gives
- * up after a time limit, counts the giving-up block in
- * moe_async_wait_timeouts(), lets the copies it started land, and returns,
- * leaving that block's part of the output unwritten. These two calls run the
- * staged combine gather and the bulk-copy permute with a shorter limit and one
- * unit of work whose barrier is armed for 16 bytes that no copy delivers (in
- * the first block, or the first warp), so that the give-up path runs while no
- * copy is in flight for that unit. Not for production use.
+ * kernels (the one-pass int8 combine, the smooth-scaled int8 dispatch) wait on
+ * mbarriers for their own bulk copies; every such wait gives up after a time
+ * limit, counts the giving-up block (or warp) in moe_async_wait_timeouts(),
+ * lets the copies it started land, and returns, leaving its part of the output
+ * unwritten. These two calls run those kernels with a shorter limit and one
+ * unit of work whose barrier is armed for 16 bytes that no copy delivers, so
+ * that the give-up path runs while no copy is in flight for that unit. Not for
+ * production use.
  *   wait_limit_ns   limit of the pipeline waits, in (0, 1e9] ns
- *   withhold_unit   index, among the units of the first block (combine: token
- *                   column chunks; permute: the first warp's units), of the
- *                   unit whose copies are withheld; >= 0
- * Other arguments as moe_combine_fwd / moe_dispatch_permute (mode 0). Returns
- * MOE_ERR_UNSUPPORTED for shapes those calls run on other kernels (rows
- * narrower than 32 vectors of 16 bytes).
+ *   withhold_unit   >= 0: the int8 combine's first block's token number
+ *                   withhold_unit (in that block's order), or the smooth
+ *                   dispatch's first warp's slot number withhold_unit
+ * Other arguments as moe_combine_fwd_comm_quant (mode 2) and
+ * moe_dispatch_permute_smooth. MOE_ERR_UNSUPPORTED for shapes those calls run
+ * on other kernels (K > 8, or rows whose buffers do not fit in shared memory).
  */
-moe_status moe_test_combine_fwd_wait_timeout(const moe_shape* shape, const void* expand_x,
-                                             const int32_t* topk_idx, const float* topk_weights,
-                                             const int32_t* assist_info,
-                                             const uint8_t* x_active_mask,
-                                             const void* shared_expert_x, const void* ori_x,
-                                             const void* const_alpha_1,
-                                             const void* const_alpha_2, const void* const_v,
-                                             void* out, uint64_t wait_limit_ns,
-                                             int withhold_unit, void* stream);
-moe_status moe_test_dispatch_permute_wait_timeout(const moe_shape* shape, const void* x,
-                                                  const int32_t* assist_info, void* expand_x,
-                                                  uint64_t wait_limit_ns, int withhold_unit,
-                                                  void* stream);
+moe_status moe_test_combine_fwd_comm_quant_wait_timeout(
+    const moe_shape* shape, const void* expand_x, const int32_t* topk_idx,
+    const float* topk_weights, const int32_t* assist_info, const uint8_t* x_active_mask,
+    const void* shared_expert_x, const void* ori_x, const void* const_alpha_1,
+    const void* const_alpha_2, const void* const_v, void* out, uint64_t wait_limit_ns,
+    int withhold_unit, void* stream);
+moe_status moe_test_dispatch_permute_smooth_wait_timeout(
+    const moe_shape* shape, const void* x, const int32_t* topk_idx, const int32_t* assist_info,
+    const int32_t* ep_send_counts, const float* smooth_scales, void* expand_x,
+    float* dynamic_scales, uint64_t wait_limit_ns, int withhold_unit, void* stream);
 
 #ifdef __cplusplus
 }

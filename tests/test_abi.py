@@ -135,9 +135,10 @@ def test_sizes():
     s = moe.Shape(bs=128, k=8, h=1536, num_experts=64)
     assert moe.moe_assist_info_elems(ctypes.byref(s.c())) == 1024 + 128 * 8
     assert moe.moe_layout_workspace_bytes(ctypes.byref(s.c())) == 0  # cluster layout
-    # the cluster layout takes up to 16384 tokens while its masks fit in shared memory
-    for bs, e, need_ws in ((16384, 256, False), (16385, 64, True), (8192, 1024, False),
-                           (9000, 1024, True)):
+    # the cluster layout takes up to 16384 tokens while its masks and pair lists fit in
+    # shared memory
+    for bs, e, need_ws in ((16384, 256, False), (16385, 64, True), (8192, 512, False),
+                           (8192, 1024, True)):
         sh = moe.Shape(bs=bs, k=8, h=1536, num_experts=e)
         assert (moe.moe_layout_workspace_bytes(ctypes.byref(sh.c())) > 0) == need_ws
     assert moe.moe_status_string(moe.MOE_ERR_CUDA) == b"CUDA error"
