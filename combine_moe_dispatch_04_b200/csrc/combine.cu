@@ -89,12 +89,17 @@ template <bool SPECIAL, bool UNIT, bool CHECK_REPEATS = true, bool SRC_ROWS = fa
 __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, int k) {
   PairMeta m{kSkip, 0, 1.0f};
   const size_t tk = static_cast<size_t>(t) * a.K + k;
-  // every load first (none depends on another), so the pair costs one round trip
+  // With special experts the id and the slot are loaded together, so the pair
+  // costs one round trip instead of two (the slot load would otherwise wait for
+  // the id's range check). Without them the slot is loaded after the mask test,
+  // which measured faster (8192-token step 195.8 vs 199.6 us).
   if (!UNIT) m.w = __ldg(a.weights + tk);
-  const int s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
+  int s = -1;
+  if (SPECIAL) s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
   const int32_t* ids = a.topk_idx + static_cast<size_t>(t) * a.K;
   const int id = SPECIAL ? __ldg(ids + k) : 0;
   if (!pair_active(a.mask, a.mask_ndim, t, k, a.K)) return m;
+  if (!SPECIAL) s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
   if (SPECIAL) {
     if (id < 0 || id >= a.E + a.Z + a.C + a.Q) return m;
     if (CHECK_REPEATS)

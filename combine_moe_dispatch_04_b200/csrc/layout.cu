@@ -115,6 +115,41 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
   return before + inc - v;
 }
 
+// The same for two values per thread at once (one pass of barriers).
+__device__ __forceinline__ int2 block_exclusive_scan2(int2 v, int2* warp_sums, int2* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  int2 inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int nx = __shfl_up_sync(0xFFFFFFFFu, inc.x, d);
+    const int ny = __shfl_up_sync(0xFFFFFFFFu, inc.y, d);
+    if (lane >= d) {
+      inc.x += nx;
+      inc.y += ny;
+    }
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int2 s = lane < nwarps ? warp_sums[lane] : make_int2(0, 0);
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int nx = __shfl_up_sync(0xFFFFFFFFu, s.x, d);
+      const int ny = __shfl_up_sync(0xFFFFFFFFu, s.y, d);
+      if (lane >= d) {
+        s.x += nx;
+        s.y += ny;
+      }
+    }
+    if (lane < nwarps) warp_sums[lane] = s;  // inclusive warp prefix
+  }
+  __syncthreads();
+  const int2 before = warp == 0 ? make_int2(0, 0) : warp_sums[warp - 1];
+  *total = warp_sums[nwarps - 1];
+  return make_int2(before.x + inc.x - v.x, before.y + inc.y - v.y);
+}
+
 // Writes both halves of assist_info for token t's pairs given their slots.
 template <int KM>
 __device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const int (&e)[KM],
@@ -167,6 +202,8 @@ __device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t ran
 }
 
 __host__ __device__ constexpr int cluster_stride(int E) { return E | 1; }
+
+constexpr int kClusterMaxCtas = 16;  // blocks per cluster, at most
 
 // Per (sub-block, warp, expert): the lane mask of the warp's tokens routed to
 // the expert (x) and the number of the CTA's earlier tokens routed there (y).
@@ -263,7 +300,7 @@ __device__ __forceinline__ int cta_rank(const MaskPre* mp, int i, int S, int ex)
 template <int KM, int TPT, int NT>
 __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ int warp_sums[32];
+  __shared__ int2 warp_sums2[32];
   __shared__ uint32_t status, status_all;
   const int E = a.E;
   const int S = cluster_stride(E);
@@ -289,13 +326,18 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
   cluster_arrive_release();  // tot and status are published to the cluster
   cluster_wait_acquire();
 
-  // grand totals and the pairs of the CTAs before this one, per expert
+  // grand totals and the pairs of the CTAs before this one, per expert (all the
+  // remote loads are issued before any is used)
   int grand = 0, before = 0;
   if (threadIdx.x < E) {
-    for (uint32_t c = 0; c < cs; ++c) {
-      const int v = static_cast<int>(ld_dsmem_u32(tot + threadIdx.x, c));
-      grand += v;
-      before += c < rank ? v : 0;
+    int v[kClusterMaxCtas];
+#pragma unroll
+    for (int c = 0; c < kClusterMaxCtas; ++c)
+      v[c] = c < static_cast<int>(cs) ? static_cast<int>(ld_dsmem_u32(tot + threadIdx.x, c)) : 0;
+#pragma unroll
+    for (int c = 0; c < kClusterMaxCtas; ++c) {
+      grand += v[c];
+      before += c < static_cast<int>(rank) ? v[c] : 0;
     }
   }
   uint32_t cst = 0;
@@ -303,11 +345,13 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
   __syncwarp();
   cluster_arrive_release();  // done reading the other CTAs' shared memory
   if (cst) atomicOr(&status_all, cst);
-  int total, cta_total;
-  const int excl = block_exclusive_scan(threadIdx.x < E ? grand : 0, warp_sums, &total);
-  __syncthreads();  // every thread has read warp_sums before the second scan rewrites it
-  const int lexcl = block_exclusive_scan(threadIdx.x < E ? tot[threadIdx.x] : 0, warp_sums,
-                                         &cta_total);
+  // exclusive scans over the experts of the grand totals (global first slots) and
+  // of this CTA's totals (positions in its expert-ordered pair list)
+  int2 totals;
+  const int2 ex2 = block_exclusive_scan2(
+      threadIdx.x < E ? make_int2(grand, tot[threadIdx.x]) : make_int2(0, 0), warp_sums2, &totals);
+  const int total = totals.x;
+  const int excl = ex2.x, lexcl = ex2.y;
   if (threadIdx.x < E) {
     bo[threadIdx.x] = BaseOfs{excl + before, lexcl};
     if (rank == 0) {
