@@ -197,7 +197,8 @@ def layout_launches(bs: int, num_experts: int, k: int) -> int:
     """Launches of moe_dispatch_layout: one thread-block cluster for BS <= 16384 when
     its lane masks and pair lists fit in shared memory, else count, column scan and
     scatter."""
-    nt = 512 if bs <= 8192 and num_experts <= 512 else 1024
+    nt = (256 if bs <= 256 and num_experts <= 256
+          else 512 if bs <= 8192 and num_experts <= 512 else 1024)
     stride = num_experts | 1
     smem = (nt // 32) * stride * 8 + num_experts * 12 + nt * k * 4
     return 1 if bs <= 16384 and smem <= 210 * 1024 else 3

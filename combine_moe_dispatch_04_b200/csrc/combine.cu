@@ -130,9 +130,15 @@ __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, i
 // ascending k.
 // Resident blocks per SM the forward kernel is compiled for (a register cap
 // that avoids spills for each variant).
+// Blocks per SM of the special-expert variant for K <= 8: at 4 (64 registers, a
+// few bytes of spill) it ran 67 us against 76 us at 3 (72 registers, no spill)
+// on the 8192-token H 2048 special workload.
+#ifndef MOE_FWD_SPECIAL_MIN_BLOCKS
+#define MOE_FWD_SPECIAL_MIN_BLOCKS 4
+#endif
 template <int KMAX, bool SPECIAL>
 __host__ __device__ constexpr int fwd_min_blocks() {
-  return SPECIAL ? (KMAX <= 8 ? 3 : 2) : KMAX == 16 ? 2 : KMAX == 4 ? 3 : 4;
+  return SPECIAL ? (KMAX <= 8 ? MOE_FWD_SPECIAL_MIN_BLOCKS : 2) : KMAX == 16 ? 2 : KMAX == 4 ? 3 : 4;
 }
 
 template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool SHARED>

@@ -401,10 +401,11 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
 // would (the ids are at most 64 KB and sit in L2), CTA 0 alone writes the
 // layout's outputs, and CTA c copies the rows of tokens [c * per, (c+1) * per)
 // to their slots: one thread per 16-byte vector, read once, stored K times.
-// Dynamic shared memory: mp[32][S], bo[E], tot[E].
-template <int KM>
-__global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, const uint4* x,
-                                                                 uint4* expand_x, int V, int per) {
+// NT threads (256 for up to 256 tokens and experts, else 1024). Dynamic shared
+// memory: mp[NT / 32][S], bo[E], tot[E].
+template <int KM, int NT>
+__global__ void __launch_bounds__(NT, 1) dispatch_small_kernel(LayoutArgs a, const uint4* x,
+                                                               uint4* expand_x, int V, int per) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int warp_sums[32];
   __shared__ uint32_t status;
@@ -412,16 +413,17 @@ __global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, c
   const int E = a.E;
   const int S = cluster_stride(E);
   MaskPre* mp = reinterpret_cast<MaskPre*>(smem);
-  BaseOfs* bo = reinterpret_cast<BaseOfs*>(smem + static_cast<size_t>(32) * S * sizeof(MaskPre));
+  BaseOfs* bo = reinterpret_cast<BaseOfs*>(smem + static_cast<size_t>(NT / 32) * S *
+                                                      sizeof(MaskPre));
   int* tot = reinterpret_cast<int*>(bo + E);
   const bool writer = blockIdx.x == 0;
   pdl_trigger();
-  for (int i = threadIdx.x; i < 32 * S; i += blockDim.x) mp[i] = MaskPre{0u, 0u};
+  for (int i = threadIdx.x; i < (NT / 32) * S; i += NT) mp[i] = MaskPre{0u, 0u};
   if (threadIdx.x == 0) status = 0;
   __syncthreads();
   pdl_wait();
   int e[1][KM];
-  cta_count_scan<KM, 1, 1024>(a, 0, S, mp, tot, &status, e);
+  cta_count_scan<KM, 1, NT>(a, 0, S, mp, tot, &status, e);
   __syncthreads();
   const int cnt = threadIdx.x < E ? tot[threadIdx.x] : 0;
   int total;
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(1024, 1) dispatch_small_kernel(LayoutArgs a, c
     int slot[KM];
 #pragma unroll
     for (int k = 0; k < KM; ++k)
-      slot[k] = (k < a.K && e[0][k] >= 0) ? bo[e[0][k]].first + cta_rank<1024>(mp, 0, S, e[0][k])
+      slot[k] = (k < a.K && e[0][k] >= 0) ? bo[e[0][k]].first + cta_rank<NT>(mp, 0, S, e[0][k])
                                           : -1;
     if (writer) write_slots<KM>(a, t, e[0], slot);
     if (t >= t0 && t < t0 + per) {
@@ -664,9 +666,9 @@ __global__ void __launch_bounds__(kLayoutTileTokens) layout_scatter_kernel(Layou
     a.assist[s] = -1;
 }
 
-template <int KM>
-cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* expand_x, int H,
-                                    cudaStream_t st) {
+template <int KM, int NT>
+cudaError_t launch_dispatch_small_nt(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                     cudaStream_t st) {
   const int V = H / kVecElems;
   // at most kLayoutSmallMaxTokens / 8 tokens per CTA (the slot buffer's size)
   int blocks = sm_count();
@@ -675,18 +677,25 @@ cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* ex
   if (per > kLayoutSmallMaxTokens / 8) per = kLayoutSmallMaxTokens / 8;
   if (per < 1) per = 1;
   blocks = a.bs > 0 ? (a.bs + per - 1) / per : 1;
-  const size_t smem = cluster_smem_bytes(a.E, 1);
-  cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel<KM>,
+  const size_t smem = cluster_smem_bytes(a.E, 1, NT);
+  cudaError_t err = cudaFuncSetAttribute(dispatch_small_kernel<KM, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  return launch_pdl(dispatch_small_kernel<KM>, dim3(blocks), dim3(1024), smem, st, a,
+  return launch_pdl(dispatch_small_kernel<KM, NT>, dim3(blocks), dim3(NT), smem, st, a,
                     static_cast<const uint4*>(x), static_cast<uint4*>(expand_x), V, per);
 }
 
-// The cluster layout: CS <= 16 CTAs of NT threads, one token per thread: 512
-// threads per CTA up to 8192 tokens (and E <= 512), so that up to 16 SMs share
-// the work, else 1024.
+template <int KM>
+cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* expand_x, int H,
+                                    cudaStream_t st) {
+  if (a.bs <= 256 && a.E <= 256) return launch_dispatch_small_nt<KM, 256>(a, x, expand_x, H, st);
+  return launch_dispatch_small_nt<KM, 1024>(a, x, expand_x, H, st);
+}
+
+// The cluster layout: CS <= 16 CTAs of NT threads, one token per thread: 256
+// threads for up to 256 tokens and experts (one block), 512 up to 8192 tokens
+// and E <= 512, so that up to 16 SMs share the work, else 1024.
 #ifndef MOE_LAYOUT_CLUSTER_MAX_TOKENS
 #define MOE_LAYOUT_CLUSTER_MAX_TOKENS (16 * 1024)
 #endif
@@ -695,7 +704,10 @@ constexpr size_t kClusterSmemMax = 210 * 1024;
 
 // The kernel gives each expert one thread (its grand total, scan entry and first
 // slot), so E <= threads: 512 threads only for E <= 512.
-int cluster_threads(int bs, int E) { return (bs <= 16 * 512 && E <= 512) ? 512 : 1024; }
+int cluster_threads(int bs, int E) {
+  if (bs <= 256 && E <= 256) return 256;
+  return (bs <= 16 * 512 && E <= 512) ? 512 : 1024;
+}
 
 // Workspace of the tiled path: tile counts, expert totals, tile status words.
 size_t tiled_workspace_bytes(int bs, int E) {
@@ -756,9 +768,10 @@ template <int KM>
 cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t st) {
   if (cluster_layout_applies(a.bs, a.E, a.K)) {
     bool fits = false;
-    const cudaError_t err = cluster_threads(a.bs, a.E) == 512
-                                ? launch_layout_cluster<KM, 1, 512>(a, st, &fits)
-                                : launch_layout_cluster<KM, 1, 1024>(a, st, &fits);
+    const int nt = cluster_threads(a.bs, a.E);
+    const cudaError_t err = nt == 256   ? launch_layout_cluster<KM, 1, 256>(a, st, &fits)
+                            : nt == 512 ? launch_layout_cluster<KM, 1, 512>(a, st, &fits)
+                                        : launch_layout_cluster<KM, 1, 1024>(a, st, &fits);
     if (err != cudaSuccess || fits) return err;
     // a device that cannot hold the cluster: the tiled path, if given its workspace
     if (a.workspace == nullptr || a.workspace_bytes < tiled_workspace_bytes(a.bs, a.E))

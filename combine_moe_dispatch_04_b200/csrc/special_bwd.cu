@@ -9,7 +9,7 @@
 //   grad_alpha2[j]   = fl(S[j] v[j]),   grad_v[j] = fl(S[j] alpha2[j])
 //
 // Three launches: warp-per-token grad_w dots (fixed butterfly) and grad_ori_x,
-// per-(token chunk, const expert) partial sums into the workspace, and one
+// per-(token chunk, const expert) partial sums into the workspace, and a
 // fixed-order sum over the chunks. Every result is deterministic.
 #include "common.cuh"
 #include "launch.cuh"
@@ -41,12 +41,14 @@ struct SpecialBwdArgs {
 
 // grad_w of the copy/const pairs and grad_ori_x: one warp per token on a
 // persistent grid. Lanes 0..K-1 classify the token's pairs (a repeat of an id
-// held by an earlier lane takes no part); the warp walks the ballot of those
-// pairs, taking each pair's kind, weight and const row by shuffle. A token
-// without such pairs only writes its zero grad_ori_x row. Otherwise the warp
-// writes grad_ori_x (pairs in ascending k), then makes one pass over the row
-// per pair for its dot (grad_out[t] and ori_x[t] from L1 after the first
-// touch), reduced with a fixed butterfly.
+// held by an earlier lane takes no part). A token without such pairs only
+// writes its zero grad_ori_x row. Otherwise the warp makes one pass over the
+// row, kUV vectors per lane at a time with all their grad_out and ori_x loads
+// issued first: per vector it adds the pairs' terms to grad_ori_x in ascending
+// k and each pair's products to that pair's own dot accumulator (pair k in
+// register k); the dots are reduced with a fixed butterfly at the end.
+constexpr int kUV = 2;
+
 template <typename T16, int KMAX>
 __global__ void __launch_bounds__(kThreads) special_token_kernel(SpecialBwdArgs a) {
   pdl_trigger();
@@ -74,68 +76,69 @@ __global__ void __launch_bounds__(kThreads) special_token_kernel(SpecialBwdArgs 
     }
     uint4* go = static_cast<uint4*>(a.grad_ori_x) + static_cast<size_t>(t) * V;
     const unsigned spec = __ballot_sync(0xFFFFFFFFu, my_kind != 0);
+    if (spec == 0) {  // no copy/const pair: a zero grad_ori_x row
+      for (int v = lane; v < V; v += 32) st_v4(go + v, make_uint4(0u, 0u, 0u, 0u));
+      continue;
+    }
     const uint4* g = static_cast<const uint4*>(a.grad_out) + static_cast<size_t>(t) * V;
     const uint4* x = static_cast<const uint4*>(a.ori_x) + static_cast<size_t>(t) * V;
-    // grad_ori_x, pairs in ascending k (a token without such pairs gets zeros)
-    // (every lane runs every iteration: the shuffles below need the whole warp)
-    for (int v0 = 0; v0 < V; v0 += 32) {
-      const int v = v0 + lane;
-      const bool in = v < V;
-      float acc[8];
+    float d[KMAX];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-      if (spec != 0) {
-        float gf[8];
-        widen8<T16>(in ? __ldg(g + v) : make_uint4(0, 0, 0, 0), gf);  // kept in L1 for the dots
-        for (unsigned m = spec; m != 0; m &= m - 1) {
-          const int j = __ffs(m) - 1;
+    for (int j = 0; j < KMAX; ++j) d[j] = 0.0f;
+    // every lane runs every iteration: the shuffles below need the whole warp
+    for (int v0 = 0; v0 < V; v0 += 32 * kUV) {
+      uint4 gv[kUV], xv[kUV];
+#pragma unroll
+      for (int u = 0; u < kUV; ++u) {
+        const int v = v0 + 32 * u + lane;
+        gv[u] = v < V ? ld_nc_v4(g + v) : make_uint4(0u, 0u, 0u, 0u);
+        xv[u] = v < V ? ld_nc_v4(x + v) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kUV; ++u) {
+        const int v = v0 + 32 * u + lane;
+        const bool in = v < V;
+        float gf[8], xf[8], acc[8];
+        widen8<T16>(gv[u], gf);
+        widen8<T16>(xv[u], xf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (!((spec >> j) & 1u)) continue;  // warp-uniform
           const int kind = __shfl_sync(0xFFFFFFFFu, my_kind, j);
           const float w = __shfl_sync(0xFFFFFFFFu, my_w, j);
           const int q = __shfl_sync(0xFFFFFFFFu, my_q, j);
-          if (kind == 1) {
+          if (kind == 1) {  // copy: c = fl(w g) into grad_ori_x, <g, ori_x> into the dot
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, gf[i]));
-          } else {
-            float a1[8];
-            widen8<T16>(in ? __ldg(static_cast<const uint4*>(a.alpha1) +
-                                   static_cast<size_t>(q) * V + v)
-                           : make_uint4(0, 0, 0, 0),
-                        a1);
+            for (int i = 0; i < 8; ++i) {
+              acc[i] = __fadd_rn(acc[i], __fmul_rn(w, gf[i]));
+              d[j] = __fmaf_rn(gf[i], xf[i], d[j]);
+            }
+          } else {  // const: fl(c alpha_1), and <g, fl(fl(a1 x) + fl(a2 v))>
+            const size_t r = static_cast<size_t>(q) * V + (in ? v : 0);
+            float a1[8], a2[8], cv[8];
+            widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + r), a1);
+            widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + r), a2);
+            widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + r), cv);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 8; ++i) {
               acc[i] = __fadd_rn(acc[i], __fmul_rn(__fmul_rn(w, gf[i]), a1[i]));
+              d[j] = __fmaf_rn(gf[i], __fadd_rn(__fmul_rn(a1[i], xf[i]), __fmul_rn(a2[i], cv[i])),
+                               d[j]);
+            }
           }
         }
+        if (in) st_v4(go + v, narrow8<T16>(acc));
       }
-      if (in) st_v4(go + v, narrow8<T16>(acc));
     }
-    // grad_w: one pass over the row per copy/const pair, then a fixed butterfly
-    for (unsigned m = spec; m != 0; m &= m - 1) {
-      const int j = __ffs(m) - 1;
-      const int kind = __shfl_sync(0xFFFFFFFFu, my_kind, j);
-      const int q = __shfl_sync(0xFFFFFFFFu, my_q, j);
-      float d = 0.0f;
-      for (int v = lane; v < V; v += 32) {
-        float gf[8], xf[8];
-        widen8<T16>(__ldg(g + v), gf);
-        widen8<T16>(__ldg(x + v), xf);
-        if (kind == 1) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) d = __fmaf_rn(gf[i], xf[i], d);
-        } else {
-          const size_t r = static_cast<size_t>(q) * V + v;
-          float a1[8], a2[8], cv[8];
-          widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha1) + r), a1);
-          widen8<T16>(__ldg(static_cast<const uint4*>(a.alpha2) + r), a2);
-          widen8<T16>(__ldg(static_cast<const uint4*>(a.const_v) + r), cv);
+    for (int j = 0; j < KMAX; ++j) {
+      if (!((spec >> j) & 1u)) continue;
+      float dj = d[j];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d = __fmaf_rn(gf[i], __fadd_rn(__fmul_rn(a1[i], xf[i]), __fmul_rn(a2[i], cv[i])), d);
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xFFFFFFFFu, d, off);
-      if (lane == 0) a.grad_w[static_cast<size_t>(t) * K + j] = d;
+      for (int off = 16; off > 0; off >>= 1) dj += __shfl_xor_sync(0xFFFFFFFFu, dj, off);
+      if (lane == 0) a.grad_w[static_cast<size_t>(t) * K + j] = dj;
     }
   }
 }
@@ -230,19 +233,38 @@ __global__ void __launch_bounds__(kThreads) special_partial_kernel(SpecialBwdArg
   pcv[1] = make_float4(sc[4], sc[5], sc[6], sc[7]);
 }
 
-// Sum of the partials over the chunks, in chunk order: grad_alpha1, and the
-// alpha_2 / v gradients from S.
+// Sum of the partials over the chunks: grad_alpha1, and the alpha_2 / v
+// gradients from S. A block takes 32 elements; its 8 warps sum the chunks
+// c = w, w + 8, ... of each (lane = element), then one fixed-order pass over
+// the 8 sums: the same order every run.
+constexpr int kFinalParts = kThreads / 32;
+
 template <typename T16>
 __global__ void __launch_bounds__(kThreads) special_final_kernel(SpecialBwdArgs a, int chunks) {
+  __shared__ float s1p[kFinalParts][32], scp[kFinalParts][32];
   pdl_trigger();
   pdl_wait();
   const size_t qh = static_cast<size_t>(a.Q) * a.H;
-  const size_t i = static_cast<size_t>(blockIdx.x) * kThreads + threadIdx.x;
-  if (i >= qh) return;
+  const int lane = threadIdx.x & 31, part = threadIdx.x >> 5;
+  const size_t i = static_cast<size_t>(blockIdx.x) * 32 + lane;
   float s1 = 0.0f, sc = 0.0f;
-  for (int c = 0; c < chunks; ++c) {
-    s1 = __fadd_rn(s1, a.partials[static_cast<size_t>(c) * 2 * qh + i]);
-    sc = __fadd_rn(sc, a.partials[static_cast<size_t>(c) * 2 * qh + qh + i]);
+  if (i < qh) {
+#pragma unroll 4
+    for (int c = part; c < chunks; c += kFinalParts) {
+      s1 = __fadd_rn(s1, a.partials[static_cast<size_t>(c) * 2 * qh + i]);
+      sc = __fadd_rn(sc, a.partials[static_cast<size_t>(c) * 2 * qh + qh + i]);
+    }
+  }
+  s1p[part][lane] = s1;
+  scp[part][lane] = sc;
+  __syncthreads();
+  if (part != 0 || i >= qh) return;
+  s1 = s1p[0][lane];
+  sc = scp[0][lane];
+#pragma unroll
+  for (int p = 1; p < kFinalParts; ++p) {
+    s1 = __fadd_rn(s1, s1p[p][lane]);
+    sc = __fadd_rn(sc, scp[p][lane]);
   }
   // element i of alpha_2 and v: the pair of 16-bit values holding it, widened
   const size_t pi = i / 2;
@@ -279,9 +301,8 @@ cudaError_t launch_t(const SpecialBwdArgs& a, cudaStream_t st) {
                    dim3(chunks, a.Q, (V + kThreads - 1) / kThreads), dim3(kThreads), 0, st, a);
   if (err != cudaSuccess) return err;
   const long long qh = static_cast<long long>(a.Q) * a.H;
-  return launch_pdl(special_final_kernel<T16>,
-                    dim3(static_cast<int>((qh + kThreads - 1) / kThreads)), dim3(kThreads), 0, st,
-                    a, chunks);
+  return launch_pdl(special_final_kernel<T16>, dim3(static_cast<int>((qh + 31) / 32)),
+                    dim3(kThreads), 0, st, a, chunks);
 }
 
 }  // namespace
