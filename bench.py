@@ -562,9 +562,10 @@ class Bench:
 
     def timed_run(self, steps, warmup, flush_l2, world, sampler=None):
         """W warm-up steps, then `steps` timed steps (an L2 flush before each, outside
-        the step's events). Every DOM_EVERY-th step also brackets the dominant kernel
-        with events (an event between two kernels costs both their launch overlap, so
-        the other steps carry only the step's own start/end events)."""
+        the step's events), each carrying only its own start/end events; then, in the
+        same bracketed window, ceil(steps / DOM_EVERY) more steps with events around
+        the dominant kernel as well (an event between two kernels costs both their
+        launch overlap, so those steps are kept out of the step statistics)."""
         import torch.distributed as dist
         torch = self.torch
         dom = self.dominant
@@ -572,19 +573,12 @@ class Bench:
             flush_l2()
             self.step(graph=self.plain_graph)
         torch.cuda.synchronize()
-        sampled = [i % DOM_EVERY == DOM_EVERY - 1 for i in range(steps)]
-        marks, graphs = [], []
-        for i in range(steps):
-            m = self.new_marks([])
-            if sampled[i]:
-                inner = self.new_marks([dom], external=self.use_graph)
-                m[dom] = inner[dom]
-                graphs.append(self.capture({dom: inner[dom]}) if self.use_graph else None)
-            else:
-                graphs.append(self.plain_graph)
-            marks.append(m)
+        n_dom = max(1, -(-steps // DOM_EVERY))
+        marks = [self.new_marks([]) for _ in range(steps)]
+        dmarks = [self.new_marks([dom], external=self.use_graph) for _ in range(n_dom)]
+        dgraphs = [self.capture({dom: m[dom]}) if self.use_graph else None for m in dmarks]
         if self.use_graph:
-            for g in {id(g): g for g in graphs}.values():  # warm every graph once
+            for g in dgraphs:  # warm every graph once
                 flush_l2()
                 self.step(graph=g)
             torch.cuda.synchronize()
@@ -596,19 +590,23 @@ class Bench:
         t0 = time.time()
         for i in range(steps):
             flush_l2()
+            self.step({"start": marks[i]["start"], "end": marks[i]["end"]},
+                      graph=self.plain_graph)
+        for i in range(n_dom):
+            flush_l2()
             if self.use_graph:
-                self.step({"start": marks[i]["start"], "end": marks[i]["end"]}, graph=graphs[i])
+                self.step({"start": dmarks[i]["start"], "end": dmarks[i]["end"]},
+                          graph=dgraphs[i])
             else:
-                self.step(marks[i] if sampled[i] else
-                          {"start": marks[i]["start"], "end": marks[i]["end"]})
+                self.step(dmarks[i])
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         t1 = time.time()
         clocks = sampler.stop(t0, t1) if sampler is not None else None
         step_ms = [m["start"].elapsed_time(m["end"]) for m in marks]
-        dom_ms = [m[dom][0].elapsed_time(m[dom][1]) for m in marks if dom in m]
-        del graphs
+        dom_ms = [m[dom][0].elapsed_time(m[dom][1]) for m in dmarks]
+        del dgraphs
         return step_ms, dom_ms, clocks
 
     def accepted_run(self, steps, warmup, flush_l2, world, rank, uuid):
@@ -853,7 +851,7 @@ def main():
         roof = dict(head["roofline"])
         roof.update(peak_kind=peak_kind,
                     traffic=profiled_traffic(line_extra["dominant"], line_extra["traffic_key"]),
-                    timed=f"CUDA events around this kernel in every {DOM_EVERY}th timed step "
+                    timed=f"CUDA events around this kernel in ceil(steps / {DOM_EVERY}) more steps "
                           f"({len(run['dom_ms'])} launches)")
         st = run["stats"]
         cq = args.combine_comm_quant
@@ -875,8 +873,9 @@ def main():
                        "l2": "flushed before every step (write of 2x L2, then a read of another "
                              "2x L2 so no dirty flush lines are written back inside the step), "
                              "outside the step events",
-                       "statistics": f"value and ms_per_step: mean of the timed steps without "
-                                     f"the {DROP_TOP} slowest, max over ranks; accepted when "
+                       "statistics": f"value and ms_per_step: mean of the K timed steps (each "
+                                     f"with only its start/end events) without the {DROP_TOP} "
+                                     f"slowest, max over ranks; accepted when "
                                      f"std/mean <= {ACCEPT_CV:.0%}, else rerun (at most "
                                      f"{MAX_RUNS} runs, the steadiest kept)"},
             "hbm_gbs": head["hbm_gbs"], "hbm_frac_of_8tbs": head["hbm_frac_of_8tbs"],
@@ -885,7 +884,7 @@ def main():
             "roofline": roof,
             "kernels_diagnostic": {"note": "separate untimed steps with events around every "
                                            "kernel (no launch overlap)", **kstats},
-            "gpu_launches": launches * args.steps,
+            "gpu_launches": launches * (args.steps + len(run["dom_ms"])),
             "e2e": e2e,
             "clocks": run["clocks"],
             "step_ms_stats": {"trimmed_mean_drop_top3": st["mean"], "std": st["std"],

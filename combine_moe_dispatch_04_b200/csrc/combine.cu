@@ -120,19 +120,10 @@ __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, i
   return m;
 }
 
-// Each warp owns a contiguous span of 32 * U output vectors (8 values each);
-// lane l handles vectors l, l + 32, ... of the span, so every load of the warp
-// is 32 consecutive 16-byte vectors. When a span fits in two tokens' rows
-// (V >= 32 * U), lanes 0..K-1 classify the first token's pairs and lanes
-// 16..16+K-1 the second's, once for the whole span, and every lane takes its
-// token's metadata by shuffle. (Narrower rows: every thread classifies its own
-// token's pairs.) All routed rows' loads are issued before accumulating in
-// ascending k.
 // Resident blocks per SM the forward kernel is compiled for (a register cap
-// that avoids spills for each variant).
-// Blocks per SM of the special-expert variant for K <= 8: at 4 (64 registers, a
-// few bytes of spill) it ran 67 us against 76 us at 3 (72 registers, no spill)
-// on the 8192-token H 2048 special workload.
+// that avoids spills for each variant). For the special-expert variant with
+// K <= 8: at 4 (64 registers, a few bytes of spill) it ran 67 us against 76 us
+// at 3 (72 registers, no spill) on the 8192-token H 2048 special workload.
 #ifndef MOE_FWD_SPECIAL_MIN_BLOCKS
 #define MOE_FWD_SPECIAL_MIN_BLOCKS 4
 #endif
@@ -141,7 +132,15 @@ __host__ __device__ constexpr int fwd_min_blocks() {
   return SPECIAL ? (KMAX <= 8 ? MOE_FWD_SPECIAL_MIN_BLOCKS : 2) : KMAX == 16 ? 2 : KMAX == 4 ? 3 : 4;
 }
 
-template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool SHARED>
+// Each warp owns a contiguous span of 32 * U output vectors (8 values each);
+// lane l handles vectors l, l + 32, ... of the span, so every load of the warp
+// is 32 consecutive 16-byte vectors. When a span fits in two tokens' rows
+// (V >= 32 * U, the WARP_META variant), lanes 0..K-1 classify the first token's
+// pairs and lanes 16..16+K-1 the second's, once for the whole span, and every
+// lane takes its token's metadata by shuffle. (Narrower rows: every thread
+// classifies its own token's pairs.) Every row a pair reads is loaded in one
+// batch before the sum in ascending k.
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool WARP_META>
 __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>()))
     combine_fwd_kernel(CombineArgs a) {
   constexpr int U = fwd_vectors_per_thread<KMAX>();
@@ -157,7 +156,7 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
   uint4 val[U][KMAX];
   int kind[U][KMAX], row[U][KMAX];
   float wt[U][KMAX];
-  if (SHARED) {  // the launcher picks SHARED only when V >= 32 * U
+  if (WARP_META) {  // the launcher picks WARP_META only when V >= 32 * U
     const int t0 = span / V;
     const int tm = t0 + (lane >> 4), km = lane & 15;
     const bool mine = km < K && tm < a.bs;
@@ -217,6 +216,10 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
       else if (SPECIAL && (kd == kCopy || kd == kConst))
         val[u][j] = ld_nc_v4(ORI + static_cast<size_t>(row[u][j]) * V + v);
     }
+    // the shared-expert row, added last, goes to L2 meanwhile (else it costs a
+    // second DRAM round trip after the sum: DSv3-shaped step 443.9 -> 441.6 us)
+    if (!UNIT && a.shared != nullptr && item < n)
+      prefetch_l2(static_cast<const uint4*>(a.shared) + item);
   }
 #pragma unroll
   for (int u = 0; u < U; ++u) {
