@@ -47,6 +47,10 @@ __device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int
 #pragma unroll
     for (int k = 0; k < KM; ++k) ids[k] = k < a.K ? __ldg(row + k) : -1;
   }
+  // the mask is loaded with the ids, not after them (one DRAM round trip)
+  bool act[KM];
+#pragma unroll
+  for (int k = 0; k < KM; ++k) act[k] = k < a.K && pair_active(a.mask, a.mask_ndim, t, k, a.K);
   uint32_t st = 0;
 #pragma unroll
   for (int k = 0; k < KM; ++k) {
@@ -64,7 +68,7 @@ __device__ __forceinline__ uint32_t classify_row(const LayoutArgs& a, int t, int
       st |= MOE_DEV_DUP_ID;
       continue;
     }
-    if (id < a.E && pair_active(a.mask, a.mask_ndim, t, k, a.K)) e[k] = id;
+    if (id < a.E && act[k]) e[k] = id;
   }
   return st;
 }
@@ -150,19 +154,6 @@ __device__ __forceinline__ int2 block_exclusive_scan2(int2 v, int2* warp_sums, i
   return make_int2(before.x + inc.x - v.x, before.y + inc.y - v.y);
 }
 
-// Writes both halves of assist_info for token t's pairs given their slots.
-template <int KM>
-__device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const int (&e)[KM],
-                                            const int (&slot)[KM]) {
-  const size_t A = static_cast<size_t>(a.A);
-#pragma unroll
-  for (int k = 0; k < KM; ++k) {
-    if (k >= a.K) continue;
-    const int tk = t * a.K + k;
-    if (e[k] >= 0) a.assist[slot[k]] = tk;
-    a.assist[A + tk] = e[k] >= 0 ? slot[k] : -1;
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Cluster layout. CTA r of the cluster (CS <= 8 CTAs of 1024 threads) takes the
@@ -221,13 +212,15 @@ struct alignas(8) BaseOfs {
 
 // mp[tpt][nt / 32][S], bo[E], tot[E] (cluster kernel and fused dispatch, nt
 // threads); the cluster kernel also keeps its pairs in expert order,
-// ltk[tpt * nt * K].
+// ltk[tpt * nt * K], and when `flat`, each list entry's expert,
+// lex[tpt * nt * K] (16-bit).
 __host__ __device__ constexpr size_t cluster_smem_bytes(int E, int tpt, int nt = 1024) {
   return static_cast<size_t>(tpt) * (nt / 32) * cluster_stride(E) * sizeof(MaskPre) +
          static_cast<size_t>(E) * (4 + sizeof(BaseOfs));
 }
-__host__ __device__ constexpr size_t cluster_kernel_smem_bytes(int E, int tpt, int K, int nt) {
-  return cluster_smem_bytes(E, tpt, nt) + static_cast<size_t>(tpt) * nt * K * 4;
+__host__ __device__ constexpr size_t cluster_kernel_smem_bytes(int E, int tpt, int K, int nt,
+                                                               bool flat = false) {
+  return cluster_smem_bytes(E, tpt, nt) + static_cast<size_t>(tpt) * nt * K * (flat ? 6 : 4);
 }
 
 // The slot -> pair half of assist_info for a block's routed pairs, written run
@@ -244,12 +237,68 @@ __device__ __forceinline__ void write_runs(const LayoutArgs& a, const int* first
   }
 }
 
+// The same from a list that also records each entry's expert (lex[p]): thread
+// i writes list positions i, i + NT, ... (four loads in flight), so
+// neighbouring threads write neighbouring slots however short the runs are.
+__device__ __forceinline__ void write_flat(const LayoutArgs& a, const BaseOfs* bo,
+                                           const uint16_t* lex, const int* ltk, int n) {
+  const int nt = static_cast<int>(blockDim.x);
+  for (int p0 = threadIdx.x; p0 < n; p0 += 4 * nt) {
+    int v[4], s[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = p0 + q * nt;
+      s[q] = -1;
+      if (p < n) {
+        const BaseOfs b = bo[lex[p]];
+        s[q] = b.first + (p - b.lofs);
+        v[q] = ltk[p];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (s[q] >= 0) a.assist[s[q]] = v[q];
+  }
+}
+
+// Token t's K pair -> slot entries (assist[A + t K + k]), with 16- or 8-byte
+// stores when K and A allow them (K consecutive ints per thread).
+template <int KM>
+__device__ __forceinline__ void store_pair_slots(const LayoutArgs& a, int t, const int (&slot)[KM]) {
+  int* dst = a.assist + static_cast<size_t>(a.A) + static_cast<size_t>(t) * a.K;
+  const uintptr_t addr = reinterpret_cast<uintptr_t>(dst);
+  if (KM >= 4 && (a.K & 3) == 0 && (addr & 15) == 0) {
+#pragma unroll
+    for (int q = 0; q < KM / 4; ++q)
+      if (4 * q < a.K)
+        reinterpret_cast<int4*>(dst)[q] =
+            make_int4(slot[4 * q], slot[4 * q + 1], slot[4 * q + 2], slot[4 * q + 3]);
+  } else if (KM >= 2 && (a.K & 1) == 0 && (addr & 7) == 0) {
+#pragma unroll
+    for (int q = 0; q < KM / 2; ++q)
+      if (2 * q < a.K) reinterpret_cast<int2*>(dst)[q] = make_int2(slot[2 * q], slot[2 * q + 1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < KM; ++k)
+      if (k < a.K) dst[k] = slot[k];
+  }
+}
+
+// Writes both halves of assist_info for token t's pairs given their slots (-1
+// for a pair that is not routed).
+template <int KM>
+__device__ __forceinline__ void write_slots(const LayoutArgs& a, int t, const int (&slot)[KM]) {
+#pragma unroll
+  for (int k = 0; k < KM; ++k)
+    if (k < a.K && slot[k] >= 0) a.assist[slot[k]] = t * a.K + k;
+  store_pair_slots<KM>(a, t, slot);
+}
+
 // Counts this CTA's tokens [t0, t0 + TPT * NT) (one per thread and sub-block)
 // into the lane masks, then per expert the exclusive prefix of the popcounts
-// over (sub-block, warp) into mp[].pre and the CTA's total into tot (warp w
-// scans the columns w, w + NW, ...; lane = warp of the column). mp must be
-// zero on entry; e receives each token's routed experts (-1 elsewhere) and the
-// status bits are ORed into *status.
+// over (sub-block, warp) into mp[].pre and the CTA's total into tot (thread e
+// takes expert e's column). mp must be zero on entry; e receives each token's
+// routed experts (-1 elsewhere) and the status bits are ORed into *status.
 template <int KM, int TPT, int NT>
 __device__ __forceinline__ void cta_count_scan(const LayoutArgs& a, int t0, int S, MaskPre* mp,
                                                int* tot, uint32_t* status, int (&e)[TPT][KM]) {
@@ -272,21 +321,25 @@ __device__ __forceinline__ void cta_count_scan(const LayoutArgs& a, int t0, int 
   }
   if (st) atomicOr(status, st);
   __syncthreads();
-  for (int ex = warp; ex < a.E; ex += NW) {
-    int carry = 0;
+  // one thread per expert column (E <= NT): its popcounts over (sub-block,
+  // warp), eight entries loaded together at a time, their running sum stored as
+  // each entry's prefix, and the CTA's total
+  if (static_cast<int>(threadIdx.x) < a.E) {
+    const int ex = threadIdx.x;
+    constexpr int N = TPT * NW, CH = N < 8 ? N : 8;
+    int run = 0;
 #pragma unroll
-    for (int i = 0; i < TPT; ++i) {
-      const int c = lane < NW ? __popc(mp[(i * NW + lane) * S + ex].mask) : 0;
-      int inc = c;
+    for (int i0 = 0; i0 < N; i0 += CH) {
+      int c[CH];
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, d);
-        if (lane >= d) inc += n;
+      for (int i = 0; i < CH; ++i) c[i] = __popc(mp[(i0 + i) * S + ex].mask);
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        mp[(i0 + i) * S + ex].pre = static_cast<uint32_t>(run);
+        run += c[i];
       }
-      if (lane < NW) mp[(i * NW + lane) * S + ex].pre = static_cast<uint32_t>(carry + inc - c);
-      carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
     }
-    if (lane == 0) tot[ex] = carry;
+    tot[ex] = run;
   }
 }
 
@@ -298,7 +351,7 @@ __device__ __forceinline__ int cta_rank(const MaskPre* mp, int i, int S, int ex)
 }
 
 template <int KM, int TPT, int NT>
-__global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
+__global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a, int flat) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int2 warp_sums2[32];
   __shared__ uint32_t status, status_all;
@@ -309,6 +362,7 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
                                                       sizeof(MaskPre));
   int* tot = reinterpret_cast<int*>(bo + E);
   int* ltk = tot + E;
+  uint16_t* lex = reinterpret_cast<uint16_t*>(ltk + TPT * NT * a.K);  // when flat
   const uint32_t rank = cluster_ctarank(), cs = cluster_nctarank();
   pdl_trigger();
   for (int i = threadIdx.x; i < TPT * (NT / 32) * S; i += NT) mp[i] = MaskPre{0u, 0u};
@@ -350,7 +404,7 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
   int2 totals;
   const int2 ex2 = block_exclusive_scan2(
       threadIdx.x < E ? make_int2(grand, tot[threadIdx.x]) : make_int2(0, 0), warp_sums2, &totals);
-  const int total = totals.x;
+  const int total = totals.x, listed = totals.y;
   const int excl = ex2.x, lexcl = ex2.y;
   if (threadIdx.x < E) {
     bo[threadIdx.x] = BaseOfs{excl + before, lexcl};
@@ -365,29 +419,38 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a) {
     if (a.dev_status) *a.dev_status = status_all;
   }
   // pair -> slot per token (contiguous per thread); each pair's t * K + k into
-  // the block's expert-ordered list for the slot -> pair half
-  const size_t A = static_cast<size_t>(a.A);
+  // the block's expert-ordered list for the slot -> pair half. Every pair's
+  // rank and base are loaded before any store, so the loads overlap.
 #pragma unroll
   for (int i = 0; i < TPT; ++i) {
     const int t = t0 + i * NT + threadIdx.x;
     if (t >= a.bs) continue;
+    int slot[KM], pos[KM];
 #pragma unroll
     for (int k = 0; k < KM; ++k) {
-      if (k >= a.K) continue;
+      slot[k] = -1;
+      pos[k] = 0;
       const int ex = e[i][k];
-      const int tk = t * a.K + k;
-      int slot = -1;
-      if (ex >= 0) {
+      if (k < a.K && ex >= 0) {
         const int r = cta_rank<NT>(mp, i, S, ex);
         const BaseOfs b = bo[ex];
-        slot = b.first + r;
-        ltk[b.lofs + r] = tk;
+        slot[k] = b.first + r;
+        pos[k] = b.lofs + r;
       }
-      a.assist[A + tk] = slot;
     }
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      if (k >= a.K || slot[k] < 0) continue;
+      ltk[pos[k]] = t * a.K + k;
+      if (flat) lex[pos[k]] = static_cast<uint16_t>(e[i][k]);
+    }
+    store_pair_slots<KM>(a, t, slot);
   }
   __syncthreads();
-  write_runs(a, &bo[0].first, tot, &bo[0].lofs, ltk, 2);
+  if (flat)
+    write_flat(a, bo, lex, ltk, listed);
+  else
+    write_runs(a, &bo[0].first, tot, &bo[0].lofs, ltk, 2);
   for (int s = total + static_cast<int>(rank * blockDim.x + threadIdx.x); s < a.A;
        s += static_cast<int>(cs * blockDim.x))
     a.assist[s] = -1;
@@ -445,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1) dispatch_small_kernel(LayoutArgs a, con
     for (int k = 0; k < KM; ++k)
       slot[k] = (k < a.K && e[0][k] >= 0) ? bo[e[0][k]].first + cta_rank<NT>(mp, 0, S, e[0][k])
                                           : -1;
-    if (writer) write_slots<KM>(a, t, e[0], slot);
+    if (writer) write_slots<KM>(a, t, slot);
     if (t >= t0 && t < t0 + per) {
 #pragma unroll
       for (int k = 0; k < KM; ++k)
@@ -725,7 +788,9 @@ bool cluster_layout_applies(int bs, int E, int K) {
 template <int KM, int TPT, int NT>
 cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st, bool* fits) {
   constexpr auto kernel = layout_cluster_kernel<KM, TPT, NT>;
-  const size_t smem = cluster_kernel_smem_bytes(a.E, TPT, a.K, NT);
+  // the flat slot -> pair writer when its expert list fits as well
+  const int flat = cluster_kernel_smem_bytes(a.E, TPT, a.K, NT, true) <= kClusterSmemMax ? 1 : 0;
+  const size_t smem = cluster_kernel_smem_bytes(a.E, TPT, a.K, NT, flat != 0);
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
@@ -761,7 +826,7 @@ cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st, bool* fi
     return cudaSuccess;
   }
   *fits = true;
-  return cudaLaunchKernelEx(&cfg, kernel, a);
+  return cudaLaunchKernelEx(&cfg, kernel, a, flat);
 }
 
 template <int KM>
