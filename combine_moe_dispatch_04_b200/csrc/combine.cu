@@ -156,8 +156,10 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
   uint4 val[U][KMAX];
   int kind[U][KMAX], row[U][KMAX];
   float wt[U][KMAX];
+  int col[U];  // each vector's column in its row (one division per span)
   if (WARP_META) {  // the launcher picks WARP_META only when V >= 32 * U
     const int t0 = span / V;
+    const int v0 = span - t0 * V;
     const int tm = t0 + (lane >> 4), km = lane & 15;
     const bool mine = km < K && tm < a.bs;
     PairMeta m{kSkip, 0, 1.0f};
@@ -176,7 +178,14 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int item = span + u * 32 + lane;
-      const int src_base = item / V == t0 ? 0 : 16;
+      // the span's first token, or the next one past its end (V >= 32 * U: at
+      // most one wrap)
+      int src_base = 0;
+      col[u] = v0 + u * 32 + lane;
+      if (col[u] >= V) {
+        col[u] -= V;
+        src_base = 16;
+      }
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         kind[u][j] = __shfl_sync(0xFFFFFFFFu, m.kind, src_base + j);
@@ -189,12 +198,14 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int item = span + u * 32 + lane;
+      const int t = item / V;
+      col[u] = item - t * V;
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         kind[u][j] = kSkip;
         wt[u][j] = 1.0f;
         if (j >= K || item >= n) continue;
-        const PairMeta m = classify_pair<SPECIAL, UNIT, true, true>(a, item / V, j);
+        const PairMeta m = classify_pair<SPECIAL, UNIT, true, true>(a, t, j);
         kind[u][j] = m.kind;
         row[u][j] = m.row;
         wt[u][j] = m.w;
@@ -206,8 +217,7 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
   const uint4* ORI = static_cast<const uint4*>(a.ori_x);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    const int item = span + u * 32 + lane;
-    const int v = item % V;
+    const int v = col[u];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       const int kd = SPECIAL ? (kind[u][j] & 7) : kind[u][j];
@@ -216,16 +226,21 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
       else if (SPECIAL && (kd == kCopy || kd == kConst))
         val[u][j] = ld_nc_v4(ORI + static_cast<size_t>(row[u][j]) * V + v);
     }
-    // the shared-expert row, added last, goes to L2 meanwhile (else it costs a
-    // second DRAM round trip after the sum: DSv3-shaped step 443.9 -> 441.6 us)
-    if (!UNIT && a.shared != nullptr && item < n)
-      prefetch_l2(static_cast<const uint4*>(a.shared) + item);
+  }
+  // the shared-expert row, added last, goes to L2 meanwhile (else it costs a
+  // second DRAM round trip after the sum: DSv3-shaped step 443.9 -> 441.6 us)
+  if (!UNIT && a.shared != nullptr) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = span + u * 32 + lane;
+      if (item < n) prefetch_l2(static_cast<const uint4*>(a.shared) + item);
+    }
   }
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int item = span + u * 32 + lane;
     if (item >= n) continue;
-    const int v = item % V;
+    const int v = col[u];
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
@@ -319,6 +334,7 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, false>() - 
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
   // lanes 0..K-1 classify the span's first token's pairs, lanes 16..16+K-1 the next one's
   const int t0 = span / V;
+  const int v0 = span - t0 * V;
   const int tm = t0 + (lane >> 4), km = lane & 15;
   PairMeta pm{kSkip, 0, 1.0f};
   if (km < K && tm < a.bs) pm = classify_pair<false, false, false>(a, tm, km);
@@ -329,8 +345,12 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, false>() - 
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int item = span + u * 32 + lane;
-    const int v = item % V;
-    src[u] = item / V == t0 ? 0 : 16;
+    int v = v0 + u * 32 + lane;  // past the first token's row: the next one's
+    src[u] = 0;
+    if (v >= V) {
+      v -= V;
+      src[u] = 16;
+    }
     routed[u] = 0;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
