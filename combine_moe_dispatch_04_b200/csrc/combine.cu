@@ -92,7 +92,9 @@ __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, i
   // With special experts the id and the slot are loaded together, so the pair
   // costs one round trip instead of two (the slot load would otherwise wait for
   // the id's range check). Without them the slot is loaded after the mask test,
-  // which measured faster (8192-token step 195.8 vs 199.6 us).
+  // which measured faster (8192-token step 195.8 vs 199.6 us; loading it with
+  // the mask byte instead gained nothing on the masked Mixtral-shaped step and
+  // cost the 8192-token one 2 us).
   if (!UNIT) m.w = __ldg(a.weights + tk);
   int s = -1;
   if (SPECIAL) s = __ldg(a.assist + static_cast<size_t>(a.A) + tk);
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
       const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
       bool dup = false;
 #pragma unroll
-      for (int jj = 0; jj < 15; ++jj) {
+      for (int jj = 0; jj < KMAX - 1; ++jj) {  // km < K <= KMAX
         const int other = __shfl_sync(0xFFFFFFFFu, id, (lane & 16) | jj);
         dup |= jj < km && other == id;
       }

@@ -95,9 +95,10 @@ __device__ __forceinline__ float absmax_final(uint32_t acc) {
 
 // Packed fp32 pairs: __fadd2_rn / __fmul2_rn / __ffma2_rn, one instruction
 // per pair. A packed product that feeds a packed sum was observed to lose its
-// own rounding on B200 (outputs one ulp off), so every product that is then
-// added is a scalar __fmul_rn (never contracted); packed multiplies only feed
-// other multiplies or stores.
+// own rounding on B200 (outputs one ulp off), with the intrinsic and with an
+// inline PTX mul.rn.f32x2 alike, so every product that is then added is a
+// scalar __fmul_rn (never contracted); packed multiplies only feed other
+// multiplies or stores.
 __device__ __forceinline__ float2 f2(float lo, float hi) { return make_float2(lo, hi); }
 
 // acc[i] = acc[i] + w * m[i] for 8 values, product and sum each rounded once
