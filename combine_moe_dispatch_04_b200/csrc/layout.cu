@@ -182,6 +182,19 @@ __device__ __forceinline__ void cluster_arrive_release() {
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// First half of a cluster barrier that orders nothing (this CTA has started),
+// and the matching wait.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+// Stores v into the shared memory of CTA `rank` of this cluster, at the
+// position of `local` in this CTA's shared memory.
+__device__ __forceinline__ void st_dsmem_u32(void* local, uint32_t rank, uint32_t v) {
+  const uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+  uint32_t raddr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(addr), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(raddr), "r"(v) : "memory");
+}
 // A 32-bit word of the shared memory of CTA `rank` of this cluster, at the
 // position of `local` in this CTA's shared memory.
 __device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t rank) {
@@ -350,8 +363,16 @@ __device__ __forceinline__ int cta_rank(const MaskPre* mp, int i, int S, int ex)
   return static_cast<int>(m.pre) + __popc(m.mask & lanemask_lt());
 }
 
+// Two ways to exchange the per-expert totals. With `push` (when cs * E + 16
+// ints fit in the pair-list area, which is not yet in use), every CTA stores
+// its totals (and its status word, for CTA 0) into every CTA's shared memory
+// before one cluster barrier, after which all reads are local; a first
+// barrier, arrived at on entry, makes sure every CTA has started before any
+// store reaches it. Otherwise each CTA loads the others' totals after the
+// barrier, and a second barrier keeps every CTA alive until those loads are
+// done.
 template <int KM, int TPT, int NT>
-__global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a, int flat) {
+__global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a, int flat, int push) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int2 warp_sums2[32];
   __shared__ uint32_t status, status_all;
@@ -364,7 +385,10 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a, int
   int* ltk = tot + E;
   uint16_t* lex = reinterpret_cast<uint16_t*>(ltk + TPT * NT * a.K);  // when flat
   const uint32_t rank = cluster_ctarank(), cs = cluster_nctarank();
+  int* xch = ltk;           // push: [cs][E] totals, then [cs] status words
+  int* xst = ltk + cs * E;  //   (the pair list is written only after they are read)
   pdl_trigger();
+  if (push) cluster_arrive_relaxed();  // this CTA has started
   for (int i = threadIdx.x; i < TPT * (NT / 32) * S; i += NT) mp[i] = MaskPre{0u, 0u};
   if (threadIdx.x == 0) {
     status = 0;
@@ -376,28 +400,48 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a, int
   const int t0 = static_cast<int>(rank) * TPT * NT;
   int e[TPT][KM];
   cta_count_scan<KM, TPT, NT>(a, t0, S, mp, tot, &status, e);
-  __syncwarp();
-  cluster_arrive_release();  // tot and status are published to the cluster
-  cluster_wait_acquire();
-
-  // grand totals and the pairs of the CTAs before this one, per expert (all the
-  // remote loads are issued before any is used)
   int grand = 0, before = 0;
-  if (threadIdx.x < E) {
-    int v[kClusterMaxCtas];
-#pragma unroll
-    for (int c = 0; c < kClusterMaxCtas; ++c)
-      v[c] = c < static_cast<int>(cs) ? static_cast<int>(ld_dsmem_u32(tot + threadIdx.x, c)) : 0;
-#pragma unroll
-    for (int c = 0; c < kClusterMaxCtas; ++c) {
-      grand += v[c];
-      before += c < static_cast<int>(rank) ? v[c] : 0;
-    }
-  }
   uint32_t cst = 0;
-  if (rank == 0 && threadIdx.x < cs) cst = ld_dsmem_u32(&status, threadIdx.x);
-  __syncwarp();
-  cluster_arrive_release();  // done reading the other CTAs' shared memory
+  if (push) {
+    __syncwarp();
+    cluster_wait_acquire();  // every CTA of the cluster has started
+    if (threadIdx.x < E) {
+      const uint32_t mine = static_cast<uint32_t>(tot[threadIdx.x]);
+      for (uint32_t c = 0; c < cs; ++c) st_dsmem_u32(xch + rank * E + threadIdx.x, c, mine);
+    }
+    if (threadIdx.x == 0) st_dsmem_u32(xst + rank, 0, status);
+    __syncwarp();
+    cluster_arrive_release();  // the stores are published to the cluster
+    cluster_wait_acquire();
+    if (threadIdx.x < E) {
+      for (int c = 0; c < static_cast<int>(cs); ++c) {
+        const int v = xch[c * E + threadIdx.x];
+        grand += v;
+        before += c < static_cast<int>(rank) ? v : 0;
+      }
+    }
+    if (rank == 0 && threadIdx.x < cs) cst = static_cast<uint32_t>(xst[threadIdx.x]);
+  } else {
+    __syncwarp();
+    cluster_arrive_release();  // tot and status are published to the cluster
+    cluster_wait_acquire();
+    // grand totals and the pairs of the CTAs before this one, per expert (all
+    // the remote loads are issued before any is used)
+    if (threadIdx.x < E) {
+      int v[kClusterMaxCtas];
+#pragma unroll
+      for (int c = 0; c < kClusterMaxCtas; ++c)
+        v[c] = c < static_cast<int>(cs) ? static_cast<int>(ld_dsmem_u32(tot + threadIdx.x, c)) : 0;
+#pragma unroll
+      for (int c = 0; c < kClusterMaxCtas; ++c) {
+        grand += v[c];
+        before += c < static_cast<int>(rank) ? v[c] : 0;
+      }
+    }
+    if (rank == 0 && threadIdx.x < cs) cst = ld_dsmem_u32(&status, threadIdx.x);
+    __syncwarp();
+    cluster_arrive_release();  // done reading the other CTAs' shared memory
+  }
   if (cst) atomicOr(&status_all, cst);
   // exclusive scans over the experts of the grand totals (global first slots) and
   // of this CTA's totals (positions in its expert-ordered pair list)
@@ -454,8 +498,10 @@ __global__ void __launch_bounds__(NT, 1) layout_cluster_kernel(LayoutArgs a, int
   for (int s = total + static_cast<int>(rank * blockDim.x + threadIdx.x); s < a.A;
        s += static_cast<int>(cs * blockDim.x))
     a.assist[s] = -1;
-  __syncwarp();
-  cluster_wait_acquire();  // no CTA leaves while another may still read its tot
+  if (!push) {
+    __syncwarp();
+    cluster_wait_acquire();  // no CTA leaves while another may still read its tot
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -759,6 +805,9 @@ cudaError_t launch_dispatch_small_k(const LayoutArgs& a, const void* x, void* ex
 // The cluster layout: CS <= 16 CTAs of NT threads, one token per thread: 256
 // threads for up to 256 tokens and experts (one block), 512 up to 8192 tokens
 // and E <= 512, so that up to 16 SMs share the work, else 1024.
+#ifndef MOE_LAYOUT_PUSH
+#define MOE_LAYOUT_PUSH 1
+#endif
 #ifndef MOE_LAYOUT_CLUSTER_MAX_TOKENS
 #define MOE_LAYOUT_CLUSTER_MAX_TOKENS (16 * 1024)
 #endif
@@ -790,6 +839,11 @@ cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st, bool* fi
   constexpr auto kernel = layout_cluster_kernel<KM, TPT, NT>;
   // the flat slot -> pair writer when its expert list fits as well
   const int flat = cluster_kernel_smem_bytes(a.E, TPT, a.K, NT, true) <= kClusterSmemMax ? 1 : 0;
+  int cs_launch = (a.bs + TPT * NT - 1) / (TPT * NT);
+  if (cs_launch < 1) cs_launch = 1;
+  // the pushed exchange when its [cs][E] totals and [cs] status words fit the
+  // pair-list area
+  const int push = MOE_LAYOUT_PUSH && cs_launch * (a.E + 1) <= TPT * NT * a.K ? 1 : 0;
   const size_t smem = cluster_kernel_smem_bytes(a.E, TPT, a.K, NT, flat != 0);
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -826,7 +880,7 @@ cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t st, bool* fi
     return cudaSuccess;
   }
   *fits = true;
-  return cudaLaunchKernelEx(&cfg, kernel, a, flat);
+  return cudaLaunchKernelEx(&cfg, kernel, a, flat, push);
 }
 
 template <int KM>

@@ -55,8 +55,29 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
   const int C = H / 16;  // chunks per row
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
-  for (int t = blockIdx.x; t < bs; t += gridDim.x) {
+  // the CTA's next token row is requested while the current one is quantised
+  // and stored (raw 16-bit values, two 16-byte vectors per chunk)
+  uint4 next[CPT][2];
+  auto load_row = [&](int t) {
     const uint4* xr = x + static_cast<size_t>(t) * (H / 8);
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = threadIdx.x + j * blockDim.x;
+      if (c < C) {
+        next[j][0] = ld_nc_v4(xr + 2 * c);
+        next[j][1] = ld_nc_v4(xr + 2 * c + 1);
+      }
+    }
+  };
+  if (blockIdx.x < bs) load_row(blockIdx.x);
+  for (int t = blockIdx.x; t < bs; t += gridDim.x) {
+    uint4 cur[CPT][2];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      cur[j][0] = next[j][0];
+      cur[j][1] = next[j][1];
+    }
+    if (t + static_cast<int>(gridDim.x) < bs) load_row(t + gridDim.x);
     const int32_t* slots = assist + static_cast<size_t>(A) + static_cast<size_t>(t) * K;
     const int my_slot = lane < K ? __ldg(slots + lane) : -1;  // every warp holds the K slots
     float f[CPT][16];
@@ -66,8 +87,8 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
       const int c = threadIdx.x + j * blockDim.x;
       if (c < C) {
         float lo[8], hi[8];
-        widen8<T16>(ld_nc_v4(xr + 2 * c), lo);
-        widen8<T16>(ld_nc_v4(xr + 2 * c + 1), hi);
+        widen8<T16>(cur[j][0], lo);
+        widen8<T16>(cur[j][1], hi);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           f[j][i] = lo[i];
