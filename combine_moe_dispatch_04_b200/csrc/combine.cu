@@ -628,9 +628,13 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
     const int lkind = lane < K ? lpm.kind : static_cast<int>(kSkip);
     const float lw = lpm.w;
     const uint32_t routed = __ballot_sync(0xFFFFFFFFu, lkind == kRouted);
-    // zero experts too: their +0 terms can change the sign of a zero sum
-    const bool any_special = __any_sync(0xFFFFFFFFu, lkind == kZero || lkind == kCopy || lkind == kConst);
+    const uint32_t zerom = SPECIAL ? __ballot_sync(0xFFFFFFFFu, lkind == kZero) : 0u;
+    const uint32_t copym = SPECIAL ? __ballot_sync(0xFFFFFFFFu, lkind == kCopy) : 0u;
+    const uint32_t constm = SPECIAL ? __ballot_sync(0xFFFFFFFFu, lkind == kConst) : 0u;
     const uint32_t fastm = __ballot_sync(0xFFFFFFFFu, rm == 0.0f || rs >= kFastMinScale);
+    // routed rows with a scale too small for the fast reciprocal take the
+    // general path below (IEEE divisions); everything else the loop here
+    const bool tiny = (routed & ~fastm) != 0u;
     // Whole warps walk the vectors (the shuffles below need every lane); a lane
     // past the row end works on vector 0 and stores nothing.
     for (int v0 = warp * 32; v0 < V; v0 += kQ8sConsumers) {
@@ -640,33 +644,41 @@ __global__ void __launch_bounds__(kQ8sThreads, 2) combine_fwd_q8s_kernel(Combine
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-      uint32_t redo = any_special ? 1u : 0u;
-      if (!redo) {
-        // Routed rows only: every row computed without a branch, its terms
-        // selected in (unselected ones add -0, which leaves any sum as it is).
+      if (!tiny) {
+        // one pair at a time in ascending k, each term added as in the
+        // oracle; the branches follow the token's pair kinds (warp-uniform)
+        float ori[8];
+        if (SPECIAL && (copym | constm) != 0u)  // requested before the loop
+          widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
 #pragma unroll 1
         for (int j = 0; j < KMAX; ++j) {
           const float rfj = __shfl_sync(0xFFFFFFFFu, rf, j);
           const float rsj = __shfl_sync(0xFFFFFFFFu, rs, j);
           const float wj = __shfl_sync(0xFFFFFFFFu, lw, j);
-          float y[8], n[8], b[8], prod[8];
-          widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
-          quant_codes8<false>(y, rsj, rfj, true, n, b);  // exact, ties included
-          const bool use = (routed >> j) & 1u;
-          redo |= (use && !((fastm >> j) & 1u)) ? 1u : 0u;  // a tiny scale: IEEE divisions
+          float prod[8];
+          if ((routed >> j) & 1u) {
+            float y[8], n[8], b[8];
+            widen8<T16>(brows[static_cast<size_t>(j) * V + v], y);
+            quant_codes8<false>(y, rsj, rfj, true, n, b);  // exact, ties included
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float p = __fmul_rn(wj, __fmul_rn(n[i], rsj));
-            prod[i] = use ? p : -0.0f;
+            for (int i = 0; i < 8; ++i) prod[i] = __fmul_rn(wj, __fmul_rn(n[i], rsj));
+          } else if (SPECIAL && ((zerom | copym | constm) >> j) & 1u) {
+            const int kind = (zerom >> j) & 1u ? kZero : (copym >> j) & 1u ? kCopy : kConst;
+            float m[8];
+            pair_values<T16, SPECIAL>(a, kind, pmeta[j].row, V, v, make_uint4(0, 0, 0, 0), ori, m);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) prod[i] = __fmul_rn(wj, m[i]);
+          } else {
+            continue;
           }
           add8_rn(acc, prod);
         }
       }
-      // special pairs, or a row with a tiny scale: the general path
-      // (the shuffles need the whole warp, so every lane walks it when any does)
-      if (__any_sync(0xFFFFFFFFu, redo != 0u)) {
+      uint32_t redo = tiny ? 1u : 0u;
+      // a routed row with a tiny scale: the general path (warp-uniform)
+      if (redo != 0u) {
         float ori[8];
-        if (SPECIAL && any_special && a.ori_x != nullptr)
+        if (SPECIAL && (copym | constm) != 0u)
           widen8<T16>(ld_nc_v4(static_cast<const uint4*>(a.ori_x) + item), ori);
         float acc2[8];
 #pragma unroll
