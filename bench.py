@@ -54,6 +54,7 @@ FALLBACK_HBM_GBS = 6650.0
 KERNELS = ("layout", "permute", "combine_fwd", "combine_bwd", "combine_bwd_special",
            "dispatch_bwd")
 DOM_EVERY = 4
+FUSED_DISPATCH_MAX_TOKENS = 1024  # moe_dispatch is one launch up to this batch
 DROP_TOP = 3          # slowest steps dropped before the mean and std
 ACCEPT_CV = 0.02      # std / mean at or below which a run is accepted
 MAX_RUNS = 5          # runs of one workload before the best one is kept
@@ -830,12 +831,15 @@ def main():
                     "clocks")}
             else:
                 pc_args = argparse.Namespace(**vars(args))
-                pc_args.fused_dispatch = False
+                # small batches take the one-launch dispatch (layout + permute), the
+                # library's call for them; the others the two calls
+                pc_args.fused_dispatch = w.bs <= FUSED_DISPATCH_MAX_TOKENS
                 pc_args.combine_comm_quant = 0
                 bw = Bench(w, pc_args, dev, rank)
                 rw = bw.accepted_run(args.per_config_steps, args.warmup, flush_l2, world, rank,
                                      uuid)
                 per_config[w.name] = bw.summary(rw, peak)
+                per_config[w.name]["fused_dispatch"] = pc_args.fused_dispatch
                 del bw
                 torch.cuda.empty_cache()
             pc = per_config[w.name]
