@@ -76,11 +76,16 @@ EDGE = [
     _custom("fp16_quant", bs=1030, h=2064, dtype="fp16", quant_mode=2, expert="dequant",
             backward=False),
     _custom("zipf_hot", bs=2048, k=2, num_experts=300, routing="zipf", zipf_s=3.0),
-    # layout paths: the cluster kernel with 16 blocks of 512 and of 1024 threads, then
-    # the tiled count / column-scan / scatter path where the cluster's shared memory
-    # does not suffice, just above its token limit, and at 65536 tokens with E = 1024
+    # layout paths: the cluster kernel with 16 blocks of 512 and of 1024 threads (its
+    # totals pushed to every block, or, at E = 512 with K = 16 where 16 x 513 totals do
+    # not fit the pair-list area, loaded after the barrier; its slot -> pair entries
+    # written per list entry, or, at E = 700 with K = 6 where the expert list does not
+    # fit, per expert run), then the tiled count / column-scan / scatter path where the
+    # cluster's shared memory does not suffice, just above its token limit, and at
+    # 65536 tokens with E = 1024
     _custom("cluster16_e512_k16", bs=8192, k=16, num_experts=512, h=64),
     _custom("cluster_e700_1024_threads", bs=1500, k=4, num_experts=700, h=64),
+    _custom("cluster_runs_e700_k6", bs=1500, k=6, num_experts=700, h=64),
     _custom("cluster_1024_threads", bs=16384, k=8, num_experts=256, h=64, mask_ndim=1,
             mask_false_p=0.2, backward=False),
     _custom("tiled_k16_e1024", bs=12000, k=16, num_experts=1024, h=64),
