@@ -122,6 +122,10 @@ __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, i
   return m;
 }
 
+// Sixteen-byte vectors of zeros that skipped pairs read (branch-free sum).
+constexpr int kZeroVecs = 64;
+__device__ uint4 g_zero_vecs[kZeroVecs];
+
 // Resident blocks per SM the forward kernel is compiled for (a register cap
 // that avoids spills for each variant). For the special-expert variant with
 // K <= 8: at 4 (64 registers, a few bytes of spill) it ran 67 us against 76 us
@@ -146,6 +150,12 @@ template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool WARP_META>
 __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>()))
     combine_fwd_kernel(CombineArgs a) {
   constexpr int U = fwd_vectors_per_thread<KMAX>();
+  // the branch-free sum (below) where it measured faster: unit weights (DSv3-shaped
+  // dispatch backward 87.7 -> 87.3 us, Mixtral-shaped 65.9 -> 62.5) and K > 4
+  // without special experts (DSv3-shaped combine 101.4 -> 98.7); slower with
+  // special experts (64.9 -> 66.9) and for the weighted K <= 4 gather (Mixtral
+  // combine 67.9 -> 86.5)
+  constexpr bool BRANCHFREE = UNIT || (!SPECIAL && KMAX > 4);
   pdl_trigger();
   pdl_wait();
   const int V = a.H / kVecElems;
@@ -217,16 +227,35 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
   // every row a pair reads (a routed row, or the ori_x row of a copy / const
   // pair) is loaded in one batch, before any is used
   const uint4* ORI = static_cast<const uint4*>(a.ori_x);
+  if constexpr (BRANCHFREE) {
+    // A sum that starts at +0 never becomes -0 (x + y is -0 only when both
+    // are), so adding w * 0 never changes it: a skipped pair reads a vector of
+    // zeros with weight 0 (its product is 0 whatever the weight held) and is
+    // summed like the others, without a branch per pair.
+    static_assert(!SPECIAL, "routed and skipped pairs only");
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int v = col[u];
+    for (int u = 0; u < U; ++u) {
+      const int v = col[u];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      const int kd = SPECIAL ? (kind[u][j] & 7) : kind[u][j];
-      if (kd == kRouted)
-        val[u][j] = ld_nc_v4(Y + static_cast<size_t>(row[u][j]) * V + v);
-      else if (SPECIAL && (kd == kCopy || kd == kConst))
-        val[u][j] = ld_nc_v4(ORI + static_cast<size_t>(row[u][j]) * V + v);
+      for (int j = 0; j < KMAX; ++j) {
+        const bool routed = kind[u][j] == kRouted;
+        val[u][j] = ld_nc_v4(routed ? Y + static_cast<size_t>(row[u][j]) * V + v
+                                    : g_zero_vecs + (v & (kZeroVecs - 1)));
+        if (!routed) wt[u][j] = 0.0f;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = col[u];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        const int kd = SPECIAL ? (kind[u][j] & 7) : kind[u][j];
+        if (kd == kRouted)
+          val[u][j] = ld_nc_v4(Y + static_cast<size_t>(row[u][j]) * V + v);
+        else if (SPECIAL && (kd == kCopy || kd == kConst))
+          val[u][j] = ld_nc_v4(ORI + static_cast<size_t>(row[u][j]) * V + v);
+      }
     }
   }
   // the shared-expert row, added last, goes to L2 meanwhile (else it costs a
@@ -249,14 +278,9 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       const int kd = SPECIAL ? (kind[u][j] & 7) : kind[u][j];
-      if (kd == kSkip) continue;
+      if (!BRANCHFREE && kd == kSkip) continue;
       float m[8];
-      if (!SPECIAL || kd == kRouted || kd == kCopy) {
-        widen8<T16>(val[u][j], m);
-      } else if (kd == kZero) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m[i] = 0.0f;
-      } else {  // alpha_1 * ori_x + alpha_2 * v, each product and the sum rounded
+      if (SPECIAL && kd == kConst) {  // alpha_1 * ori_x + alpha_2 * v, each product and the sum rounded
         const size_t r = static_cast<size_t>(kind[u][j] >> 3) * V + v;
         float o[8], a1[8], a2[8], cv[8];
         widen8<T16>(val[u][j], o);
@@ -266,6 +290,11 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           m[i] = __fadd_rn(__fmul_rn(a1[i], o[i]), __fmul_rn(a2[i], cv[i]));
+      } else if (SPECIAL && !BRANCHFREE && kd == kZero) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+      } else {  // a routed or ori_x row (or, branch-free, a vector of zeros)
+        widen8<T16>(val[u][j], m);
       }
       if (UNIT)
         add8_rn(acc, m);
