@@ -531,6 +531,14 @@ __global__ void __launch_bounds__(NT, 1) dispatch_small_kernel(LayoutArgs a, con
   if (threadIdx.x == 0) status = 0;
   __syncthreads();
   pdl_wait();
+  // this CTA's rows are contiguous in x: each thread's first vector is requested
+  // now, so its DRAM round trip overlaps the layout work below
+  const int t0 = blockIdx.x * per;
+  const int t1 = min(a.bs, t0 + per);
+  const int nvec = (t1 - t0) * V;
+  const uint4* xr = x + static_cast<size_t>(t0) * V;
+  uint4 first = make_uint4(0u, 0u, 0u, 0u);
+  if (static_cast<int>(threadIdx.x) < nvec) first = ld_nc_v4(xr + threadIdx.x);
   int e[1][KM];
   cta_count_scan<KM, 1, NT>(a, 0, S, mp, tot, &status, e);
   __syncthreads();
@@ -547,7 +555,6 @@ __global__ void __launch_bounds__(NT, 1) dispatch_small_kernel(LayoutArgs a, con
   if (writer && threadIdx.x == 0) a.ep_send_counts[E] = total;
   __syncthreads();
   const int t = threadIdx.x;
-  const int t0 = blockIdx.x * per;
   if (t < a.bs) {
     int slot[KM];
 #pragma unroll
@@ -566,11 +573,10 @@ __global__ void __launch_bounds__(NT, 1) dispatch_small_kernel(LayoutArgs a, con
     if (threadIdx.x == 0 && a.dev_status) *a.dev_status = status;
   }
   __syncthreads();
-  const int t1 = min(a.bs, t0 + per);
-  for (int i = threadIdx.x; i < (t1 - t0) * V; i += blockDim.x) {
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
     const int tl = i / V;
     const int v = i - tl * V;
-    const uint4 val = ld_nc_v4(x + static_cast<size_t>(t0 + tl) * V + v);
+    const uint4 val = i == static_cast<int>(threadIdx.x) ? first : ld_nc_v4(xr + i);
     for (int k = 0; k < a.K; ++k) {
       const int s = slot_sh[tl][k];
       if (s >= 0) st_v4(expand_x + static_cast<size_t>(s) * V + v, val);
