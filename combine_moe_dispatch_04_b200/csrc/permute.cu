@@ -21,6 +21,7 @@ constexpr int kCopyItems = 2;  // vectors per thread, a block apart
 
 // One thread per 16-byte vector of x (coalesced along the row) in one-shot
 // blocks: the vector is read once and stored to each of the token's K slots.
+template <int KM>
 __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
     int bs, int K, int V, int A) {
@@ -28,19 +29,44 @@ __global__ void __launch_bounds__(kCopyThreads) permute_copy_kernel(
   pdl_wait();
   const int n = bs * V;
   const int32_t* slots_all = assist + static_cast<size_t>(A);
+  // a token's K slots are loaded together (16-byte loads when K and A allow),
+  // then its K stores go out back to back
+  const bool vec4 = KM >= 4 && (K & 3) == 0 && (A & 3) == 0 &&
+                    (reinterpret_cast<uintptr_t>(assist) & 15) == 0;
+  // every item's vector and slots are requested before any store
+  uint4 val[kCopyItems];
+  int s[kCopyItems][KM], v[kCopyItems];
 #pragma unroll
   for (int i = 0; i < kCopyItems; ++i) {
     const int item = (blockIdx.x * kCopyItems + i) * kCopyThreads + threadIdx.x;
-    if (item >= n) return;
+#pragma unroll
+    for (int k = 0; k < KM; ++k) s[i][k] = -1;
+    v[i] = 0;
+    if (item >= n) continue;
     const int t = item / V;
-    const int v = item - t * V;
-    const uint4 val = ld_nc_v4(x + item);
+    v[i] = item - t * V;
+    val[i] = ld_nc_v4(x + item);
     const int32_t* slots = slots_all + static_cast<size_t>(t) * K;
-    for (int k = 0; k < K; ++k) {
-      const int s = __ldg(slots + k);
-      if (s >= 0) st_v4(out + static_cast<size_t>(s) * V + v, val);
+    if (vec4) {
+#pragma unroll
+      for (int q = 0; q < KM / 4; ++q) {
+        int4 w = make_int4(-1, -1, -1, -1);
+        if (4 * q < K) w = __ldg(reinterpret_cast<const int4*>(slots) + q);
+        s[i][4 * q] = w.x;
+        s[i][4 * q + 1] = w.y;
+        s[i][4 * q + 2] = w.z;
+        s[i][4 * q + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < KM; ++k) s[i][k] = k < K ? __ldg(slots + k) : -1;
     }
   }
+#pragma unroll
+  for (int i = 0; i < kCopyItems; ++i)
+#pragma unroll
+    for (int k = 0; k < KM; ++k)
+      if (s[i][k] >= 0) st_v4(out + static_cast<size_t>(s[i][k]) * V + v[i], val[i]);
 }
 
 // CPT 16-element chunks per thread (1, 2 or 4), chosen by the launcher so a
@@ -511,7 +537,11 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
     const long long n = static_cast<long long>(a.bs) * V;
     const int per_block = kCopyThreads * kCopyItems;
     const int blocks = static_cast<int>((n + per_block - 1) / per_block);
-    return launch_pdl(permute_copy_kernel, dim3(blocks), dim3(kCopyThreads), 0, st,
+    const auto kernel = a.K <= 2   ? permute_copy_kernel<2>
+                        : a.K <= 4 ? permute_copy_kernel<4>
+                        : a.K <= 8 ? permute_copy_kernel<8>
+                                   : permute_copy_kernel<16>;
+    return launch_pdl(kernel, dim3(blocks), dim3(kCopyThreads), 0, st,
                       static_cast<const uint4*>(a.x), a.assist, static_cast<uint4*>(a.expand_x),
                       a.bs, a.K, V, a.A);
   }

@@ -449,3 +449,39 @@ def test_combine_bwd_comm_quant_mode2(wl):
     err = np.abs(host(gw).astype(np.float64) - gw_ref.astype(np.float64))
     bound = gpu_chain.GRAD_W_RTOL * np.maximum(np.abs(gw_ref.astype(np.float64)), mag)
     assert np.all(err <= bound), float((err / np.maximum(bound, 1e-30)).max())
+
+
+@pytest.mark.parametrize("k", [8, 2])
+def test_combine_ignores_weights_of_skipped_pairs(k):
+    """Masked pairs, invalid and repeated ids carry NaN weights: combine must
+    leave them out exactly as the oracle does (the K > 4 gather sums a skipped
+    pair as a zero vector with weight 0, so the weight it holds never enters)."""
+    import gpu_chain
+    import oracle
+    import combine_moe_dispatch_04_b200 as moe
+
+    wl = _custom(f"nan_skip_k{k}", bs=900, k=k, num_experts=32, h=256, mask_ndim=2,
+                 mask_false_p=0.3, backward=False)
+    inp = workloads.generate(wl)
+    idx = inp["topk_idx"].copy()
+    idx[::7, 0] = wl.num_experts + 5      # out of range
+    idx[1::11, k - 1] = idx[1::11, 0]     # a repeat of the token's first id
+    w = inp["topk_weights"].copy()
+    skipped = (inp["mask"] == 0)
+    skipped[::7, 0] = True
+    skipped[1::11, k - 1] = True
+    w[skipped] = np.nan
+    _, send, assist, _ = oracle.dispatch_layout(idx, wl.num_experts, wl.n_ids, wl.a_capacity,
+                                                inp["mask"])
+    rng = np.random.default_rng(5)
+    y = workloads.encode16(rng.standard_normal((wl.a_capacity, wl.h)), wl.dtype)
+    want = oracle.combine_fwd(y, idx, w, assist, num_experts=wl.num_experts,
+                              a_capacity=wl.a_capacity, dtype=wl.dtype, mask=inp["mask"])
+    assert not np.isnan(workloads.decode16(want, wl.dtype)).any()
+    sh = gpu_chain.shape_of(wl)
+    idx_d, mask_d = gpu_chain.dev(idx), gpu_chain.dev(inp["mask"])
+    lay = moe.dispatch_layout(sh, idx_d, mask_d)
+    out = moe.combine_fwd(sh, gpu_chain.dev(y, wl.dtype), idx_d, gpu_chain.dev(w), lay,
+                          x_active_mask=mask_d)
+    torch.cuda.synchronize()
+    assert np.array_equal(gpu_chain.host(out), want)
