@@ -36,7 +36,10 @@ unsigned* wait_timeout_counter() {
 
 namespace {
 
-constexpr int kFwdThreads = 256;
+// Threads per block of the weighted gathers: 128-thread blocks (at the same
+// registers, so twice the blocks per SM) ran the special-expert combine in
+// 62.6 us against 65.0 and the Mixtral-shaped one in 66.3 against 68.0.
+constexpr int kFwdThreads = 128;
 
 enum PairKind : int { kSkip = 0, kRouted = 1, kZero = 2, kCopy = 3, kConst = 4 };
 
@@ -126,16 +129,21 @@ __device__ __forceinline__ PairMeta classify_pair(const CombineArgs& a, int t, i
 constexpr int kZeroVecs = 64;
 __device__ uint4 g_zero_vecs[kZeroVecs];
 
-// Resident blocks per SM the forward kernel is compiled for (a register cap
-// that avoids spills for each variant). For the special-expert variant with
-// K <= 8: at 4 (64 registers, a few bytes of spill) it ran 67 us against 76 us
-// at 3 (72 registers, no spill) on the 8192-token H 2048 special workload.
+// Resident blocks per SM the forward kernel is compiled for, counted in
+// 256-thread blocks (a register cap that avoids spills for each variant). For
+// the special-expert variant with K <= 8: at 4 (64 registers, a few bytes of
+// spill) it ran 67 us against 76 us at 3 (72 registers, no spill) on the
+// 8192-token H 2048 special workload.
 #ifndef MOE_FWD_SPECIAL_MIN_BLOCKS
 #define MOE_FWD_SPECIAL_MIN_BLOCKS 4
 #endif
 template <int KMAX, bool SPECIAL>
-__host__ __device__ constexpr int fwd_min_blocks() {
+__host__ __device__ constexpr int fwd_blocks_of_256() {
   return SPECIAL ? (KMAX <= 8 ? MOE_FWD_SPECIAL_MIN_BLOCKS : 2) : KMAX == 16 ? 2 : KMAX == 4 ? 3 : 4;
+}
+template <int KMAX, bool SPECIAL>
+__host__ __device__ constexpr int fwd_min_blocks() {
+  return fwd_blocks_of_256<KMAX, SPECIAL>() * (256 / kFwdThreads);
 }
 
 // Each warp owns a contiguous span of 32 * U output vectors (8 values each);
@@ -351,7 +359,7 @@ __global__ void __launch_bounds__(256) row_scale_kernel(const uint4* __restrict_
 // a pair also holds its (scale, reciprocal); every lane fetches them by
 // shuffle when the pair's turn comes, so no per-pair array is kept.
 template <typename T16, int KMAX>
-__global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, false>() - 1))
+__global__ void __launch_bounds__(kFwdThreads, (fwd_blocks_of_256<KMAX, false>() - 1) * (256 / kFwdThreads))
     combine_fwd_rt_kernel(CombineArgs a, const float2* __restrict__ rscale) {
   constexpr int U = fwd_vectors_per_thread<KMAX>();
   pdl_trigger();
