@@ -154,9 +154,15 @@ __host__ __device__ constexpr int fwd_min_blocks() {
 // lane takes its token's metadata by shuffle. (Narrower rows: every thread
 // classifies its own token's pairs.) Every row a pair reads is loaded in one
 // batch before the sum in ascending k.
-template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool WARP_META>
-__global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>()))
-    combine_fwd_kernel(CombineArgs a) {
+// The rows of one warp span, from its pairs' kinds, rows and weights: every
+// row a pair reads is loaded in one batch, then summed in ascending k and
+// stored. SPECIAL: the pairs may be zero, copy or const experts.
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
+__device__ __forceinline__ void gather_span(const CombineArgs& a, int span, int V, int n,
+                                            int lane, int (&kind)[fwd_vectors_per_thread<KMAX>()][KMAX],
+                                            const int (&row)[fwd_vectors_per_thread<KMAX>()][KMAX],
+                                            float (&wt)[fwd_vectors_per_thread<KMAX>()][KMAX],
+                                            const int (&col)[fwd_vectors_per_thread<KMAX>()]) {
   constexpr int U = fwd_vectors_per_thread<KMAX>();
   // the branch-free sum (below) where it measured faster: unit weights (DSv3-shaped
   // dispatch backward 87.7 -> 87.3 us, Mixtral-shaped 65.9 -> 62.5) and K > 4
@@ -164,74 +170,8 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
   // special experts (64.9 -> 66.9) and for the weighted K <= 4 gather (Mixtral
   // combine 67.9 -> 86.5)
   constexpr bool BRANCHFREE = UNIT || (!SPECIAL && KMAX > 4);
-  pdl_trigger();
-  pdl_wait();
-  const int V = a.H / kVecElems;
-  const int K = a.K;
-  const int n = a.bs * V;
-  const int lane = threadIdx.x & 31;
-  const int span = blockIdx.x * (kFwdThreads * U) + (threadIdx.x >> 5) * (32 * U);
-  if (span >= n) return;  // warp-uniform
   const uint4* Y = static_cast<const uint4*>(a.expand_x);
   uint4 val[U][KMAX];
-  int kind[U][KMAX], row[U][KMAX];
-  float wt[U][KMAX];
-  int col[U];  // each vector's column in its row (one division per span)
-  if (WARP_META) {  // the launcher picks WARP_META only when V >= 32 * U
-    const int t0 = span / V;
-    const int v0 = span - t0 * V;
-    const int tm = t0 + (lane >> 4), km = lane & 15;
-    const bool mine = km < K && tm < a.bs;
-    PairMeta m{kSkip, 0, 1.0f};
-    if (mine) m = classify_pair<SPECIAL, UNIT, false, true>(a, tm, km);
-    if (SPECIAL) {
-      // a repeat of an id held by an earlier lane of the same token takes no part
-      const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
-      bool dup = false;
-#pragma unroll
-      for (int jj = 0; jj < KMAX - 1; ++jj) {  // km < K <= KMAX
-        const int other = __shfl_sync(0xFFFFFFFFu, id, (lane & 16) | jj);
-        dup |= jj < km && other == id;
-      }
-      if (dup) m.kind = kSkip;
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int item = span + u * 32 + lane;
-      // the span's first token, or the next one past its end (V >= 32 * U: at
-      // most one wrap)
-      int src_base = 0;
-      col[u] = v0 + u * 32 + lane;
-      if (col[u] >= V) {
-        col[u] -= V;
-        src_base = 16;
-      }
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        kind[u][j] = __shfl_sync(0xFFFFFFFFu, m.kind, src_base + j);
-        row[u][j] = __shfl_sync(0xFFFFFFFFu, m.row, src_base + j);
-        wt[u][j] = UNIT ? 1.0f : __shfl_sync(0xFFFFFFFFu, m.w, src_base + j);
-        if (j >= K || item >= n) kind[u][j] = kSkip;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int item = span + u * 32 + lane;
-      const int t = item / V;
-      col[u] = item - t * V;
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        kind[u][j] = kSkip;
-        wt[u][j] = 1.0f;
-        if (j >= K || item >= n) continue;
-        const PairMeta m = classify_pair<SPECIAL, UNIT, true, true>(a, t, j);
-        kind[u][j] = m.kind;
-        row[u][j] = m.row;
-        wt[u][j] = m.w;
-      }
-    }
-  }
   // every row a pair reads (a routed row, or the ori_x row of a copy / const
   // pair) is loaded in one batch, before any is used
   const uint4* ORI = static_cast<const uint4*>(a.ori_x);
@@ -316,6 +256,103 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
     }
     st_v4(static_cast<uint4*>(a.out) + item, narrow8<T16>(acc));
   }
+}
+
+
+// Shuffles the classifying lanes' pair metadata to every lane of the span
+// (lanes 0..15: the span's first token, 16..31: the next one).
+template <int KMAX, bool UNIT>
+__device__ __forceinline__ void spread_meta(const PairMeta& m, int span, int v0, int V, int K,
+                                            int n, int lane,
+                                            int (&kind)[fwd_vectors_per_thread<KMAX>()][KMAX],
+                                            int (&row)[fwd_vectors_per_thread<KMAX>()][KMAX],
+                                            float (&wt)[fwd_vectors_per_thread<KMAX>()][KMAX],
+                                            int (&col)[fwd_vectors_per_thread<KMAX>()]) {
+  constexpr int U = fwd_vectors_per_thread<KMAX>();
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int item = span + u * 32 + lane;
+    // the span's first token, or the next one past its end (V >= 32 * U: at
+    // most one wrap)
+    int src_base = 0;
+    col[u] = v0 + u * 32 + lane;
+    if (col[u] >= V) {
+      col[u] -= V;
+      src_base = 16;
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      kind[u][j] = __shfl_sync(0xFFFFFFFFu, m.kind, src_base + j);
+      row[u][j] = __shfl_sync(0xFFFFFFFFu, m.row, src_base + j);
+      wt[u][j] = UNIT ? 1.0f : __shfl_sync(0xFFFFFFFFu, m.w, src_base + j);
+      if (j >= K || item >= n) kind[u][j] = kSkip;
+    }
+  }
+}
+
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool WARP_META>
+__global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>()))
+    combine_fwd_kernel(CombineArgs a) {
+  constexpr int U = fwd_vectors_per_thread<KMAX>();
+  pdl_trigger();
+  pdl_wait();
+  const int V = a.H / kVecElems;
+  const int K = a.K;
+  const int n = a.bs * V;
+  const int lane = threadIdx.x & 31;
+  const int span = blockIdx.x * (kFwdThreads * U) + (threadIdx.x >> 5) * (32 * U);
+  if (span >= n) return;  // warp-uniform
+  int kind[U][KMAX], row[U][KMAX];
+  float wt[U][KMAX];
+  int col[U];  // each vector's column in its row (one division per span)
+  if (WARP_META) {  // the launcher picks WARP_META only when V >= 32 * U
+    const int t0 = span / V;
+    const int v0 = span - t0 * V;
+    const int tm = t0 + (lane >> 4), km = lane & 15;
+    const bool mine = km < K && tm < a.bs;
+    PairMeta m{kSkip, 0, 1.0f};
+    if (mine) m = classify_pair<SPECIAL, UNIT, false, true>(a, tm, km);
+    if (SPECIAL) {
+      // a span whose tokens have routed (or skipped) pairs only takes the plain
+      // gather (warp-uniform): a repeated routed id already has no slot, so the
+      // repeat check is needed only where special ids are present
+      const bool plain = !__any_sync(0xFFFFFFFFu, (m.kind & 7) >= kZero);
+      if (plain) {
+        spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
+        gather_span<T16, KMAX, false, UNIT>(a, span, V, n, lane, kind, row, wt, col);
+        return;
+      }
+      // a repeat of an id held by an earlier lane of the same token takes no part
+      const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
+      bool dup = false;
+#pragma unroll
+      for (int jj = 0; jj < KMAX - 1; ++jj) {  // km < K <= KMAX
+        const int other = __shfl_sync(0xFFFFFFFFu, id, (lane & 16) | jj);
+        dup |= jj < km && other == id;
+      }
+      if (dup) m.kind = kSkip;
+    }
+    spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
+  } else {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = span + u * 32 + lane;
+      const int t = item / V;
+      col[u] = item - t * V;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        kind[u][j] = kSkip;
+        row[u][j] = 0;
+        wt[u][j] = 1.0f;
+        if (j >= K || item >= n) continue;
+        const PairMeta m = classify_pair<SPECIAL, UNIT, true, true>(a, t, j);
+        kind[u][j] = m.kind;
+        row[u][j] = m.row;
+        wt[u][j] = m.w;
+      }
+    }
+  }
+  gather_span<T16, KMAX, SPECIAL, UNIT>(a, span, V, n, lane, kind, row, wt, col);
 }
 
 // ---------------------------------------------------------------------------
