@@ -179,8 +179,10 @@ __device__ __forceinline__ void gather_span(const CombineArgs& a, int span, int 
     // A sum that starts at +0 never becomes -0 (x + y is -0 only when both
     // are), so adding w * 0 never changes it: a skipped pair reads a vector of
     // zeros with weight 0 (its product is 0 whatever the weight held) and is
-    // summed like the others, without a branch per pair.
-    static_assert(!SPECIAL, "routed and skipped pairs only");
+    // summed like the others, without a branch per pair. A zero-expert pair
+    // (the special-expert kernel's plain spans) reads the zeros with its own
+    // weight: its term w * 0 is the oracle's.
+    static_assert(!SPECIAL, "routed, zero-expert and skipped pairs only");
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int v = col[u];
@@ -189,7 +191,7 @@ __device__ __forceinline__ void gather_span(const CombineArgs& a, int span, int 
         const bool routed = kind[u][j] == kRouted;
         val[u][j] = ld_nc_v4(routed ? Y + static_cast<size_t>(row[u][j]) * V + v
                                     : g_zero_vecs + (v & (kZeroVecs - 1)));
-        if (!routed) wt[u][j] = 0.0f;
+        if (kind[u][j] == kSkip) wt[u][j] = 0.0f;
       }
     }
   } else {
@@ -313,26 +315,35 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
     PairMeta m{kSkip, 0, 1.0f};
     if (mine) m = classify_pair<SPECIAL, UNIT, false, true>(a, tm, km);
     if (SPECIAL) {
-      // a span whose tokens have routed (or skipped) pairs only takes the plain
-      // gather (warp-uniform): a repeated routed id already has no slot, so the
-      // repeat check is needed only where special ids are present
-      const bool plain = !__any_sync(0xFFFFFFFFu, (m.kind & 7) >= kZero);
+      // A span whose tokens have no copy or const pair takes the plain gather
+      // (warp-uniform): with routed (or skipped) pairs only for any K, and with
+      // zero-expert pairs too where the plain gather is branch-free (K > 4),
+      // which sums them as zero vectors with their weights. A repeated routed
+      // id already has no slot, so the repeat check is needed only where
+      // special ids are present.
+      const int kd = m.kind & 7;
+      const bool any_special = __any_sync(0xFFFFFFFFu, kd >= kZero);
+      if (any_special) {
+        // a repeat of an id held by an earlier lane of the same token takes no part
+        const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
+        bool dup = false;
+#pragma unroll
+        for (int jj = 0; jj < KMAX - 1; ++jj) {  // km < K <= KMAX
+          const int other = __shfl_sync(0xFFFFFFFFu, id, (lane & 16) | jj);
+          dup |= jj < km && other == id;
+        }
+        if (dup) m.kind = kSkip;
+      }
+      const bool plain = KMAX > 4 ? !__any_sync(0xFFFFFFFFu, kd == kCopy || kd == kConst)
+                                  : !any_special;
+      spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
       if (plain) {
-        spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
         gather_span<T16, KMAX, false, UNIT>(a, span, V, n, lane, kind, row, wt, col);
         return;
       }
-      // a repeat of an id held by an earlier lane of the same token takes no part
-      const int id = mine ? __ldg(a.topk_idx + static_cast<size_t>(tm) * K + km) : -1;
-      bool dup = false;
-#pragma unroll
-      for (int jj = 0; jj < KMAX - 1; ++jj) {  // km < K <= KMAX
-        const int other = __shfl_sync(0xFFFFFFFFu, id, (lane & 16) | jj);
-        dup |= jj < km && other == id;
-      }
-      if (dup) m.kind = kSkip;
+    } else {
+      spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
     }
-    spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
   } else {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
