@@ -157,7 +157,7 @@ __host__ __device__ constexpr int fwd_min_blocks() {
 // The rows of one warp span, from its pairs' kinds, rows and weights: every
 // row a pair reads is loaded in one batch, then summed in ascending k and
 // stored. SPECIAL: the pairs may be zero, copy or const experts.
-template <typename T16, int KMAX, bool SPECIAL, bool UNIT>
+template <typename T16, int KMAX, bool SPECIAL, bool UNIT, bool COPY = false>
 __device__ __forceinline__ void gather_span(const CombineArgs& a, int span, int V, int n,
                                             int lane, int (&kind)[fwd_vectors_per_thread<KMAX>()][KMAX],
                                             const int (&row)[fwd_vectors_per_thread<KMAX>()][KMAX],
@@ -179,19 +179,22 @@ __device__ __forceinline__ void gather_span(const CombineArgs& a, int span, int 
     // A sum that starts at +0 never becomes -0 (x + y is -0 only when both
     // are), so adding w * 0 never changes it: a skipped pair reads a vector of
     // zeros with weight 0 (its product is 0 whatever the weight held) and is
-    // summed like the others, without a branch per pair. A zero-expert pair
-    // (the special-expert kernel's plain spans) reads the zeros with its own
-    // weight: its term w * 0 is the oracle's.
-    static_assert(!SPECIAL, "routed, zero-expert and skipped pairs only");
+    // summed like the others, without a branch per pair. In the special-expert
+    // kernel's plain spans a zero-expert pair reads the zeros with its own
+    // weight (its term w * 0 is the oracle's) and, with COPY, a copy pair reads
+    // its token's ori_x row like a routed row.
+    static_assert(!SPECIAL, "routed, copy, zero-expert and skipped pairs only");
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int v = col[u];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
-        const bool routed = kind[u][j] == kRouted;
-        val[u][j] = ld_nc_v4(routed ? Y + static_cast<size_t>(row[u][j]) * V + v
-                                    : g_zero_vecs + (v & (kZeroVecs - 1)));
-        if (kind[u][j] == kSkip) wt[u][j] = 0.0f;
+        const int kd = kind[u][j];
+        const uint4* src = g_zero_vecs + (v & (kZeroVecs - 1));
+        if (kd == kRouted) src = Y + static_cast<size_t>(row[u][j]) * V + v;
+        if (COPY && kd == kCopy) src = ORI + static_cast<size_t>(row[u][j]) * V + v;
+        val[u][j] = ld_nc_v4(src);
+        if (kd == kSkip) wt[u][j] = 0.0f;
       }
     }
   } else {
@@ -315,12 +318,12 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
     PairMeta m{kSkip, 0, 1.0f};
     if (mine) m = classify_pair<SPECIAL, UNIT, false, true>(a, tm, km);
     if (SPECIAL) {
-      // A span whose tokens have no copy or const pair takes the plain gather
+      // A span whose tokens have no const pair takes the plain gather
       // (warp-uniform): with routed (or skipped) pairs only for any K, and with
-      // zero-expert pairs too where the plain gather is branch-free (K > 4),
-      // which sums them as zero vectors with their weights. A repeated routed
-      // id already has no slot, so the repeat check is needed only where
-      // special ids are present.
+      // zero-expert and copy pairs too where the plain gather is branch-free
+      // (K > 4), which sums them as zero vectors or ori_x rows with their
+      // weights. A repeated routed id already has no slot, so the repeat check
+      // is needed only where special ids are present.
       const int kd = m.kind & 7;
       const bool any_special = __any_sync(0xFFFFFFFFu, kd >= kZero);
       if (any_special) {
@@ -334,11 +337,10 @@ __global__ void __launch_bounds__(kFwdThreads, (fwd_min_blocks<KMAX, SPECIAL>())
         }
         if (dup) m.kind = kSkip;
       }
-      const bool plain = KMAX > 4 ? !__any_sync(0xFFFFFFFFu, kd == kCopy || kd == kConst)
-                                  : !any_special;
+      const bool plain = KMAX > 4 ? !__any_sync(0xFFFFFFFFu, kd == kConst) : !any_special;
       spread_meta<KMAX, UNIT>(m, span, v0, V, K, n, lane, kind, row, wt, col);
       if (plain) {
-        gather_span<T16, KMAX, false, UNIT>(a, span, V, n, lane, kind, row, wt, col);
+        gather_span<T16, KMAX, false, UNIT, true>(a, span, V, n, lane, kind, row, wt, col);
         return;
       }
     } else {
