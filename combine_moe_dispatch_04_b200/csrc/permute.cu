@@ -75,7 +75,11 @@ template <typename T16, int CPT>
 __global__ void __launch_bounds__(256) permute_quant_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ assist, uint4* __restrict__ out,
     float* __restrict__ scales, int bs, int K, int H, int A) {
-  __shared__ float warp_max[8];
+  // per-warp maxima, two sets used alternately: a warp writes set p for the next
+  // token only after that token's barrier, which every warp reaches after
+  // reading this token's set, so one barrier per token suffices
+  __shared__ float warp_max[2][8];
+  int par = 0;
   pdl_trigger();
   pdl_wait();
   const int C = H / 16;  // chunks per row
@@ -125,11 +129,11 @@ __global__ void __launch_bounds__(256) permute_quant_kernel(
     }
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
-    if (lane == 0) warp_max[warp] = amax;
+    if (lane == 0) warp_max[par][warp] = amax;
     __syncthreads();
-    amax = warp_max[0];
-    for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, warp_max[w]);
-    __syncthreads();  // warp_max is reused by the next token
+    amax = warp_max[par][0];
+    for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, warp_max[par][w]);
+    par ^= 1;
     const float scale = __fdiv_rn(amax, 127.0f);
     const float inv_scale = 1.0f / scale;
 #pragma unroll
@@ -547,22 +551,24 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   }
   int threads, cpt;
   quant_shape(a.H, &threads, &cpt);
-  const int cap = sm_count() * (2048 / threads);
-  const int blocks = a.bs < cap ? a.bs : cap;
   const uint4* x = static_cast<const uint4*>(a.x);
   uint4* out = static_cast<uint4*>(a.expand_x);
   const bool bf = a.dtype == MOE_BF16;
-  if (cpt <= 1)
-    return launch_pdl(bf ? permute_quant_kernel<Bf16, 1> : permute_quant_kernel<Fp16, 1>,
-                      dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales, a.bs, a.K,
-                      a.H, a.A);
-  if (cpt <= 2)
-    return launch_pdl(bf ? permute_quant_kernel<Bf16, 2> : permute_quant_kernel<Fp16, 2>,
-                      dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales, a.bs, a.K,
-                      a.H, a.A);
-  return launch_pdl(bf ? permute_quant_kernel<Bf16, 4> : permute_quant_kernel<Fp16, 4>,
-                    dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales, a.bs, a.K,
-                    a.H, a.A);
+  // a persistent grid of as many CTAs as are resident at once (each walks its
+  // tokens with the next row in flight), so no partial second wave
+  auto launch = [&](auto kernel) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    const int cap = sm_count() * per_sm;
+    const int blocks = a.bs < cap ? a.bs : cap;
+    return launch_pdl(kernel, dim3(blocks), dim3(threads), 0, st, x, a.assist, out, a.scales,
+                      a.bs, a.K, a.H, a.A);
+  };
+  if (cpt <= 1) return launch(bf ? permute_quant_kernel<Bf16, 1> : permute_quant_kernel<Fp16, 1>);
+  if (cpt <= 2) return launch(bf ? permute_quant_kernel<Bf16, 2> : permute_quant_kernel<Fp16, 2>);
+  return launch(bf ? permute_quant_kernel<Bf16, 4> : permute_quant_kernel<Fp16, 4>);
 }
 
 }  // namespace moe
